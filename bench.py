@@ -1,0 +1,413 @@
+"""Decode-step benchmark: paged decode attention seq-steps/s and KV-read GB/s.
+
+One step = one pass of the whole hot path on one batch of synthetic input:
+copy_blocks (copy-on-write pairs, when the workload has them) ->
+reshape_and_cache (one new token per sequence) -> paged_attention_decode.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload cfg2]
+    python bench.py --impl reference ...     # the fp64 CPU oracle, bounded sample
+
+Multi-GPU (torchrun): every rank runs its own batch of the same workload
+(sequences are independent; no data-path collective) -> weak scaling; the
+time is the max over ranks.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention seq-steps/s and KV-read HBM GB/s (% of B200 peak)"
+L2_BYTES = 126 * 1024 * 1024
+WORKLOADS = {"cfg1": 1, "cfg2": 2, "cfg3": 3, "cfg4": 4, "cfg5": 5}
+
+
+# ---------------------------------------------------------------- distributed
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Each rank draws its own batch (weak scaling): seed offset per rank."""
+    return 1000 * rank
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max over ranks of a timing (a timing reduction, not a data-path exchange)."""
+    if world <= 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- workload
+def make_workload(name: str, rank: int):
+    from paged_kv_cache_373_b200 import workloads as W
+    cfg = WORKLOADS[name]
+    wl = W.make_config(cfg)
+    if rank:
+        # a different, equally shaped batch per rank
+        import math
+        if cfg == 5:
+            wl = W.config5()
+        else:
+            gen = torch.Generator().manual_seed(W._seed(cfg) * 1000 + rank_seed_offset(rank))
+            lens = wl.seq_lens.tolist()
+            perm = torch.randperm(len(lens), generator=gen).tolist()
+            lens = [lens[i] for i in perm]
+            wl = W.build_decode(wl.name, lens, wl.num_heads, wl.num_kv_heads, wl.head_dim,
+                                wl.block_size, wl.kv_dtype, wl.q_dtype,
+                                W._seed(cfg) + rank_seed_offset(rank),
+                                num_blocks=wl.num_blocks, scale=wl.scale)
+    return wl
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def recorded_traffic(workload: str):
+    """dram read+write bytes per attention launch from a committed ncu summary
+    (profiles/traffic.json), or None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    return d.get(workload)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for ln in f:
+                parts = [x.strip() for x in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle leg
+class OracleSample:
+    """The oracle (as it stands) timed on the first k sequences of the workload,
+    k chosen once so that one call costs about `budget_s` seconds."""
+
+    def __init__(self, wl, budget_s: float, threads: int = 0):
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        import oracle
+        from pkv_testutil import oracle_caches
+        self.oracle, self.wl = oracle, wl
+        self.cores = threads or oracle.num_threads_available()
+        kmax = wl.num_seqs if not wl.is_fp8 else min(wl.num_seqs, 64)
+        self.kc, self.vc = oracle_caches(wl, None if not wl.is_fp8 else list(range(kmax)))
+        k = 1
+        while True:
+            dt = self.time(k)
+            if dt >= budget_s / 2 or k >= kmax:
+                break
+            k = min(kmax, max(k + 1, int(k * min(8.0, budget_s / max(dt, 1e-4)))))
+        self.k = k
+
+    def time(self, k: int) -> float:
+        wl = self.wl
+        t0 = time.perf_counter()
+        self.oracle.paged_attention_decode(wl.query, self.kc, self.vc, wl.block_tables, wl.seq_lens,
+                                           wl.scale, wl.k_scale, wl.v_scale,
+                                           seq_subset=list(range(k)), num_threads=self.cores)
+        return time.perf_counter() - t0
+
+    def rate(self) -> float:
+        return self.k / self.time(self.k)
+
+
+def run_reference(args):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return 0
+    wl = make_workload(args.workload, 0)
+    # each step is a bounded sample so the whole run stays within a few minutes
+    smp = OracleSample(wl, budget_s=max(0.5, min(args.ref_budget, 120.0 / max(1, args.steps))))
+    rates = [smp.rate() for _ in range(args.steps)]
+    k_used, cores = smp.k, smp.cores
+    value = statistics.median(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "seq-steps/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * wl.num_seqs / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "num_seqs": wl.num_seqs},
+        "cpu_baseline": {"value": value, "unit": "seq-steps/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first {k_used} of {wl.num_seqs} sequences per step, fp64 C oracle"},
+        "e2e": {"value": value, "unit": "seq-steps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------- GPU leg
+def run_ours(args):
+    import paged_kv_cache_373_b200 as pkv
+    from paged_kv_cache_373_b200 import _build
+    _build.build()
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = make_workload(args.workload, rank)
+
+    # ---- resident device state
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from pkv_testutil import gpu_inputs
+    g = gpu_inputs(wl, dev)
+    pristine = None
+    out = torch.empty_like(g["q"])
+    ws = pkv.alloc_workspace(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim,
+                             args.num_ctas, device=dev)
+    has_pairs = g["pairs"].numel() > 0
+    stream = torch.cuda.current_stream()
+    kv_bytes = (wl.num_blocks * wl.block_size * wl.num_kv_heads * wl.head_dim *
+                wl.kv_elem_bytes() * 2)
+    flush = kv_bytes < 2 * L2_BYTES
+    scratch = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if flush else None
+
+    def step(ev_a0=None, ev_a1=None):
+        if has_pairs:
+            pkv.copy_blocks([g["kc"]], [g["vc"]], g["pairs"])
+        pkv.reshape_and_cache(g["nk"], g["nv"], g["kc"], g["vc"], g["slots"], g["ks"], g["vs"])
+        if ev_a0 is not None:
+            ev_a0.record(stream)
+        pkv.paged_attention_decode(out, g["q"], g["kc"], g["vc"], g["tables"], g["lens"], wl.scale,
+                                   g["ks"], g["vs"], workspace=ws, num_ctas=args.num_ctas)
+        if ev_a1 is not None:
+            ev_a1.record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if pkv.get_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(K):
+            if flush:
+                scratch.fill_(i & 0xff)     # evict the small workload from L2 (outside the step events)
+            ev[i][0].record(stream)
+            step(ev[i][1], ev[i][2])
+            ev[i][3].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    step_ms = [a.elapsed_time(d) for a, _, _, d in ev]
+    attn_ms = [b.elapsed_time(c) for _, b, c, _ in ev]
+    total_ms = sum(step_ms) if flush else t_start.elapsed_time(t_end)
+    total_ms = reduce_max(total_ms, world, dev)
+    if pkv.get_device_error() != 0:
+        raise RuntimeError("device error during the timed steps")
+
+    ms_per_step = total_ms / K
+    value = world * wl.num_seqs / (ms_per_step / 1000.0)
+    attn_avg_ms = statistics.mean(attn_ms)
+    b_alg = wl.algorithmic_bytes()
+    peak, peak_kind = measured_peaks()
+    achieved = b_alg / (attn_avg_ms / 1000.0) / 1e9
+
+    # ---- end-to-end through the C ABI with host buffers
+    e2e = e2e_leg(pkv, wl, g, ws, args, dev) if not args.no_e2e else None
+    e2e_value = reduce_max(e2e["ms"], world, dev) if e2e else None
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        smp = OracleSample(wl, budget_s=args.ref_budget)
+        r = smp.rate()
+        cpu = {"value": r, "unit": "seq-steps/s", "cores": smp.cores, "kind": "oracle",
+               "sample": f"first {smp.k} of {wl.num_seqs} sequences of the same workload, "
+                         f"fp64 C oracle, {smp.cores} OpenMP threads"}
+
+    launches_per_step = (1 if has_pairs else 0) + 1 + 2
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "seq-steps/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": {True: "fp8_e4m3 kv / fp32 accum", False: str(wl.kv_dtype).replace("torch.", "")
+                      + " kv / fp32 accum"}[wl.is_fp8],
+            "data": "synthetic",
+            "config": {"workload": wl.name, "num_seqs": wl.num_seqs, "num_heads": wl.num_heads,
+                       "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                       "block_size": wl.block_size, "num_blocks": wl.num_blocks,
+                       "max_seq_len": wl.max_seq_len, "cow_pairs": int(wl.cow_pairs.shape[0]),
+                       "kv_bytes_alg": b_alg,
+                       "l2": "flushed between steps" if flush else "inputs larger than L2 (126 MB)",
+                       "parallelism": f"replicas x{world} (independent batches)"},
+            "attention_ms": attn_avg_ms,
+            "kv_read_gbs": achieved,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
+                         "traffic": recorded_traffic(wl.name)},
+            "clocks": clk.summary(),
+            "gpu_launches": launches_per_step * K,
+            "e2e": None if e2e is None else {
+                "value": world * wl.num_seqs / (e2e_value / 1000.0), "unit": "seq-steps/s",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def e2e_leg(pkv, wl, g, ws, args, dev):
+    """decode_step_host: pinned host inputs -> H2D -> step -> D2H -> sync."""
+    pin = lambda t: t.contiguous().pin_memory()
+    h = dict(q=pin(wl.query), nk=pin(wl.new_key.to(wl.q_dtype)), nv=pin(wl.new_value.to(wl.q_dtype)),
+             slots=pin(wl.slot_mapping), tables=pin(wl.block_tables), lens=pin(wl.seq_lens),
+             pairs=pin(wl.cow_pairs), out=torch.empty_like(wl.query).pin_memory())
+    d = dict(q=torch.empty_like(g["q"]), nk=torch.empty_like(g["nk"]), nv=torch.empty_like(g["nv"]),
+             slots=torch.empty_like(g["slots"]), tables=torch.empty_like(g["tables"]),
+             lens=torch.empty_like(g["lens"]), pairs=torch.empty_like(g["pairs"]),
+             out=torch.empty_like(g["q"]))
+    a = pkv.DecodeStepArgs()
+    a.num_seqs, a.num_heads, a.num_kv_heads = wl.num_seqs, wl.num_heads, wl.num_kv_heads
+    a.head_dim, a.block_size, a.max_blocks_per_seq = wl.head_dim, wl.block_size, wl.max_blocks_per_seq
+    a.num_blocks = wl.num_blocks
+    a.q_dtype = pkv.dtype_code(wl.query)
+    a.cache_dtype = pkv.PKV_FP8_E4M3 if wl.is_fp8 else pkv.dtype_code(wl.query)
+    a.scale, a.num_ctas = wl.scale, args.num_ctas
+    a.h_query, a.h_new_key, a.h_new_value = h["q"].data_ptr(), h["nk"].data_ptr(), h["nv"].data_ptr()
+    a.h_slot_mapping, a.h_block_tables = h["slots"].data_ptr(), h["tables"].data_ptr()
+    a.h_seq_lens, a.h_out = h["lens"].data_ptr(), h["out"].data_ptr()
+    a.num_cow_pairs = int(wl.cow_pairs.shape[0])
+    a.h_cow_pairs = h["pairs"].data_ptr() if a.num_cow_pairs else None
+    a.d_query, a.d_new_key, a.d_new_value = d["q"].data_ptr(), d["nk"].data_ptr(), d["nv"].data_ptr()
+    a.d_slot_mapping, a.d_block_tables = d["slots"].data_ptr(), d["tables"].data_ptr()
+    a.d_seq_lens, a.d_out = d["lens"].data_ptr(), d["out"].data_ptr()
+    a.d_cow_pairs = d["pairs"].data_ptr() if a.num_cow_pairs else None
+    a.key_cache, a.value_cache = g["kc"].data_ptr(), g["vc"].data_ptr()
+    a.k_scale = g["ks"].data_ptr() if g["ks"] is not None else None
+    a.v_scale = g["vs"].data_ptr() if g["vs"] is not None else None
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        pkv.decode_step_host(a, stream)
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(K):
+        pkv.decode_step_host(a, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    h2d = sum(h[k].numel() * h[k].element_size() for k in ("q", "nk", "nv", "slots", "tables", "lens"))
+    h2d += h["pairs"].numel() * 8
+    d2h = h["out"].numel() * h["out"].element_size()
+    return {"ms": e0.elapsed_time(e1) / K, "h2d": h2d, "d2h": d2h}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="cfg2", choices=sorted(WORKLOADS))
+    ap.add_argument("--num-ctas", type=int, default=0)
+    ap.add_argument("--ref-budget", type=float, default=15.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    return run_reference(args) if args.impl == "reference" else run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

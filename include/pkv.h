@@ -1,0 +1,239 @@
+/*
+ * pkv.h -- C ABI of the B200 (sm_100a) paged KV-cache decode library.
+ *
+ * The KV cache of one attention layer is a pool of fixed-size physical
+ * blocks; each sequence reaches its blocks through a per-sequence block table
+ * (zwxr.cn/news/121728 "PagedAttention 与 Continuous Batching", sections 3.1
+ * and 3.2).  This library implements the device side of one decode step:
+ *
+ *   pkv_copy_blocks            copy-on-write copies of shared blocks (3.4)
+ *   pkv_reshape_and_cache      write each new token's K/V into its slot (3.1)
+ *   pkv_paged_attention_decode single-token attention through the block
+ *                              table with the block-wise softmax merge (3.3)
+ *
+ * Conventions for every call
+ *   - The caller owns all memory.  Pointers named d_* or documented as
+ *     "device" are CUDA device pointers; "host" pointers are CPU memory.
+ *     The library allocates nothing (its only device state is a static
+ *     error word).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) except pkv_get_device_error and pkv_decode_step_host,
+ *     which synchronise it.
+ *   - Arguments are validated on the host before any launch: a bad argument
+ *     returns PKV_EINVAL, a valid but unimplemented combination
+ *     PKV_EUNSUPPORTED, and nothing is launched.  A CUDA launch/copy failure
+ *     returns PKV_ECUDA.
+ *   - Data-dependent faults (a block id outside [0, num_blocks), a slot past
+ *     the pool, a seq_len longer than its table row) are detected on the
+ *     device: the offending access is skipped or clamped to block 0, the
+ *     result is unspecified, and a bit is OR-ed into the device error word
+ *     that pkv_get_device_error returns.  Nothing traps.
+ *   - Thread safety: calls on different streams may run concurrently; calls
+ *     that share a workspace must be ordered by the caller.
+ *
+ * Layouts (row-major, innermost last):
+ *   query, out        [num_seqs, num_heads, head_dim]           q dtype
+ *   new key/value     [num_tokens, num_kv_heads, head_dim]      source dtype
+ *   key/value cache   [num_blocks, block_size, num_kv_heads, head_dim]
+ *   block_tables      int32 [num_seqs, max_blocks_per_seq]
+ *   seq_lens          int32 [num_seqs]
+ *   slot_mapping      int64 [num_tokens]
+ *   block_mapping     int64 [num_pairs, 2]  (src, dst)
+ * GQA: q head h reads kv head h / (num_heads / num_kv_heads).
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* pkv_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    PKV_F32 = 0,
+    PKV_F16 = 1,
+    PKV_BF16 = 2,
+    PKV_FP8_E4M3 = 3 /* OCP E4M3 "fn": max 448, no inf, S.1111.111 = NaN */
+} pkv_dtype;
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_EINVAL = 1,       /* bad argument (null pointer, bad shape, bad alignment) */
+    PKV_EUNSUPPORTED = 2, /* valid but not implemented (e.g. head_dim 96) */
+    PKV_ECUDA = 3,        /* a CUDA runtime call failed */
+    PKV_EDEVICE = 4       /* the device error word is non-zero */
+} pkv_status;
+
+/* Bits of the device error word. */
+#define PKV_DEVERR_BLOCK_ID 0x1   /* block table entry outside [0, num_blocks) */
+#define PKV_DEVERR_SLOT     0x2   /* slot_mapping entry >= num_blocks * block_size */
+#define PKV_DEVERR_SEQ_LEN  0x4   /* seq_len < 0 or > max_blocks_per_seq * block_size */
+#define PKV_DEVERR_COPY_ID  0x8   /* copy_blocks src/dst outside [0, num_blocks) */
+#define PKV_DEVERR_TIMEOUT  0x10  /* a pipeline wait gave up (about 2 s); results invalid */
+
+/*
+ * pkv_reshape_and_cache -- store the K/V of new tokens in their cache slots.
+ * zwxr.cn section 3.1: a token occupies a slot once it is produced; the slot
+ * is physical_block * block_size + offset (section 3.2).
+ *
+ * For i in [0, num_tokens) with s = slot_mapping[i]:
+ *   s < 0                     : token i is padding, skipped;
+ *   s >= num_blocks*block_size: skipped, PKV_DEVERR_SLOT;
+ *   else key_cache[s / block_size, s % block_size, :, :] = key[i, :, :]
+ *        (same for value).
+ * cache_dtype == src_dtype  : a bit-exact copy (f32, f16 or bf16).
+ * cache_dtype == FP8_E4M3   : src_dtype in {f32, f16, bf16}; each element is
+ *   stored as round-to-nearest-even, saturating E4M3 of the IEEE fp32
+ *   quotient x / *k_scale (resp. *v_scale); NaN stays NaN.  k_scale and
+ *   v_scale are device pointers to one fp32 each, required for FP8 and
+ *   ignored otherwise.
+ * key, value, key_cache, value_cache must be 16-byte aligned.
+ * head_dim in {64, 128}; block_size > 0; num_kv_heads > 0.
+ */
+pkv_status pkv_reshape_and_cache(const void* key, const void* value, pkv_dtype src_dtype,
+                                 void* key_cache, void* value_cache, pkv_dtype cache_dtype,
+                                 const int64_t* slot_mapping, int64_t num_tokens,
+                                 int64_t num_blocks, int block_size, int num_kv_heads,
+                                 int head_dim, const float* k_scale, const float* v_scale,
+                                 pkv_stream_t stream);
+
+/*
+ * pkv_copy_blocks -- copy-on-write duplication of whole physical blocks.
+ * zwxr.cn section 3.4 / ttlab.hopto.org section 2: shared blocks are
+ * read-only; a sequence about to write into a shared block first copies it.
+ *
+ * For every pair p and every layer l:
+ *   key_caches[l] block block_mapping[p][1] = key_caches[l] block block_mapping[p][0]
+ * (same for value_caches), each block being block_bytes contiguous bytes
+ * (block_size * num_kv_heads * head_dim * element size), unused slots included.
+ * key_caches / value_caches: HOST arrays of num_layers DEVICE pointers
+ * (num_layers in [1, 128]); block_mapping: DEVICE int64 [num_pairs, 2].
+ * block_bytes must be a multiple of 16 and every cache 16-byte aligned.
+ * Destinations must be distinct and disjoint from all sources (otherwise
+ * the result is unspecified).  Ids outside [0, num_blocks) skip the pair
+ * and set PKV_DEVERR_COPY_ID.
+ */
+pkv_status pkv_copy_blocks(void* const* key_caches, void* const* value_caches, int num_layers,
+                           const int64_t* block_mapping, int64_t num_pairs, int64_t num_blocks,
+                           size_t block_bytes, pkv_stream_t stream);
+
+/*
+ * Workspace for pkv_paged_attention_decode: fp32 partial results of the
+ * split sequences, (num_ctas + units) x heads_per_unit x (head_dim + 2)
+ * floats, where units = num_seqs * num_kv_heads * ceil(g / 8) and
+ * g = num_heads / num_kv_heads.  num_ctas = 0 means the default grid of the
+ * current device (pkv_default_num_ctas).  Returns 0 for invalid shapes.
+ * The workspace needs no initialisation.
+ */
+size_t pkv_paged_attention_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
+                                           int head_dim, int num_ctas);
+
+/* Persistent grid size used when num_ctas = 0: one CTA per SM of the
+ * current device (148 on B200).  Returns 0 on error. */
+int pkv_default_num_ctas(void);
+
+/*
+ * pkv_paged_attention_decode -- single-token decode attention over a paged
+ * KV cache.  thinkmoon.cn "PagedAttention不够用了之后" (the paged_attention
+ * pseudocode: gather the sequence's blocks, q.K^T / sqrt(d), softmax, .V)
+ * with zwxr.cn section 3.3 (block-wise softmax: per-block running max m and
+ * normaliser l merged by rescaling, exactly the global softmax).
+ *
+ * For every sequence s (L = seq_lens[s]) and q head h (kv head kh = h / g):
+ *   score_t = scale * <query[s,h,:], K_t>       for t in [0, L)
+ *   out[s,h,:] = sum_t softmax(score)_t * V_t   (L == 0 -> zeros)
+ * where K_t / V_t is row (block_tables[s][t / block_size], t % block_size, kh)
+ * of the caches (times *k_scale / *v_scale for FP8 caches).
+ *
+ * Supported: cache_dtype f32 (q f32), f16 (q f16), bf16 (q bf16),
+ *   FP8_E4M3 (q f16 or bf16, head_dim 128); head_dim in {64, 128};
+ *   block_size in {16, 32}; num_heads % num_kv_heads == 0; any g.
+ * Numerics: fp32 accumulation and fp32 online softmax; for 16-bit and FP8
+ * caches the q.K and P.V products run on tensor cores with 16-bit operands
+ * (P rounded to the cache's 16-bit type, f16 for FP8).  Output is rounded
+ * to the q dtype (RNE).
+ * Long sequences are split across CTAs (balanced over all (sequence, kv head)
+ * work) and their partial (m, l, o) are merged exactly by a second kernel on
+ * the same stream.  Results are bit-identical under any permutation of the
+ * physical block ids and independent of block sharing, for a fixed num_ctas.
+ * workspace: device, >= pkv_paged_attention_workspace_bytes(...) bytes,
+ *   16-byte aligned, contents need no initialisation.
+ * num_ctas: 0 = default; otherwise the persistent grid size (sets the split).
+ * out, query, caches: 16-byte aligned device pointers.
+ */
+pkv_status pkv_paged_attention_decode(void* out, const void* query, pkv_dtype q_dtype,
+                                      const void* key_cache, const void* value_cache,
+                                      pkv_dtype cache_dtype, const int32_t* block_tables,
+                                      int max_blocks_per_seq, const int32_t* seq_lens,
+                                      int num_seqs, int num_heads, int num_kv_heads,
+                                      int head_dim, int block_size, int64_t num_blocks,
+                                      float scale, const float* k_scale, const float* v_scale,
+                                      void* workspace, size_t workspace_bytes, int num_ctas,
+                                      pkv_stream_t stream);
+
+/*
+ * pkv_decode_step_host -- one whole decode step driven from host buffers:
+ * copies the step's inputs host -> device, runs copy_blocks (if
+ * num_cow_pairs > 0), reshape_and_cache of one new token per sequence and
+ * the decode attention, copies the output device -> host and synchronises
+ * the stream.  Host buffers should be pinned for asynchronous copies.
+ * The caches stay resident on the device.  Device staging buffers are
+ * caller-owned and sized like their host counterparts.
+ */
+typedef struct pkv_decode_step_args {
+    /* shapes */
+    int num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq;
+    int64_t num_blocks;
+    pkv_dtype q_dtype;      /* also the dtype of the new K/V rows */
+    pkv_dtype cache_dtype;
+    float scale;
+    int num_ctas;           /* 0 = default */
+    /* host inputs / output */
+    const void* h_query;              /* [S, Hq, D] */
+    const void* h_new_key;            /* [S, Hkv, D] */
+    const void* h_new_value;          /* [S, Hkv, D] */
+    const int64_t* h_slot_mapping;    /* [S] */
+    const int32_t* h_block_tables;    /* [S, max_blocks_per_seq] */
+    const int32_t* h_seq_lens;        /* [S] */
+    const int64_t* h_cow_pairs;       /* [num_cow_pairs, 2] or NULL */
+    int64_t num_cow_pairs;
+    void* h_out;                      /* [S, Hq, D] */
+    /* device staging (same sizes as the host buffers) */
+    void* d_query;
+    void* d_new_key;
+    void* d_new_value;
+    int64_t* d_slot_mapping;
+    int32_t* d_block_tables;
+    int32_t* d_seq_lens;
+    int64_t* d_cow_pairs;
+    void* d_out;
+    /* device state */
+    void* key_cache;
+    void* value_cache;
+    const float* k_scale;             /* device, FP8 only */
+    const float* v_scale;
+    void* workspace;
+    size_t workspace_bytes;
+} pkv_decode_step_args;
+
+pkv_status pkv_decode_step_host(const pkv_decode_step_args* args, pkv_stream_t stream);
+
+/* Synchronise `stream`, return the device error word of the current device
+ * in *code_out and clear it.  Returns PKV_EDEVICE if it was non-zero. */
+pkv_status pkv_get_device_error(int32_t* code_out, pkv_stream_t stream);
+
+/* Static description of a status code. */
+const char* pkv_status_string(pkv_status status);
+
+/* Detail of the last host-side failure on the calling thread ("" if none). */
+const char* pkv_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */

@@ -1,0 +1,202 @@
+"""paged_kv_cache_373_b200 -- B200 (sm_100a) paged KV-cache decode library.
+
+Thin ctypes binding over ``libpkv.so`` (C ABI in include/pkv.h).  Every
+function here only marshals arguments: all work runs in the library's CUDA
+kernels.  There is no CPU fallback; if the library is missing or the tensors
+are not on a CUDA device, the call raises.
+
+Names follow the C entry points without their ``pkv_`` prefix:
+  reshape_and_cache, copy_blocks, paged_attention_decode,
+  paged_attention_workspace_bytes, default_num_ctas, decode_step_host,
+  get_device_error, status_string
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpkv.so")
+
+PKV_F32, PKV_F16, PKV_BF16, PKV_FP8_E4M3 = 0, 1, 2, 3
+PKV_OK, PKV_EINVAL, PKV_EUNSUPPORTED, PKV_ECUDA, PKV_EDEVICE = 0, 1, 2, 3, 4
+DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_SEQ_LEN, DEVERR_COPY_ID, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
+
+_DTYPES = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF16,
+           torch.uint8: PKV_FP8_E4M3, torch.float8_e4m3fn: PKV_FP8_E4M3}
+
+EXPORTED = ("pkv_reshape_and_cache", "pkv_copy_blocks", "pkv_paged_attention_workspace_bytes",
+            "pkv_default_num_ctas", "pkv_paged_attention_decode", "pkv_decode_step_host",
+            "pkv_get_device_error", "pkv_status_string", "pkv_last_error_message")
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"pkv status {status}: {message}")
+        self.status = status
+
+
+class DecodeStepArgs(ctypes.Structure):
+    """Mirror of ``pkv_decode_step_args``."""
+    _fields_ = [
+        ("num_seqs", ctypes.c_int), ("num_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int), ("block_size", ctypes.c_int),
+        ("max_blocks_per_seq", ctypes.c_int), ("num_blocks", ctypes.c_int64),
+        ("q_dtype", ctypes.c_int), ("cache_dtype", ctypes.c_int), ("scale", ctypes.c_float),
+        ("num_ctas", ctypes.c_int),
+        ("h_query", ctypes.c_void_p), ("h_new_key", ctypes.c_void_p),
+        ("h_new_value", ctypes.c_void_p), ("h_slot_mapping", ctypes.c_void_p),
+        ("h_block_tables", ctypes.c_void_p), ("h_seq_lens", ctypes.c_void_p),
+        ("h_cow_pairs", ctypes.c_void_p), ("num_cow_pairs", ctypes.c_int64),
+        ("h_out", ctypes.c_void_p),
+        ("d_query", ctypes.c_void_p), ("d_new_key", ctypes.c_void_p),
+        ("d_new_value", ctypes.c_void_p), ("d_slot_mapping", ctypes.c_void_p),
+        ("d_block_tables", ctypes.c_void_p), ("d_seq_lens", ctypes.c_void_p),
+        ("d_cow_pairs", ctypes.c_void_p), ("d_out", ctypes.c_void_p),
+        ("key_cache", ctypes.c_void_p), ("value_cache", ctypes.c_void_p),
+        ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+_lib_handle = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libpkv.so (raises if it has not been built)."""
+    global _lib_handle
+    if _lib_handle is not None:
+        return _lib_handle
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m paged_kv_cache_373_b200._build` (no CPU fallback exists)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, c_int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+    L.pkv_reshape_and_cache.restype = c_int
+    L.pkv_reshape_and_cache.argtypes = [vp, vp, c_int, vp, vp, c_int, vp, i64, i64, c_int, c_int,
+                                        c_int, vp, vp, vp]
+    L.pkv_copy_blocks.restype = c_int
+    L.pkv_copy_blocks.argtypes = [vp, vp, c_int, vp, i64, i64, ctypes.c_size_t, vp]
+    L.pkv_paged_attention_workspace_bytes.restype = ctypes.c_size_t
+    L.pkv_paged_attention_workspace_bytes.argtypes = [c_int, c_int, c_int, c_int, c_int]
+    L.pkv_default_num_ctas.restype = c_int
+    L.pkv_default_num_ctas.argtypes = []
+    L.pkv_paged_attention_decode.restype = c_int
+    L.pkv_paged_attention_decode.argtypes = [vp, vp, c_int, vp, vp, c_int, vp, c_int, vp, c_int,
+                                             c_int, c_int, c_int, c_int, i64, ctypes.c_float, vp,
+                                             vp, vp, ctypes.c_size_t, c_int, vp]
+    L.pkv_decode_step_host.restype = c_int
+    L.pkv_decode_step_host.argtypes = [ctypes.POINTER(DecodeStepArgs), vp]
+    L.pkv_get_device_error.restype = c_int
+    L.pkv_get_device_error.argtypes = [ctypes.POINTER(i32), vp]
+    L.pkv_status_string.restype = ctypes.c_char_p
+    L.pkv_status_string.argtypes = [c_int]
+    L.pkv_last_error_message.restype = ctypes.c_char_p
+    L.pkv_last_error_message.argtypes = []
+    _lib_handle = L
+    return L
+
+
+def _check(status: int) -> None:
+    if status != PKV_OK:
+        L = lib()
+        raise PkvError(status, f"{L.pkv_status_string(status).decode()}: "
+                               f"{L.pkv_last_error_message().decode()}")
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def dtype_code(t: torch.Tensor) -> int:
+    return _DTYPES[t.dtype]
+
+
+def status_string(status: int) -> str:
+    return lib().pkv_status_string(status).decode()
+
+
+def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, k_scale=None,
+                      v_scale=None, stream=None) -> None:
+    """key/value [T, Hkv, D] -> caches [NB, bs, Hkv, D] at slot_mapping (int64 [T])."""
+    T, Hkv, D = key.shape
+    NB, bs = key_cache.shape[0], key_cache.shape[1]
+    _check(lib().pkv_reshape_and_cache(
+        _dev(key), _dev(value), dtype_code(key), _dev(key_cache), _dev(value_cache),
+        dtype_code(key_cache), _dev(slot_mapping), T, NB, bs, Hkv, D, _dev(k_scale), _dev(v_scale),
+        _stream(stream)))
+
+
+def copy_blocks(key_caches: Sequence[torch.Tensor], value_caches: Sequence[torch.Tensor],
+                block_mapping: torch.Tensor, stream=None) -> None:
+    """Copy whole blocks block_mapping[p,0] -> block_mapping[p,1] in every layer."""
+    n = len(key_caches)
+    kp = (ctypes.c_void_p * n)(*[_dev(t) for t in key_caches])
+    vp = (ctypes.c_void_p * n)(*[_dev(t) for t in value_caches])
+    kc = key_caches[0]
+    block_bytes = kc[0].numel() * kc.element_size()
+    _check(lib().pkv_copy_blocks(kp, vp, n, _dev(block_mapping), block_mapping.shape[0],
+                                 kc.shape[0], block_bytes, _stream(stream)))
+
+
+def paged_attention_workspace_bytes(num_seqs: int, num_heads: int, num_kv_heads: int,
+                                    head_dim: int, num_ctas: int = 0) -> int:
+    return int(lib().pkv_paged_attention_workspace_bytes(num_seqs, num_heads, num_kv_heads,
+                                                         head_dim, num_ctas))
+
+
+def default_num_ctas() -> int:
+    return int(lib().pkv_default_num_ctas())
+
+
+def alloc_workspace(num_seqs: int, num_heads: int, num_kv_heads: int, head_dim: int,
+                    num_ctas: int = 0, device=None) -> torch.Tensor:
+    n = paged_attention_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, num_ctas)
+    if n == 0:
+        raise PkvError(PKV_EINVAL, "invalid workspace shape")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def paged_attention_decode(out, query, key_cache, value_cache, block_tables, seq_lens, scale,
+                           k_scale=None, v_scale=None, workspace=None, num_ctas: int = 0,
+                           stream=None) -> torch.Tensor:
+    """out[S, Hq, D] = decode attention of query over the paged caches."""
+    S, Hq, D = query.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    if workspace is None:
+        workspace = alloc_workspace(S, Hq, Hkv, D, num_ctas, device=query.device)
+    _check(lib().pkv_paged_attention_decode(
+        _dev(out), _dev(query), dtype_code(query), _dev(key_cache), _dev(value_cache),
+        dtype_code(key_cache), _dev(block_tables), block_tables.shape[1], _dev(seq_lens), S, Hq,
+        Hkv, D, bs, NB, float(scale), _dev(k_scale), _dev(v_scale), _dev(workspace),
+        workspace.numel() * workspace.element_size(), int(num_ctas), _stream(stream)))
+    return out
+
+
+def decode_step_host(args: DecodeStepArgs, stream=None) -> None:
+    """One host-driven decode step (see pkv_decode_step_host); synchronises."""
+    _check(lib().pkv_decode_step_host(ctypes.byref(args), _stream(stream)))
+
+
+def get_device_error(stream=None) -> int:
+    """Synchronise, return and clear the device error word (PKV_DEVERR_* bits)."""
+    v = ctypes.c_int32(0)
+    st = lib().pkv_get_device_error(ctypes.byref(v), _stream(stream))
+    if st not in (PKV_OK, PKV_EDEVICE):
+        _check(st)
+    return int(v.value)

@@ -1,0 +1,36 @@
+// attn_launch.cuh -- launcher template shared by the per-variant
+// translation units (attn_*.cu): opt the kernel into its shared-memory size
+// once per device, launch the decode kernel and the split-merge kernel.
+#pragma once
+
+#include <atomic>
+#include <cstdio>
+
+#include "paged_attention.cuh"
+#include "pkv_internal.h"
+
+namespace pkv {
+
+template <class C>
+pkv_status launch_decode(const DecodeLaunchArgs& a, cudaStream_t st) {
+    static std::atomic<unsigned long long> configured{0};  // bit per device (< 64)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(PKV_ECUDA, "cudaGetDevice");
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured.load() & bit)) {
+        const cudaError_t e = cudaFuncSetAttribute(pkv_decode_kernel<C>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   C::kSmemBytes);
+        if (e != cudaSuccess) return fail(PKV_ECUDA, "smem opt-in: %s", cudaGetErrorString(e));
+        configured.fetch_or(bit);
+    }
+    pkv_decode_kernel<C><<<a.grid, kThreads, C::kSmemBytes, st>>>(*a.tmk, *a.tmv, *a.params);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PKV_ECUDA, "decode launch: %s", cudaGetErrorString(e));
+    pkv_merge_kernel<typename C::q_t><<<a.grid, 256, 0, st>>>(*a.params, C::D);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PKV_ECUDA, "merge launch: %s", cudaGetErrorString(e));
+    return PKV_OK;
+}
+
+}  // namespace pkv

@@ -1,0 +1,297 @@
+// pkv_api.cu -- host side of pkv_paged_attention_decode and the library
+// utilities: argument validation, TMA descriptor encoding, variant dispatch,
+// the device error word and the host-buffer decode step.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "paged_attention.cuh"
+#include "pkv_internal.h"
+
+namespace pkv {
+
+// The library's only device state: OR of PKV_DEVERR_* bits, one per device.
+__device__ int g_pkv_error;
+
+namespace {
+thread_local char g_msg[512] = "";
+constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices] = {nullptr};
+std::mutex g_err_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+}  // namespace
+
+pkv_status fail(pkv_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+int dtype_bytes(pkv_dtype d) {
+    switch (d) {
+    case PKV_F32: return 4;
+    case PKV_F16: case PKV_BF16: return 2;
+    case PKV_FP8_E4M3: return 1;
+    default: return 0;
+    }
+}
+
+int* device_error_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_err_mu);
+    if (!g_err_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_pkv_error) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<int*>(p);
+    }
+    return g_err_ptr[dev];
+}
+
+// 4-D tiled map over a cache [NB, bs, Hkv, D]: dims (D, Hkv, bs, NB), box
+// (128 bytes of D, 1 head, 16 tokens, 1 block), 128-byte swizzle.
+static pkv_status encode_cache_map(CUtensorMap* map, const void* base, pkv_dtype dt, int64_t nb,
+                                   int bs, int hkv, int d) {
+    auto fn = encode_fn();
+    if (!fn) return fail(PKV_ECUDA, "cuTensorMapEncodeTiled unavailable");
+    const int es = dtype_bytes(dt);
+    CUtensorMapDataType t;
+    switch (dt) {
+    case PKV_F32: t = CU_TENSOR_MAP_DATA_TYPE_FLOAT32; break;
+    case PKV_F16: t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16; break;
+    case PKV_BF16: t = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; break;
+    default: t = CU_TENSOR_MAP_DATA_TYPE_UINT8; break;
+    }
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)hkv, (cuuint64_t)bs, (cuuint64_t)nb};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * es, (cuuint64_t)hkv * d * es,
+                                   (cuuint64_t)bs * hkv * d * es};
+    const cuuint32_t box[4] = {(cuuint32_t)(128 / es), 1u, (cuuint32_t)kTileTokens, 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    const CUresult r = fn(map, t, 4, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PKV_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return PKV_OK;
+}
+
+static int default_ctas() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return sms;
+}
+
+struct WsLayout {
+    size_t o_bytes, ml_off, total;
+    int hpu, nch, grid;
+};
+
+static bool ws_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int num_ctas,
+                      WsLayout* w) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return false;
+    if (head_dim <= 0 || num_ctas < 0) return false;
+    const int g = num_heads / num_kv_heads;
+    w->grid = num_ctas > 0 ? num_ctas : default_ctas();
+    if (w->grid <= 0) return false;
+    w->nch = (g + kHeadsPerUnit - 1) / kHeadsPerUnit;
+    w->hpu = g < kHeadsPerUnit ? g : kHeadsPerUnit;
+    const size_t segs = (size_t)w->grid + (size_t)num_seqs * num_kv_heads * w->nch;
+    w->o_bytes = segs * w->hpu * head_dim * sizeof(float);
+    w->ml_off = (w->o_bytes + 255) & ~(size_t)255;
+    w->total = w->ml_off + segs * w->hpu * sizeof(float2);
+    return true;
+}
+
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" int pkv_default_num_ctas(void) { return default_ctas(); }
+
+extern "C" size_t pkv_paged_attention_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
+                                                      int head_dim, int num_ctas) {
+    WsLayout w;
+    if (!ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, num_ctas, &w)) return 0;
+    return w.total;
+}
+
+extern "C" pkv_status pkv_paged_attention_decode(void* out, const void* query, pkv_dtype q_dtype,
+                                                 const void* key_cache, const void* value_cache,
+                                                 pkv_dtype cache_dtype, const int32_t* block_tables,
+                                                 int max_blocks_per_seq, const int32_t* seq_lens,
+                                                 int num_seqs, int num_heads, int num_kv_heads,
+                                                 int head_dim, int block_size, int64_t num_blocks,
+                                                 float scale, const float* k_scale, const float* v_scale,
+                                                 void* workspace, size_t workspace_bytes, int num_ctas,
+                                                 pkv_stream_t stream) {
+    if (num_seqs < 0) return fail(PKV_EINVAL, "num_seqs < 0");
+    if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
+        return fail(PKV_EINVAL, "num_heads must be a positive multiple of num_kv_heads");
+    if (head_dim != 64 && head_dim != 128) return fail(PKV_EUNSUPPORTED, "head_dim %d", head_dim);
+    if (block_size != 16 && block_size != 32) return fail(PKV_EUNSUPPORTED, "block_size %d", block_size);
+    if (num_blocks <= 0 || num_blocks > 0x7fffffffLL) return fail(PKV_EINVAL, "num_blocks out of range");
+    if (max_blocks_per_seq <= 0 || (int64_t)max_blocks_per_seq * block_size > 0x7fffffffLL)
+        return fail(PKV_EINVAL, "max_blocks_per_seq out of range");
+    if (!std::isfinite(scale)) return fail(PKV_EINVAL, "scale must be finite");
+    if (num_ctas < 0) return fail(PKV_EINVAL, "num_ctas < 0");
+    // dtype combination -> launcher
+    pkv_status (*launch)(const DecodeLaunchArgs&, cudaStream_t) = nullptr;
+    if (cache_dtype == PKV_F32 && q_dtype == PKV_F32)
+        launch = head_dim == 64 ? launch_decode_f32_d64 : launch_decode_f32_d128;
+    else if (cache_dtype == PKV_F16 && q_dtype == PKV_F16)
+        launch = head_dim == 64 ? launch_decode_f16_d64 : launch_decode_f16_d128;
+    else if (cache_dtype == PKV_BF16 && q_dtype == PKV_BF16)
+        launch = head_dim == 64 ? launch_decode_bf16_d64 : launch_decode_bf16_d128;
+    else if (cache_dtype == PKV_FP8_E4M3 && head_dim == 128 && (q_dtype == PKV_F16 || q_dtype == PKV_BF16))
+        launch = q_dtype == PKV_F16 ? launch_decode_fp8_qf16_d128 : launch_decode_fp8_qbf16_d128;
+    if (!launch) return fail(PKV_EUNSUPPORTED, "q dtype %d with cache dtype %d, head_dim %d",
+                             (int)q_dtype, (int)cache_dtype, head_dim);
+    if (cache_dtype == PKV_FP8_E4M3 && (!k_scale || !v_scale))
+        return fail(PKV_EINVAL, "FP8 cache needs k_scale and v_scale");
+    if (num_seqs == 0) return PKV_OK;
+    if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens || !workspace)
+        return fail(PKV_EINVAL, "null pointer");
+    if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
+        !aligned16(workspace))
+        return fail(PKV_EINVAL, "out, query, caches and workspace must be 16-byte aligned");
+    WsLayout w;
+    if (!ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, num_ctas, &w))
+        return fail(PKV_ECUDA, "cannot size the grid");
+    if (workspace_bytes < w.total)
+        return fail(PKV_EINVAL, "workspace too small: %zu < %zu bytes", workspace_bytes, w.total);
+    int* err = device_error_word();
+    if (!err) return fail(PKV_ECUDA, "device error word unavailable");
+
+    CUtensorMap tmk, tmv;
+    pkv_status st;
+    if ((st = encode_cache_map(&tmk, key_cache, cache_dtype, num_blocks, block_size, num_kv_heads,
+                               head_dim)) != PKV_OK)
+        return st;
+    if ((st = encode_cache_map(&tmv, value_cache, cache_dtype, num_blocks, block_size, num_kv_heads,
+                               head_dim)) != PKV_OK)
+        return st;
+
+    DecodeParams p;
+    p.out = out;
+    p.q = query;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.k_scale = cache_dtype == PKV_FP8_E4M3 ? k_scale : nullptr;
+    p.v_scale = cache_dtype == PKV_FP8_E4M3 ? v_scale : nullptr;
+    p.ws_o = static_cast<float*>(workspace);
+    p.ws_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + w.ml_off);
+    p.err = err;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.g = num_heads / num_kv_heads;
+    p.nch = w.nch;
+    p.hpu = w.hpu;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.block_size = block_size;
+    p.num_blocks = (int)num_blocks;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    DecodeLaunchArgs a{&p, &tmk, &tmv, w.grid};
+    return launch(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" pkv_status pkv_decode_step_host(const pkv_decode_step_args* a, pkv_stream_t stream) {
+    if (!a) return fail(PKV_EINVAL, "null args");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int S = a->num_seqs;
+    if (S < 0) return fail(PKV_EINVAL, "num_seqs < 0");
+    const int qb = dtype_bytes(a->q_dtype);
+    if (qb == 0) return fail(PKV_EINVAL, "q dtype");
+    const size_t q_bytes = (size_t)S * a->num_heads * a->head_dim * qb;
+    const size_t kv_bytes = (size_t)S * a->num_kv_heads * a->head_dim * qb;
+    struct Cp { void* dst; const void* src; size_t n; };
+    const Cp h2d[] = {
+        {a->d_query, a->h_query, q_bytes},
+        {a->d_new_key, a->h_new_key, kv_bytes},
+        {a->d_new_value, a->h_new_value, kv_bytes},
+        {a->d_slot_mapping, a->h_slot_mapping, (size_t)S * sizeof(int64_t)},
+        {a->d_block_tables, a->h_block_tables, (size_t)S * a->max_blocks_per_seq * sizeof(int32_t)},
+        {a->d_seq_lens, a->h_seq_lens, (size_t)S * sizeof(int32_t)},
+        {a->d_cow_pairs, a->h_cow_pairs, (size_t)(a->num_cow_pairs > 0 ? a->num_cow_pairs : 0) * 2 * sizeof(int64_t)},
+    };
+    for (const Cp& c : h2d) {
+        if (c.n == 0) continue;
+        if (!c.dst || !c.src) return fail(PKV_EINVAL, "null staging or host buffer");
+        const cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, st);
+        if (e != cudaSuccess) return fail(PKV_ECUDA, "H2D copy: %s", cudaGetErrorString(e));
+    }
+    pkv_status s;
+    if (a->num_cow_pairs > 0) {
+        void* kcs[1] = {a->key_cache};
+        void* vcs[1] = {a->value_cache};
+        const size_t block_bytes = (size_t)a->block_size * a->num_kv_heads * a->head_dim *
+                                   dtype_bytes(a->cache_dtype);
+        if ((s = pkv_copy_blocks(kcs, vcs, 1, a->d_cow_pairs, a->num_cow_pairs, a->num_blocks,
+                                 block_bytes, stream)) != PKV_OK)
+            return s;
+    }
+    if ((s = pkv_reshape_and_cache(a->d_new_key, a->d_new_value, a->q_dtype, a->key_cache,
+                                   a->value_cache, a->cache_dtype, a->d_slot_mapping, S,
+                                   a->num_blocks, a->block_size, a->num_kv_heads, a->head_dim,
+                                   a->k_scale, a->v_scale, stream)) != PKV_OK)
+        return s;
+    if ((s = pkv_paged_attention_decode(a->d_out, a->d_query, a->q_dtype, a->key_cache, a->value_cache,
+                                        a->cache_dtype, a->d_block_tables, a->max_blocks_per_seq,
+                                        a->d_seq_lens, S, a->num_heads, a->num_kv_heads, a->head_dim,
+                                        a->block_size, a->num_blocks, a->scale, a->k_scale, a->v_scale,
+                                        a->workspace, a->workspace_bytes, a->num_ctas, stream)) != PKV_OK)
+        return s;
+    if (q_bytes) {
+        if (!a->h_out || !a->d_out) return fail(PKV_EINVAL, "null output buffer");
+        const cudaError_t e = cudaMemcpyAsync(a->h_out, a->d_out, q_bytes, cudaMemcpyDeviceToHost, st);
+        if (e != cudaSuccess) return fail(PKV_ECUDA, "D2H copy: %s", cudaGetErrorString(e));
+    }
+    const cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return fail(PKV_ECUDA, "decode step: %s", cudaGetErrorString(e));
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_get_device_error(int32_t* code_out, pkv_stream_t stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int32_t v = 0;
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&v, g_pkv_error, sizeof(v));
+    if (e == cudaSuccess) {
+        const int32_t zero = 0;
+        e = cudaMemcpyToSymbol(g_pkv_error, &zero, sizeof(zero));
+    }
+    if (e != cudaSuccess) return fail(PKV_ECUDA, "get_device_error: %s", cudaGetErrorString(e));
+    if (code_out) *code_out = v;
+    return v ? PKV_EDEVICE : PKV_OK;
+}
+
+extern "C" const char* pkv_status_string(pkv_status s) {
+    switch (s) {
+    case PKV_OK: return "ok";
+    case PKV_EINVAL: return "invalid argument";
+    case PKV_EUNSUPPORTED: return "unsupported combination";
+    case PKV_ECUDA: return "CUDA error";
+    case PKV_EDEVICE: return "device-side error flag set";
+    default: return "unknown status";
+    }
+}
+
+extern "C" const char* pkv_last_error_message(void) { return g_msg; }

@@ -1,0 +1,194 @@
+"""GPU parity of the decode step (copy_blocks -> reshape_and_cache ->
+paged_attention_decode) against the fp64 oracle, through the C ABI.
+
+Tolerances (max-abs vs the oracle): 2e-3 for f32/f16/bf16 caches, 2e-2 for
+FP8 caches (the oracle uses the same dequantised values), each plus half an
+ulp of the output dtype for the final store."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_373_b200 as pkv
+from paged_kv_cache_373_b200 import workloads as W
+from pkv_testutil import compare, gpu_inputs, gpu_step, oracle_step
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "cfg1": lambda: W.config1(),
+    "f16_mha_d128": lambda: W.build_decode("f16_mha_d128", [1, 5, 16, 17, 33, 64, 100, 250, 513],
+                                           8, 8, 128, 16, torch.float16, torch.float16, seed=31),
+    "f16_gqa_d64_bs32": lambda: W.build_decode("f16_gqa_d64_bs32", [2, 31, 32, 33, 95, 300],
+                                               8, 2, 64, 32, torch.float16, torch.float16, seed=32),
+    "bf16_gqa4_d128": lambda: W.build_decode("bf16_gqa4_d128", [1, 15, 16, 47, 64, 200, 777],
+                                             32, 8, 128, 16, torch.bfloat16, torch.bfloat16, seed=33),
+    "bf16_g1_d64": lambda: W.build_decode("bf16_g1_d64", [3, 16, 18, 129], 4, 4, 64, 16,
+                                          torch.bfloat16, torch.bfloat16, seed=34),
+    "bf16_g3_ragged": lambda: W.build_decode("bf16_g3_ragged", [7, 40, 100], 6, 2, 128, 16,
+                                             torch.bfloat16, torch.bfloat16, seed=35),
+    "bf16_g16_two_chunks": lambda: W.build_decode("bf16_g16", [9, 80, 160], 32, 2, 128, 32,
+                                                  torch.bfloat16, torch.bfloat16, seed=36),
+    "f32_d128": lambda: W.build_decode("f32_d128", [1, 17, 64, 90], 4, 2, 128, 16, torch.float32,
+                                       torch.float32, seed=37),
+    "fp8_g8_bs32_qbf16": lambda: W.build_decode("fp8_g8", [1, 33, 64, 500, 1025], 64, 8, 128, 32,
+                                                W.FP8, torch.bfloat16, seed=38),
+    "fp8_g1_bs16_qf16": lambda: W.build_decode("fp8_g1", [2, 16, 17, 260], 4, 4, 128, 16, W.FP8,
+                                               torch.float16, seed=39),
+    "cfg5_mini": lambda: W.config5(num_prompts=2, samples=4, prefix=200, tail_lo=3, tail_hi=40),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_parity(name):
+    wl = SMALL[name]()
+    out, err, _ = gpu_step(wl)
+    assert err == 0
+    compare(out, oracle_step(wl), wl)
+
+
+@pytest.mark.parametrize("num_ctas", [1, 3, 17, 148, 1000])
+def test_split_count_changes_stay_within_tolerance(num_ctas):
+    wl = SMALL["bf16_gqa4_d128"]()
+    out, err, _ = gpu_step(wl, num_ctas=num_ctas)
+    assert err == 0
+    compare(out, oracle_step(wl), wl)
+
+
+def test_physical_permutation_is_bit_identical():
+    wl = SMALL["f16_mha_d128"]()
+    out1, _, g = gpu_step(wl, num_ctas=40)
+    # relabel every physical block b -> perm[b] and move its data accordingly
+    perm = torch.randperm(wl.num_blocks, generator=torch.Generator().manual_seed(9))
+    wl2 = W.build_decode("f16_mha_d128", [1, 5, 16, 17, 33, 64, 100, 250, 513], 8, 8, 128, 16,
+                         torch.float16, torch.float16, seed=31)
+    kc, vc = torch.empty_like(wl2.key_cache), torch.empty_like(wl2.value_cache)
+    kc[perm], vc[perm] = wl2.key_cache, wl2.value_cache
+    wl2.key_cache, wl2.value_cache = kc, vc
+    t = wl2.block_tables.clone()
+    m = t >= 0
+    t[m] = perm[t[m].long()].to(torch.int32)
+    wl2.block_tables = t
+    s = wl2.slot_mapping.clone()
+    s = perm[s // 16] * 16 + s % 16
+    wl2.slot_mapping = s
+    out2, err, _ = gpu_step(wl2, num_ctas=40)
+    assert err == 0
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def test_shared_prefix_equals_private_copies_bit_identical():
+    wl = W.config5(num_prompts=3, samples=8, prefix=3000, tail_lo=32, tail_hi=512)
+    out1, err1, _ = gpu_step(wl, num_ctas=148)
+    out2, err2, _ = gpu_step(W.with_all_copies(wl), num_ctas=148)
+    assert err1 == 0 and err2 == 0
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def test_empty_and_single_token_sequences():
+    wl = W.build_decode("edge", [0, 1, 0, 16, 1, 0], 4, 2, 128, 16, torch.bfloat16,
+                        torch.bfloat16, seed=40)
+    out, err, g = gpu_step(wl)
+    assert err == 0
+    ref = oracle_step(wl)
+    compare(out, ref, wl)
+    assert float(out[0].abs().max()) == 0.0 and float(out[2].abs().max()) == 0.0
+    # seq_len 1: the output is the new token's value row (softmax of one score)
+    v1 = wl.new_value[1].float()                 # [Hkv, D]
+    for h in range(4):
+        assert torch.equal(out[1, h].float().cpu(), v1[h // 2])
+
+
+def test_all_sequences_empty():
+    wl = W.build_decode("allempty", [0, 0, 0], 4, 4, 64, 16, torch.float16, torch.float16, seed=41)
+    out, err, _ = gpu_step(wl)
+    assert err == 0 and float(out.abs().max()) == 0.0
+
+
+def test_indexing_probe_exact():
+    """One dominant key per (sequence, head) picks out one logical token; the
+    output must equal that token's value row exactly, which pins the
+    logical -> physical translation (zwxr.cn 3.2) bit for bit."""
+    S, H, D, bs = 6, 8, 128, 16
+    lens = [5, 16, 17, 64, 130, 400]
+    wl = W.build_decode("probe", lens, H, H, D, bs, torch.float16, torch.float16, seed=42)
+    NB = wl.num_blocks
+    # value rows encode (physical block, slot, head) as small exact integers
+    b = torch.arange(NB).view(NB, 1, 1, 1)
+    sl = torch.arange(bs).view(1, bs, 1, 1)
+    hh = torch.arange(H).view(1, 1, H, 1)
+    d = torch.arange(D).view(1, 1, 1, D)
+    wl.value_cache = (((b * bs + sl) * 7 + hh * 3 + d) % 2000).to(torch.float16)
+    wl.key_cache = torch.zeros((NB, bs, H, D), dtype=torch.float16)
+    wl.new_key = torch.zeros_like(wl.new_key)
+    wl.new_value = torch.full_like(wl.new_value, -1.0)
+    q = torch.zeros((S, H, D), dtype=torch.float16)
+    q[:, :, 0] = 1.0
+    g = torch.Generator().manual_seed(3)
+    target = {}
+    for s in range(S):
+        for h in range(H):
+            t = int(torch.randint(0, lens[s] - 1, (1,), generator=g))   # an existing token
+            phys = int(wl.block_tables[s, t // bs])
+            wl.key_cache[phys, t % bs, h, 0] = 1000.0
+            target[(s, h)] = (phys, t % bs)
+    wl.query = q
+    out, err, _ = gpu_step(wl)
+    assert err == 0
+    for (s, h), (phys, off) in target.items():
+        assert torch.equal(out[s, h].cpu(), wl.value_cache[phys, off, h]), (s, h)
+
+
+def test_bad_block_id_is_flagged_not_fatal():
+    wl = W.build_decode("badid", [40, 20], 4, 4, 64, 16, torch.float16, torch.float16, seed=43)
+    wl.block_tables[0, 1] = wl.num_blocks + 5
+    out, err, _ = gpu_step(wl)
+    assert err & pkv.DEVERR_BLOCK_ID
+    torch.cuda.synchronize()                       # the context is still usable
+    wl2 = SMALL["cfg1"]()
+    out2, err2, _ = gpu_step(wl2)
+    assert err2 == 0
+    compare(out2, oracle_step(wl2), wl2)
+
+
+def test_seq_len_beyond_table_is_flagged():
+    wl = W.build_decode("badlen", [40], 4, 4, 64, 16, torch.float16, torch.float16, seed=44)
+    g = gpu_inputs(wl)
+    g["lens"][0] = 1000                              # table row holds 3 blocks
+    out = torch.empty_like(g["q"])
+    pkv.paged_attention_decode(out, g["q"], g["kc"], g["vc"], g["tables"], g["lens"], wl.scale)
+    assert pkv.get_device_error() & pkv.DEVERR_SEQ_LEN
+
+
+def test_host_validation_rejects_before_launch():
+    wl = SMALL["cfg1"]()
+    g = gpu_inputs(wl)
+    out = torch.empty_like(g["q"])
+    with pytest.raises(pkv.PkvError) as e:
+        pkv.paged_attention_decode(out, g["q"], g["kc"], g["vc"], g["tables"], g["lens"], wl.scale,
+                                   workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == pkv.PKV_EINVAL
+    with pytest.raises(pkv.PkvError) as e:                       # q dtype != cache dtype
+        pkv.paged_attention_decode(out.half(), g["q"].half(), g["kc"], g["vc"], g["tables"],
+                                   g["lens"], wl.scale)
+    assert e.value.status == pkv.PKV_EUNSUPPORTED
+
+
+# ---- full-size configurations, sampled sequences ----------------------------
+def _sample(wl, k, seed):
+    g = torch.Generator().manual_seed(seed)
+    idx = torch.randperm(wl.num_seqs, generator=g)[:k].tolist()
+    # always include the longest and the shortest sequence
+    idx += [int(wl.seq_lens.argmax()), int(wl.seq_lens.argmin())]
+    return sorted(set(idx))
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+def test_full_config_sampled_parity(cfg):
+    wl = W.make_config(cfg)
+    out, err, _ = gpu_step(wl)
+    assert err == 0
+    seqs = _sample(wl, 6, cfg)
+    compare(out, oracle_step(wl, seqs=seqs), wl, seqs=seqs)
+    assert torch.isfinite(out.float()).all()
