@@ -123,9 +123,9 @@ pkv_status pkv_copy_blocks(void* const* key_caches, void* const* value_caches, i
 
 /*
  * Workspace for pkv_paged_attention_decode: fp32 partial results of the
- * split sequences, (num_ctas + units) x heads_per_unit x (head_dim + 2)
- * floats, where units = num_seqs * num_kv_heads * ceil(g / 8) and
- * g = num_heads / num_kv_heads.  num_ctas = 0 means the default grid of the
+ * split units, (8 * num_ctas + units) x heads_per_unit x (head_dim + 2)
+ * floats, where units = num_seqs * num_kv_heads * ceil(g / 8),
+ * g = num_heads / num_kv_heads and heads_per_unit = min(g, 8).  num_ctas = 0 means the default grid of the
  * current device (pkv_default_num_ctas).  Returns 0 for invalid shapes.
  * The workspace needs no initialisation.
  */
@@ -156,9 +156,10 @@ int pkv_default_num_ctas(void);
  * caches the q.K and P.V products run on tensor cores with 16-bit operands
  * (P rounded to the cache's 16-bit type, f16 for FP8).  Output is rounded
  * to the q dtype (RNE).
- * Long sequences are split across CTAs (balanced over all (sequence, kv head)
- * work) and their partial (m, l, o) are merged exactly by a second kernel on
- * the same stream.  Results are bit-identical under any permutation of the
+ * Every warp of the persistent grid takes an equal share of all
+ * (sequence, kv head) tiles, so long sequences are split across warps and
+ * their partial (m, l, o) are merged exactly by a second kernel on the same
+ * stream.  Results are bit-identical under any permutation of the
  * physical block ids and independent of block sharing, for a fixed num_ctas.
  * workspace: device, >= pkv_paged_attention_workspace_bytes(...) bytes,
  *   16-byte aligned, contents need no initialisation.

@@ -1,6 +1,7 @@
 // attn_launch.cuh -- launcher template shared by the per-variant
 // translation units (attn_*.cu): opt the kernel into its shared-memory size
-// once per device, launch the decode kernel and the split-merge kernel.
+// once per device, launch the decode kernel (one warp = one worker) and the
+// split-merge kernel (one warp per worker boundary).
 #pragma once
 
 #include <atomic>
@@ -24,10 +25,11 @@ pkv_status launch_decode(const DecodeLaunchArgs& a, cudaStream_t st) {
         if (e != cudaSuccess) return fail(PKV_ECUDA, "smem opt-in: %s", cudaGetErrorString(e));
         configured.fetch_or(bit);
     }
-    pkv_decode_kernel<C><<<a.grid, kThreads, C::kSmemBytes, st>>>(*a.tmk, *a.tmv, *a.params);
+    pkv_decode_kernel<C><<<a.grid, C::kWarps * 32, C::kSmemBytes, st>>>(*a.params);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "decode launch: %s", cudaGetErrorString(e));
-    pkv_merge_kernel<typename C::q_t><<<a.grid, 256, 0, st>>>(*a.params, C::D);
+    const int64_t workers = (int64_t)a.grid * C::kWarps;
+    pkv_merge_kernel<typename C::q_t, C::D><<<(unsigned)((workers + 7) / 8), 256, 0, st>>>(*a.params, workers);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "merge launch: %s", cudaGetErrorString(e));
     return PKV_OK;

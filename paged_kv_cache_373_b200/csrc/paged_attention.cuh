@@ -1,33 +1,32 @@
-// paged_attention.cuh -- persistent, warp-specialised decode attention over a
-// paged KV cache (sm_100a).
+// paged_attention.cuh -- decode attention over a paged KV cache (sm_100a).
 //
 // What it computes: "PagedAttention不够用了之后" (thinkmoon.cn), section
 // "PagedAttention 的计算优化": per sequence, gather the blocks named by the
-// block table, softmax(q.K^T * scale) . V -- restricted to the sequence's
-// logical length -- with the block-wise softmax of zwxr.cn section 3.3
-// (running max m and normaliser l per block, merged by rescaling).
+// block table and compute softmax(q.K^T * scale) . V over the sequence's
+// logical length, using the block-wise softmax of zwxr.cn section 3.3
+// (running max m and normaliser l, merged by rescaling).
 //
 // How (B200 design):
-//   * Work = tiles of 16 tokens of one (sequence, kv head, <= 8 q heads)
-//     "unit".  All tiles of all units form one sequence of W tiles; CTA b of
-//     the persistent grid takes the contiguous range [b*ceil(W/G), ...), so
-//     every SM streams the same number of bytes whatever the length mix.
-//     A unit cut by a range boundary leaves per-CTA partials (m, l, o) in the
-//     workspace that pkv_merge_kernel combines exactly.
-//   * Warp 8 (producer) translates each tile through the block table and
-//     issues TMA box loads of its K and V rows (16 tokens x head_dim, one kv
-//     head, 128-byte-swizzled) into a ring of shared-memory stages guarded by
-//     mbarriers; the q rows of each unit arrive by a 1-D bulk copy together
-//     with a small unit header.
-//   * Warps 0..7 (consumers) take the tiles of a unit round-robin.  q.K^T and
-//     P.V run on mma.sync tensor cores (tokens x heads and head_dim x heads
-//     tiles, fp32 accumulators in registers) so one K/V read serves all q
-//     heads of the GQA group; the online softmax runs on the accumulators.
-//     FP8 E4M3 rows are converted to f16 in registers (exact).  fp32 caches
-//     use CUDA cores.  At the end of a unit the warps' partial states are
-//     merged through shared memory.
-// Every wait is bounded; a wait that gives up raises PKV_DEVERR_TIMEOUT and
-// all warps unwind together.
+//   * Work unit = (sequence, kv head, <= 8 q heads of its GQA group); a unit
+//     of length L is ceil(L/16) tiles of 16 tokens.  The tiles of all units
+//     are laid end to end (W tiles) and every warp of the persistent grid is a
+//     worker that takes one contiguous range of ceil(W / workers) tiles, so
+//     every warp streams the same number of KV bytes whatever the length mix.
+//   * A worker streams its tiles through its own ring of shared-memory
+//     stages with 16-byte cp.async loads (the row gather of a paged cache is
+//     ~50 % faster this way than with TMA boxes on B200: 6.9 vs 4.5 TB/s
+//     measured for 256-byte rows), block-table entries prefetched 32 blocks
+//     ahead, the q rows of each unit riding in the same async group.
+//   * Tile math on tensor cores: S^T[16 tokens x 8 heads] = K q^T and
+//     O^T[head_dim x 8 heads] += V^T P^T with mma.sync (fp32 accumulators in
+//     registers) so one K/V read serves every q head of the group; the online
+//     softmax runs on the accumulator fragments (exp2 domain, fp32).  FP8 E4M3
+//     rows convert exactly to f16 in registers; fp32 caches use CUDA cores.
+//   * A worker whose range holds a whole unit writes the output; a unit cut
+//     by range boundaries leaves per-worker partials (m, l, o) that
+//     pkv_merge_kernel combines exactly.
+// No warp waits on another warp: the only synchronisation is each warp's own
+// cp.async groups, so nothing in the kernel can wait forever.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -39,21 +38,22 @@
 
 namespace pkv {
 
-constexpr int kTileTokens = 16;   // tokens per pipeline tile
-constexpr int kHeadsPerUnit = 8;  // q heads served by one KV read (one mma N tile)
-constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kSubBytes = kTileTokens * 128;  // one 128-byte-wide TMA box of 16 rows
+constexpr int kTileTokens = 16;    // tokens per pipeline tile
+constexpr int kHeadsPerUnit = 8;   // q heads served by one KV read (one mma N tile)
+constexpr int kMaxWarpsPerCta = 8; // workspace is sized for this many workers per CTA
+constexpr int kSubBytes = kTileTokens * 128;  // one 128-byte-wide column of a tile
 
 struct DecodeParams {
     void* out;
     const void* q;
+    const uint8_t* key_cache;
+    const uint8_t* value_cache;
     const int32_t* block_tables;
     const int32_t* seq_lens;
     const float* k_scale;  // device scalars (FP8 caches) or null
     const float* v_scale;
-    float* ws_o;           // [(G + units) * hpu * D] partial outputs (unnormalised)
-    float2* ws_ml;         // [(G + units) * hpu] partial (m, l), log2 domain
+    float* ws_o;           // [(workers + units) * hpu * D] partial outputs (unnormalised)
+    float2* ws_ml;         // [(workers + units) * hpu] partial (m, l), log2 domain
     int* err;
     int num_seqs, num_heads, num_kv_heads;
     int g;                 // q heads per kv head
@@ -63,24 +63,13 @@ struct DecodeParams {
     float scale_log2;      // scale * log2(e)
 };
 
-struct UnitHeader {
-    int s, kh, c, nh;  // sequence, kv head, head chunk, real heads in the chunk
-    int L;             // sequence length (clamped to the table capacity)
-    int i0, i1;        // this CTA's tile range of the unit
-    int split;         // 1: partial result goes to the workspace
-    int seg;           // workspace segment of the partial
-    int done;          // 1: no more units for this CTA
-    int pad[6];
-};
-static_assert(sizeof(UnitHeader) == 64, "header size");
-
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
 __device__ __forceinline__ int ntiles_of(int L) { return (L + kTileTokens - 1) / kTileTokens; }
 
 // Warp-collective: total tiles W = units_per_seq * sum_s ceil(L_s / 16);
 // *bad_len is set when some length is negative or overruns its table row.
 __device__ inline int64_t total_tiles(const int32_t* seq_lens, int S, int units, int cap,
-                               bool* bad_len = nullptr) {
+                                      bool* bad_len = nullptr) {
     const int lane = threadIdx.x & 31;
     int64_t tot = 0;
     bool bad = false;
@@ -141,7 +130,7 @@ __device__ inline SeqHit find_seq(const int32_t* seq_lens, int S, int units, int
                     acc += w[k];
                 }
             }
-            found = __shfl_sync(kFull, found, src) - 1;
+            found = max(__shfl_sync(kFull, found, src) - 1, 0);
             at = __shfl_sync(kFull, at, src);
             return SeqHit{found, at, clamp_len(__ldg(seq_lens + found), cap)};
         }
@@ -150,40 +139,75 @@ __device__ inline SeqHit find_seq(const int32_t* seq_lens, int S, int units, int
     return SeqHit{S, base, 0};
 }
 
+// Walk over a worker's tiles in order: (sequence, unit j, tile i).
+struct Walk {
+    int s, L, nt, j, i, seg_i0, ord;
+    int64_t T, te;
+    bool done;
+
+    __device__ void init(const int32_t* seq_lens, int S, int units, int cap, int64_t tb, int64_t te_) {
+        te = te_;
+        T = tb;
+        done = tb >= te_;
+        ord = 0;
+        s = 0; L = 0; nt = 1; j = 0; i = 0; seg_i0 = 0;
+        if (done) return;
+        const SeqHit h = find_seq(seq_lens, S, units, cap, tb);
+        s = h.s;
+        L = h.L;
+        nt = ntiles_of(L);
+        j = (int)((tb - h.base) / nt);
+        i = (int)((tb - h.base) % nt);
+        seg_i0 = i;
+    }
+    __device__ bool first() const { return i == seg_i0; }
+    __device__ bool last() const { return i == nt - 1 || T == te - 1; }
+    __device__ void advance(const int32_t* seq_lens, int S, int units, int cap) {
+        if (done) return;
+        if (++T >= te) { done = true; return; }
+        if (++i == nt) {
+            i = 0;
+            seg_i0 = 0;
+            ++ord;
+            if (++j == units) {
+                j = 0;
+                do {  // a later non-empty sequence exists because T < te <= W
+                    ++s;
+                    L = (s < S) ? clamp_len(__ldg(seq_lens + s), cap) : kTileTokens;
+                    nt = ntiles_of(L);
+                } while (nt == 0);
+            }
+        }
+    }
+};
+
 // ----------------------------------------------------------------------------
-// Per-variant traits and consumer math.
+// Per-variant traits.
 // ----------------------------------------------------------------------------
 enum class Path { kMma16, kFp8, kF32 };
 
-template <typename KvT, typename QT, int D_, Path P_>
+template <typename KvT, typename QT, int D_, Path P_, int kWarps_, int kStages_>
 struct Cfg {
     using kv_t = KvT;
     using q_t = QT;
     static constexpr Path kPath = P_;
     static constexpr int D = D_;
+    static constexpr int kWarps = kWarps_;
+    static constexpr int kStages = kStages_;
     static constexpr int kKvBytes = (int)sizeof(KvT);
     static constexpr int kQBytes = (int)sizeof(QT);
     static constexpr int kRowBytes = D * kKvBytes;
-    static constexpr int kNSub = kRowBytes / 128;       // 128-byte TMA boxes per row
-    static constexpr int kBoxElems = 128 / kKvBytes;    // elements per box row
+    static constexpr int kNSub = kRowBytes / 128;       // 128-byte columns per row
     static constexpr int kTensorTile = kNSub * kSubBytes;
     static constexpr int kStageBytes = 2 * kTensorTile; // K tile + V tile
-    static constexpr int kStages = (128 * 1024) / kStageBytes;
-    static constexpr int kQData = kHeadsPerUnit * D * kQBytes;
-    static constexpr int kQSlot = 128 + kQData;         // header (64 B) + pad + q rows
-    static constexpr int kScrStride = D + 4;            // padded head stride (floats)
-    static constexpr int kScrAcc = kConsumerWarps * kHeadsPerUnit * kScrStride * 4;
-    static constexpr int kScrMl = kConsumerWarps * kHeadsPerUnit * 8;
-    static constexpr int kOffStages = 0;
-    static constexpr int kOffQ = kOffStages + kStages * kStageBytes;
-    static constexpr int kOffScr = kOffQ + 2 * kQSlot;
-    static constexpr int kOffMl = kOffScr + kScrAcc;
-    static constexpr int kOffBar = kOffMl + kScrMl;
-    static constexpr int kNumBars = 2 * kStages + 4;
-    static constexpr int kOffAbort = kOffBar + kNumBars * 8;
-    static constexpr int kSmemBytes = kOffAbort + 16 + 1024;  // + alignment slack
-    static_assert(kRowBytes % 128 == 0, "rows must be whole 128-byte boxes");
-    static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
+    static constexpr int kQSlot = kHeadsPerUnit * D * kQBytes;
+    static constexpr int kWarpBytes = kStages * (kStageBytes + kQSlot);
+    static constexpr int kSmemBytes = kWarps * kWarpBytes + 1024;  // + alignment slack
+    static constexpr int kChunksPerRow = kRowBytes / 16;
+    static constexpr int kRowsPerInst = 32 / kChunksPerRow;         // rows one warp-wide cp.async covers
+    static_assert(kRowBytes % 128 == 0, "rows must be whole 128-byte columns");
+    static_assert(kStageBytes % 1024 == 0 && kQSlot % 1024 == 0, "1024-byte stage alignment");
+    static_assert(kWarps <= kMaxWarpsPerCta, "workspace sizing");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -194,8 +218,8 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
-// Zero rows [valid, 16) of a K or V tile (NSUB boxes of 16 x 128 B).  Used on
-// a sequence's last tile so the unused slots (never written, any bits) cannot
+// Zero rows [valid, 16) of a V tile (NSUB columns of 16 x 128 B).  Used on a
+// sequence's last tile so the unused slots (never written, any bits) cannot
 // reach the tensor-core P.V product.
 template <int kNSub>
 __device__ __forceinline__ void zero_tail_rows(uint8_t* tile, int valid, int lane) {
@@ -209,12 +233,34 @@ __device__ __forceinline__ void zero_tail_rows(uint8_t* tile, int valid, int lan
     __syncwarp();
 }
 
-// Swizzled byte offset of 16-byte chunk `c` (of the whole row) in row t.
+// Swizzled byte offset of 16-byte chunk `c` (of the whole row) of token row t
+// in a tile: column c/8, line t, chunk (c%8) XOR (t%8) -- conflict-free for
+// the ldmatrix / 16-byte shared loads below and for the cp.async writes.
 __device__ __forceinline__ uint32_t sw_off(int t, int c) {
     return (uint32_t)((c >> 3) * kSubBytes + t * 128 + ((((c & 7) ^ t) & 7) << 4));
 }
 
-// ---- 16-bit caches (f16 / bf16) and FP8 caches: tensor-core consumer --------
+// Output / workspace sink of one unit segment.
+struct Sink {
+    bool split;
+    int64_t seg;   // workspace segment (split only)
+    int64_t row0;  // output row (s * Hq + first head of the chunk)
+    int nh;
+};
+
+template <typename QT>
+__device__ __forceinline__ void sink_write(const DecodeParams& p, const Sink& k, int D, int h, int d,
+                                           float o, float l, float vscale) {
+    if (h >= k.nh) return;
+    if (!k.split) {
+        QT* out = reinterpret_cast<QT*>(p.out) + (k.row0 + h) * D + d;
+        *out = from_f32<QT>(l > 0.f ? o * vscale / l : 0.f);
+    } else {
+        p.ws_o[(k.seg * p.hpu + h) * D + d] = o * vscale;
+    }
+}
+
+// ---- 16-bit caches (f16 / bf16) and FP8 caches: tensor-core tile math --------
 template <class C>
 struct MmaConsumer {
     static constexpr bool kFp8 = C::kPath == Path::kFp8;
@@ -294,10 +340,10 @@ struct MmaConsumer {
             }
         } else {
             // K rows gid and gid+8, bytes [32*tig, 32*tig+32): two chunks each.
-            uint4 r0a = *reinterpret_cast<const uint4*>(kt + sw_off(gid, 2 * tig));
-            uint4 r0b = *reinterpret_cast<const uint4*>(kt + sw_off(gid, 2 * tig + 1));
-            uint4 r1a = *reinterpret_cast<const uint4*>(kt + sw_off(gid + 8, 2 * tig));
-            uint4 r1b = *reinterpret_cast<const uint4*>(kt + sw_off(gid + 8, 2 * tig + 1));
+            const uint4 r0a = *reinterpret_cast<const uint4*>(kt + sw_off(gid, 2 * tig));
+            const uint4 r0b = *reinterpret_cast<const uint4*>(kt + sw_off(gid, 2 * tig + 1));
+            const uint4 r1a = *reinterpret_cast<const uint4*>(kt + sw_off(gid + 8, 2 * tig));
+            const uint4 r1b = *reinterpret_cast<const uint4*>(kt + sw_off(gid + 8, 2 * tig + 1));
             const uint32_t w0[8] = {r0a.x, r0a.y, r0a.z, r0a.w, r0b.x, r0b.y, r0b.z, r0b.w};
             const uint32_t w1[8] = {r1a.x, r1a.y, r1a.z, r1a.w, r1b.x, r1b.y, r1b.z, r1b.w};
 #pragma unroll
@@ -326,12 +372,28 @@ struct MmaConsumer {
         const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
         m0 = mn0;
         m1 = mn1;
-        constexpr bool kPBf16 = kOpBf16;  // P uses the operand type of the V product
-        const uint32_t X0 = pack2<kPBf16>(ex2(x0 - mn0), ex2(x1 - mn1));
-        const uint32_t X1 = pack2<kPBf16>(ex2(x2 - mn0), ex2(x3 - mn1));
-        const float2 p0 = unpack2<kPBf16>(X0), p1 = unpack2<kPBf16>(X1);
-        l0 = l0 * al0 + p0.x + p1.x;  // normaliser from the rounded P actually used
-        l1 = l1 * al1 + p0.y + p1.y;
+        // P goes to the tensor core in the V operand's 16-bit type.  bf16 keeps
+        // only 8 significant bits, so for bf16 caches P is carried as
+        // hi + lo bf16 parts (two products, ~16 significant bits): the P.V sum
+        // then matches fp32 P to well inside the tolerance.  f16 (11 bits) and
+        // the FP8 path (f16) use one part.
+        const float e0 = ex2(x0 - mn0), e1 = ex2(x1 - mn1), e2 = ex2(x2 - mn0), e3 = ex2(x3 - mn1);
+        const uint32_t X0 = pack2<kOpBf16>(e0, e1);
+        const uint32_t X1 = pack2<kOpBf16>(e2, e3);
+        uint32_t c0 = 0, c1 = 0;
+        if constexpr (kOpBf16) {
+            const float2 h0 = unpack2<true>(X0), h1 = unpack2<true>(X1);
+            const uint32_t Y0 = pack2<true>(e0 - h0.x, e1 - h0.y);
+            const uint32_t Y1 = pack2<true>(e2 - h1.x, e3 - h1.y);
+            c0 = movm_trans(Y0);
+            c1 = movm_trans(Y1);
+            l0 = l0 * al0 + (e0 + e2);
+            l1 = l1 * al1 + (e1 + e3);
+        } else {
+            const float2 p0 = unpack2<false>(X0), p1 = unpack2<false>(X1);
+            l0 = l0 * al0 + p0.x + p1.x;  // normaliser from the rounded P actually used
+            l1 = l1 * al1 + p0.y + p1.y;
+        }
         const uint32_t b0 = movm_trans(X0), b1 = movm_trans(X1);  // P^T as mma B
 #pragma unroll
         for (int mi = 0; mi < MT; ++mi) {
@@ -345,6 +407,7 @@ struct MmaConsumer {
                 uint32_t a[4];
                 ldsm_x4_trans(a, vb + sw_off(t, 2 * mi + (mtx & 1)));
                 mma16816<kOpBf16>(acc[mi], a, b0, b1);
+                if constexpr (kOpBf16) mma16816<true>(acc[mi], a, c0, c1);
             }
         } else {
             // V^T fragments: thread gid owns d in [16*gid, 16*gid+16) (one chunk),
@@ -375,8 +438,9 @@ struct MmaConsumer {
         }
     }
 
-    // Warp partial -> shared scratch: acc[w][head][d], ml[w][head].
-    __device__ void store(float* scr, float2* ml, int warp) {
+    // End of a unit segment: the output (whole unit) or a partial (split).
+    __device__ void finish(const DecodeParams& p, const Sink& k, float vscale) {
+        using QT = typename C::q_t;
         const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
         float a0 = l0, a1 = l1;
 #pragma unroll
@@ -384,24 +448,25 @@ struct MmaConsumer {
             a0 += __shfl_xor_sync(kFull, a0, o);
             a1 += __shfl_xor_sync(kFull, a1, o);
         }
-        float* s0 = scr + (warp * kHeadsPerUnit + 2 * tig) * C::kScrStride;
-        float* s1 = s0 + C::kScrStride;
+        const int h0 = 2 * tig, h1 = 2 * tig + 1;
 #pragma unroll
         for (int mi = 0; mi < MT; ++mi) {
             int d0, d1;
             if constexpr (!kFp8) { d0 = 16 * mi + gid; d1 = d0 + 8; }
             else { d0 = 16 * gid + 2 * mi; d1 = d0 + 1; }
-            s0[d0] = acc[mi][0]; s1[d0] = acc[mi][1];
-            s0[d1] = acc[mi][2]; s1[d1] = acc[mi][3];
+            sink_write<QT>(p, k, D, h0, d0, acc[mi][0], a0, vscale);
+            sink_write<QT>(p, k, D, h1, d0, acc[mi][1], a1, vscale);
+            sink_write<QT>(p, k, D, h0, d1, acc[mi][2], a0, vscale);
+            sink_write<QT>(p, k, D, h1, d1, acc[mi][3], a1, vscale);
         }
-        if (gid == 0) {
-            ml[warp * kHeadsPerUnit + 2 * tig] = make_float2(m0, a0);
-            ml[warp * kHeadsPerUnit + 2 * tig + 1] = make_float2(m1, a1);
+        if (k.split && gid == 0) {
+            if (h0 < k.nh) p.ws_ml[k.seg * p.hpu + h0] = make_float2(m0, a0);
+            if (h1 < k.nh) p.ws_ml[k.seg * p.hpu + h1] = make_float2(m1, a1);
         }
     }
 };
 
-// ---- fp32 caches: CUDA-core consumer ----------------------------------------
+// ---- fp32 caches: CUDA-core tile math ---------------------------------------
 template <class C>
 struct F32Consumer {
     static constexpr int D = C::D;
@@ -492,7 +557,7 @@ struct F32Consumer {
             }
         }
     }
-    __device__ void store(float* scr, float2* ml, int warp) {
+    __device__ void finish(const DecodeParams& p, const Sink& k, float vscale) {
         const int lane = threadIdx.x & 31, c = lane % CPR, rh = lane / CPR;
 #pragma unroll
         for (int h = 0; h < kHeadsPerUnit; ++h) {
@@ -504,9 +569,13 @@ struct F32Consumer {
                 a.x += __shfl_xor_sync(kFull, a.x, 16); a.y += __shfl_xor_sync(kFull, a.y, 16);
                 a.z += __shfl_xor_sync(kFull, a.z, 16); a.w += __shfl_xor_sync(kFull, a.w, 16);
             }
-            if (rh == 0)
-                *reinterpret_cast<float4*>(scr + (warp * kHeadsPerUnit + h) * C::kScrStride + 4 * c) = a;
-            if (lane == 0) ml[warp * kHeadsPerUnit + h] = make_float2(m[h], ls);
+            if (rh == 0) {
+                sink_write<float>(p, k, D, h, 4 * c + 0, a.x, ls, vscale);
+                sink_write<float>(p, k, D, h, 4 * c + 1, a.y, ls, vscale);
+                sink_write<float>(p, k, D, h, 4 * c + 2, a.z, ls, vscale);
+                sink_write<float>(p, k, D, h, 4 * c + 3, a.w, ls, vscale);
+            }
+            if (k.split && lane == 0 && h < k.nh) p.ws_ml[k.seg * p.hpu + h] = make_float2(m[h], ls);
         }
     }
 };
@@ -515,276 +584,199 @@ template <class C>
 using ConsumerOf = typename std::conditional<C::kPath == Path::kF32, F32Consumer<C>, MmaConsumer<C>>::type;
 
 // ----------------------------------------------------------------------------
-// The kernel.
+// Block-table prefetcher of one warp: entries [base, base+64) of the current
+// sequence's row in two registers per lane, the second batch fetched while
+// the first is in use.
+// ----------------------------------------------------------------------------
+struct TablePrefetch {
+    int s = -1, base = 0, cur = 0, nxt = 0;
+
+    __device__ int get(const DecodeParams& p, int seq, int b, int nblk, int lane) {
+        const int32_t* row = p.block_tables + (int64_t)seq * p.max_blocks_per_seq;
+        if (seq != s || b < base || b >= base + 64) {
+            s = seq;
+            base = b;
+            cur = (b + lane < nblk) ? __ldg(row + b + lane) : 0;
+            nxt = (b + 32 + lane < nblk) ? __ldg(row + b + 32 + lane) : 0;
+        } else if (b >= base + 32) {
+            base += 32;
+            cur = nxt;
+            nxt = (base + 32 + lane < nblk) ? __ldg(row + base + 32 + lane) : 0;
+        }
+        return __shfl_sync(kFull, cur, b - base);
+    }
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Issue the async loads of the walk's current tile (and, on a unit's first
+// tile, of its q rows) into stage `stg` / q slot `qslot`.
+template <class C>
+__device__ __forceinline__ void issue_tile(const DecodeParams& p, const Walk& w, TablePrefetch& tp,
+                                           uint8_t* stg, uint8_t* qslot) {
+    const int lane = threadIdx.x & 31;
+    const int kh = w.j / p.nch, c = w.j % p.nch;
+    const int tok = w.i * kTileTokens;
+    const int nblk = (w.L + p.block_size - 1) / p.block_size;
+    int phys = tp.get(p, w.s, tok / p.block_size, nblk, lane);
+    if (phys < 0 || phys >= p.num_blocks) {
+        if (lane == 0) raise_error(p.err, PKV_DEVERR_BLOCK_ID);
+        phys = 0;
+    }
+    const int tok0 = tok % p.block_size;
+    const int64_t row_stride = (int64_t)p.num_kv_heads * C::kRowBytes;  // bytes between tokens
+    const int64_t base = (((int64_t)phys * p.block_size + tok0) * p.num_kv_heads + kh) * C::kRowBytes;
+    const uint8_t* ksrc = p.key_cache + base;
+    const uint8_t* vsrc = p.value_cache + base;
+    const uint32_t kdst = smem_u32(stg), vdst = smem_u32(stg + C::kTensorTile);
+    const int cr = lane % C::kChunksPerRow, r0 = lane / C::kChunksPerRow;
+#pragma unroll
+    for (int it = 0; it < kTileTokens / C::kRowsPerInst; ++it) {
+        const int t = it * C::kRowsPerInst + r0;
+        const int64_t off = t * row_stride + cr * 16;
+        const uint32_t so = sw_off(t, cr);
+        cp_async16(kdst + so, ksrc + off);
+        cp_async16(vdst + so, vsrc + off);
+    }
+    if (w.first()) {
+        const int nh = min(kHeadsPerUnit, p.g - kHeadsPerUnit * c);
+        const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q) +
+            ((int64_t)w.s * p.num_heads + (int64_t)kh * p.g + kHeadsPerUnit * c) * C::D * C::kQBytes;
+        const int chunks = nh * C::D * C::kQBytes / 16;
+        for (int ch = lane; ch < chunks; ch += 32) cp_async16(smem_u32(qslot + ch * 16), qsrc + ch * 16);
+    }
+}
+
+// ----------------------------------------------------------------------------
+// The kernel: every warp is an independent worker.
 // ----------------------------------------------------------------------------
 template <class C>
-__global__ void __launch_bounds__(kThreads, 1)
-pkv_decode_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                  const DecodeParams p) {
+__global__ void __launch_bounds__(C::kWarps * 32, 1)
+pkv_decode_kernel(const DecodeParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t* stages = smem + C::kOffStages;
-    uint8_t* qslots = smem + C::kOffQ;
-    float* scr = reinterpret_cast<float*>(smem + C::kOffScr);
-    float2* scr_ml = reinterpret_cast<float2*>(smem + C::kOffMl);
-    const uint32_t bar0 = smem_u32(smem + C::kOffBar);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffAbort);
-    auto full_bar = [&](int i) { return bar0 + 8u * i; };
-    auto empty_bar = [&](int i) { return bar0 + 8u * (C::kStages + i); };
-    auto qfull_bar = [&](int i) { return bar0 + 8u * (2 * C::kStages + i); };
-    auto qempty_bar = [&](int i) { return bar0 + 8u * (2 * C::kStages + 2 + i); };
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < C::kStages; ++i) {
-            mbar_init(full_bar(i), 1);
-            mbar_init(empty_bar(i), 1);
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(qfull_bar(i), 1);
-            mbar_init(qempty_bar(i), kConsumerWarps);
-        }
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    __syncthreads();
+    uint8_t* stages = smem + warp * C::kWarpBytes;
+    uint8_t* qslots = stages + C::kStages * C::kStageBytes;
 
-    const int units_per_seq = p.num_kv_heads * p.nch;
+    const int units = p.num_kv_heads * p.nch;
     const int cap = p.max_blocks_per_seq * p.block_size;
+    const int64_t workers = (int64_t)gridDim.x * C::kWarps;
+    const int64_t wid = (int64_t)blockIdx.x * C::kWarps + warp;
+    bool bad_len = false;
+    const int64_t W = total_tiles(p.seq_lens, p.num_seqs, units, cap, &bad_len);
+    if (bad_len && wid == 0 && lane == 0) raise_error(p.err, PKV_DEVERR_SEQ_LEN);
+    const int64_t chunk = (W + workers - 1) / workers;
+    const int64_t tb = min(W, wid * chunk), te = min(W, tb + chunk);
+    if (tb >= te) return;
 
-    if (warp == kConsumerWarps) {
-        // ======================= producer warp =======================
-        if (lane == 0) { prefetch_tensormap(&tmk); prefetch_tensormap(&tmv); }
-        bool bad_len = false;
-        const int64_t W = total_tiles(p.seq_lens, p.num_seqs, units_per_seq, cap, &bad_len);
-        if (bad_len && blockIdx.x == 0 && lane == 0) raise_error(p.err, PKV_DEVERR_SEQ_LEN);
-        const int64_t chunk = (W + gridDim.x - 1) / gridDim.x;
-        const int64_t tb = min(W, (int64_t)blockIdx.x * chunk), te = min(W, tb + chunk);
-        const int tpb = p.block_size / kTileTokens;
-        uint32_t n = 0;
-        int k = 0;
-        bool ok = true;
-        if (tb < te) {
-            SeqHit hit = find_seq(p.seq_lens, p.num_seqs, units_per_seq, cap, tb);
-            int s = hit.s, L = hit.L, nt = ntiles_of(L);
-            int64_t base = hit.base;
-            int j = (int)((tb - base) / nt);
-            int i0 = (int)((tb - base) % nt);
-            while (ok) {
-                const int64_t T0 = base + (int64_t)j * nt;
-                if (T0 >= te) break;
-                const int i1 = (int)min((int64_t)nt, te - T0);
-                const int kh = j / p.nch, c = j % p.nch;
-                const int nh = min(kHeadsPerUnit, p.g - kHeadsPerUnit * c);
-                const int u = (s * p.num_kv_heads + kh) * p.nch + c;
-                // ---- unit header + q rows
-                const int slot = k & 1;
-                ok = mbar_wait_bounded(qempty_bar(slot), ((k >> 1) & 1) ^ 1, abort_flag);
-                if (!ok) break;
-                if (lane == 0) {
-                    UnitHeader* hd = reinterpret_cast<UnitHeader*>(qslots + slot * C::kQSlot);
-                    hd->s = s; hd->kh = kh; hd->c = c; hd->nh = nh; hd->L = L;
-                    hd->i0 = i0; hd->i1 = i1;
-                    hd->split = (i0 != 0 || i1 != nt) ? 1 : 0;
-                    hd->seg = (int)blockIdx.x + u;
-                    hd->done = 0;
-                    const uint32_t qbytes = (uint32_t)(nh * C::D * C::kQBytes);
-                    const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q) +
-                        ((int64_t)s * p.num_heads + (int64_t)kh * p.g + kHeadsPerUnit * c) * C::D * C::kQBytes;
-                    mbar_arrive_expect_tx(qfull_bar(slot), qbytes);
-                    bulk_load(smem_u32(qslots + slot * C::kQSlot + 128), qsrc, qbytes, qfull_bar(slot));
-                }
-                ++k;
-                // ---- tiles
-                const int32_t* trow = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
-                const int nblk = (L + p.block_size - 1) / p.block_size;
-                int cbase = -64, creg = 0;
-                for (int i = i0; i < i1; ++i) {
-                    const int b = i / tpb;
-                    if (b - cbase >= 32) {
-                        cbase = b;
-                        creg = (b + lane < nblk) ? __ldg(trow + b + lane) : 0;
-                    }
-                    int phys = __shfl_sync(kFull, creg, b - cbase);
-                    if (phys < 0 || phys >= p.num_blocks) {
-                        if (lane == 0) raise_error(p.err, PKV_DEVERR_BLOCK_ID);
-                        phys = 0;
-                    }
-                    const int tok0 = (i % tpb) * kTileTokens;
-                    const int st = (int)(n % C::kStages);
-                    ok = mbar_wait_bounded(empty_bar(st), ((n / C::kStages) & 1) ^ 1, abort_flag);
-                    if (!ok) break;
-                    if (lane == 0) {
-                        uint8_t* kt = stages + st * C::kStageBytes;
-                        uint8_t* vt = kt + C::kTensorTile;
-                        mbar_arrive_expect_tx(full_bar(st), C::kStageBytes);
-#pragma unroll
-                        for (int sub = 0; sub < C::kNSub; ++sub)
-                            tma_load_4d(smem_u32(kt + sub * kSubBytes), &tmk, full_bar(st),
-                                        sub * C::kBoxElems, kh, tok0, phys);
-#pragma unroll
-                        for (int sub = 0; sub < C::kNSub; ++sub)
-                            tma_load_4d(smem_u32(vt + sub * kSubBytes), &tmv, full_bar(st),
-                                        sub * C::kBoxElems, kh, tok0, phys);
-                    }
-                    ++n;
-                }
-                if (!ok) break;
-                // ---- next unit
-                i0 = 0;
-                if (++j == units_per_seq) {
-                    j = 0;
-                    base += (int64_t)units_per_seq * nt;
-                    do {
-                        ++s;
-                        if (s >= p.num_seqs) break;
-                        L = clamp_len(__ldg(p.seq_lens + s), cap);
-                        nt = ntiles_of(L);
-                    } while (nt == 0);
-                    if (s >= p.num_seqs) break;
-                }
-            }
-        }
-        if (ok) {
-            const int slot = k & 1;
-            ok = mbar_wait_bounded(qempty_bar(slot), ((k >> 1) & 1) ^ 1, abort_flag);
-            if (ok && lane == 0) {
-                reinterpret_cast<UnitHeader*>(qslots + slot * C::kQSlot)->done = 1;
-                mbar_arrive(qfull_bar(slot));
-            }
-        }
-        if (!ok && lane == 0) raise_error(p.err, PKV_DEVERR_TIMEOUT);
-        return;
+    Walk iw, cw;  // issue walk (runs kStages-1 tiles ahead) and compute walk
+    iw.init(p.seq_lens, p.num_seqs, units, cap, tb, te);
+    cw = iw;
+    TablePrefetch tp;
+#pragma unroll 1
+    for (int k = 0; k < C::kStages - 1; ++k) {
+        if (!iw.done)
+            issue_tile<C>(p, iw, tp, stages + k * C::kStageBytes, qslots + (iw.ord % C::kStages) * C::kQSlot);
+        cp_async_commit();
+        iw.advance(p.seq_lens, p.num_seqs, units, cap);
     }
-
-    // ======================= consumer warps =======================
-    ConsumerOf<C> cs;
-    constexpr int kCT = kConsumerWarps * 32;
-    const int ctid = threadIdx.x;
     const float kscale = (C::kPath == Path::kFp8 && p.k_scale) ? __ldg(p.k_scale) : 1.f;
     const float vscale = (C::kPath == Path::kFp8 && p.v_scale) ? __ldg(p.v_scale) : 1.f;
-    uint32_t n0 = 0;
-    for (int k = 0;; ++k) {
-        const int slot = k & 1;
-        const bool got = mbar_wait_bounded(qfull_bar(slot), (k >> 1) & 1, abort_flag);
-        const UnitHeader* hd = reinterpret_cast<const UnitHeader*>(qslots + slot * C::kQSlot);
-        const bool stop = bar_sync_or(1, kCT, !got || hd->done);
-        if (stop) break;
-        const UnitHeader h = *hd;
-        cs.load_q(qslots + slot * C::kQSlot + 128, h.nh, p.scale_log2, kscale);
-        cs.reset();
+    ConsumerOf<C> cs;
+#pragma unroll 1
+    for (int n = 0; !cw.done; ++n) {
+        if (!iw.done)
+            issue_tile<C>(p, iw, tp, stages + ((n + C::kStages - 1) % C::kStages) * C::kStageBytes,
+                          qslots + (iw.ord % C::kStages) * C::kQSlot);
+        cp_async_commit();
+        iw.advance(p.seq_lens, p.num_seqs, units, cap);
+        cp_async_wait<C::kStages - 1>();
         __syncwarp();
-        if (lane == 0) mbar_arrive(qempty_bar(slot));
-        const int ntile = h.i1 - h.i0;
-        bool bad = false;
-        for (int jt = warp; jt < ntile; jt += kConsumerWarps) {
-            const uint32_t n = n0 + (uint32_t)jt;
-            const int st = (int)(n % C::kStages);
-            if (!mbar_wait_bounded(full_bar(st), (n / C::kStages) & 1, abort_flag)) { bad = true; break; }
-            uint8_t* kt = stages + st * C::kStageBytes;
-            const int tokb = (h.i0 + jt) * kTileTokens;
-            cs.tile(kt, kt + C::kTensorTile, min(kTileTokens, h.L - tokb));
-            fence_proxy_async_smem();  // generic writes (tail zeroing) before TMA reuse
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty_bar(st));
+        const int kh = cw.j / p.nch, c = cw.j % p.nch;
+        const int nh = min(kHeadsPerUnit, p.g - kHeadsPerUnit * c);
+        if (cw.first()) {
+            cs.load_q(qslots + (cw.ord % C::kStages) * C::kQSlot, nh, p.scale_log2, kscale);
+            cs.reset();
         }
-        n0 += (uint32_t)ntile;
-        if (bar_sync_or(1, kCT, bad)) break;
-        // ---- merge the warps' partial states
-        cs.store(scr, scr_ml, warp);
-        bar_sync(1, kCT);
-        const int D = C::D;
-        for (int idx = ctid; idx < h.nh * D; idx += kCT) {
-            const int hh = idx / D, d = idx % D;
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, scr_ml[w * kHeadsPerUnit + hh].x);
-            float ls = 0.f, o = 0.f;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) {
-                const float2 ml = scr_ml[w * kHeadsPerUnit + hh];
-                const float f = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M);
-                ls += ml.y * f;
-                o += scr[(w * kHeadsPerUnit + hh) * C::kScrStride + d] * f;
-            }
-            o *= vscale;
-            if (!h.split) {
-                using QT = typename C::q_t;
-                QT* out = reinterpret_cast<QT*>(p.out) +
-                          ((int64_t)h.s * p.num_heads + (int64_t)h.kh * p.g + kHeadsPerUnit * h.c + hh) * D + d;
-                *out = from_f32<QT>(ls > 0.f ? o / ls : 0.f);
-            } else {
-                p.ws_o[((int64_t)h.seg * p.hpu + hh) * D + d] = o;
-                if (d == 0) p.ws_ml[(int64_t)h.seg * p.hpu + hh] = make_float2(M, ls);
-            }
+        uint8_t* kt = stages + (n % C::kStages) * C::kStageBytes;
+        cs.tile(kt, kt + C::kTensorTile, min(kTileTokens, cw.L - cw.i * kTileTokens));
+        if (cw.last()) {
+            Sink k;
+            k.split = (cw.seg_i0 != 0) || (cw.i != cw.nt - 1);
+            k.seg = wid + ((int64_t)cw.s * p.num_kv_heads + kh) * p.nch + c;
+            k.row0 = (int64_t)cw.s * p.num_heads + (int64_t)kh * p.g + kHeadsPerUnit * c;
+            k.nh = nh;
+            cs.finish(p, k, vscale);
         }
-        bar_sync(1, kCT);
+        __syncwarp();  // every lane is done with this stage before it is refilled
+        cw.advance(p.seq_lens, p.num_seqs, units, cap);
     }
+    cp_async_wait<0>();
 }
 
 // ----------------------------------------------------------------------------
 // Exact merge of split units (zwxr.cn 3.3: M = max m_p,
 // out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p) and zero output for
-// empty sequences.  CTA b >= 1 owns the unit cut by boundary b (if it is the
-// unit's first interior boundary); CTA 0 zeroes empty sequences.
+// empty sequences.  Warp b >= 1 (global) owns the unit cut by worker
+// boundary b if that is the unit's first interior boundary; warp 0 zeroes the
+// empty sequences.  Partials are combined in worker order.
 // ----------------------------------------------------------------------------
-template <typename QT>
+template <typename QT, int D>
 __global__ void __launch_bounds__(256)
-pkv_merge_kernel(const DecodeParams p, int D) {
-    __shared__ int sh[8];
-    const int units_per_seq = p.num_kv_heads * p.nch;
+pkv_merge_kernel(const DecodeParams p, int64_t workers) {
+    const int lane = threadIdx.x & 31;
+    const int64_t b = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int units = p.num_kv_heads * p.nch;
     const int cap = p.max_blocks_per_seq * p.block_size;
-    const int G = gridDim.x;
-    if (blockIdx.x == 0) {
-        // rare: a thread per empty sequence writes its zero rows
-        for (int s = threadIdx.x; s < p.num_seqs; s += blockDim.x) {
+    if (b == 0) {
+        for (int s = 0; s < p.num_seqs; ++s) {
             if (clamp_len(__ldg(p.seq_lens + s), cap) != 0) continue;
             QT* out = reinterpret_cast<QT*>(p.out) + (int64_t)s * p.num_heads * D;
-            for (int i = 0; i < p.num_heads * D; ++i) out[i] = from_f32<QT>(0.f);
+            for (int i = lane; i < p.num_heads * D; i += 32) out[i] = from_f32<QT>(0.f);
         }
         return;
     }
-    if (threadIdx.x < 32) {
-        int flag = 0, s = 0, j = 0, bf = 0, bl = 0;
-        const int64_t W = total_tiles(p.seq_lens, p.num_seqs, units_per_seq, cap);
-        const int64_t chunk = (W + G - 1) / G;
-        const int64_t P = (int64_t)blockIdx.x * chunk;
-        if (P < W) {
-            const SeqHit hit = find_seq(p.seq_lens, p.num_seqs, units_per_seq, cap, P);
-            const int nt = ntiles_of(hit.L);
-            j = (int)((P - hit.base) / nt);
-            const int off = (int)((P - hit.base) % nt);
-            const int64_t T0 = hit.base + (int64_t)j * nt;
-            if (off != 0 && (int64_t)(blockIdx.x - 1) * chunk <= T0) {
-                flag = 1;
-                s = hit.s;
-                bf = (int)(T0 / chunk);
-                bl = (int)((T0 + nt - 1) / chunk);
-            }
-        }
-        if (threadIdx.x == 0) { sh[0] = flag; sh[1] = s; sh[2] = j; sh[3] = bf; sh[4] = bl; }
-    }
-    __syncthreads();
-    if (!sh[0]) return;
-    const int s = sh[1], j = sh[2], bf = sh[3], bl = sh[4];
+    if (b >= workers) return;
+    const int64_t W = total_tiles(p.seq_lens, p.num_seqs, units, cap);
+    const int64_t chunk = (W + workers - 1) / workers;
+    const int64_t P = b * chunk;
+    if (P >= W) return;
+    const SeqHit hit = find_seq(p.seq_lens, p.num_seqs, units, cap, P);
+    const int nt = ntiles_of(hit.L);
+    const int j = (int)((P - hit.base) / nt);
+    const int off = (int)((P - hit.base) % nt);
+    const int64_t T0 = hit.base + (int64_t)j * nt;
+    if (off == 0 || (b - 1) * chunk > T0) return;   // not an interior first boundary
+    const int64_t bf = T0 / chunk, bl = (T0 + nt - 1) / chunk;
     const int kh = j / p.nch, c = j % p.nch;
     const int nh = min(kHeadsPerUnit, p.g - kHeadsPerUnit * c);
-    const int u = (s * p.num_kv_heads + kh) * p.nch + c;
-    for (int idx = threadIdx.x; idx < nh * D; idx += blockDim.x) {
-        const int hh = idx / D, d = idx % D;
+    const int64_t u = ((int64_t)hit.s * p.num_kv_heads + kh) * p.nch + c;
+    const int64_t row0 = (int64_t)hit.s * p.num_heads + (int64_t)kh * p.g + kHeadsPerUnit * c;
+    constexpr int PER = D / 32;
+    for (int h = 0; h < nh; ++h) {
         float M = -INFINITY;
-        for (int b = bf; b <= bl; ++b) M = fmaxf(M, p.ws_ml[(int64_t)(b + u) * p.hpu + hh].x);
-        float ls = 0.f, o = 0.f;
-        for (int b = bf; b <= bl; ++b) {
-            const float2 ml = p.ws_ml[(int64_t)(b + u) * p.hpu + hh];
+        for (int64_t w = bf; w <= bl; ++w) M = fmaxf(M, p.ws_ml[(w + u) * p.hpu + h].x);
+        float ls = 0.f, o[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[e] = 0.f;
+        for (int64_t w = bf; w <= bl; ++w) {
+            const float2 ml = p.ws_ml[(w + u) * p.hpu + h];
             const float f = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M);
             ls += ml.y * f;
-            o += p.ws_o[((int64_t)(b + u) * p.hpu + hh) * D + d] * f;
+            const float* src = p.ws_o + ((w + u) * p.hpu + h) * D;
+#pragma unroll
+            for (int e = 0; e < PER; ++e) o[e] += src[lane + 32 * e] * f;
         }
-        QT* out = reinterpret_cast<QT*>(p.out) +
-                  ((int64_t)s * p.num_heads + (int64_t)kh * p.g + kHeadsPerUnit * c + hh) * D + d;
-        *out = from_f32<QT>(ls > 0.f ? o / ls : 0.f);
+        QT* out = reinterpret_cast<QT*>(p.out) + (row0 + h) * D;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) out[lane + 32 * e] = from_f32<QT>(ls > 0.f ? o[e] / ls : 0.f);
     }
 }
 

@@ -1,8 +1,6 @@
 // pkv_api.cu -- host side of pkv_paged_attention_decode and the library
-// utilities: argument validation, TMA descriptor encoding, variant dispatch,
-// the device error word and the host-buffer decode step.
-#include <cudaTypedefs.h>
-
+// utilities: argument validation, variant dispatch, workspace layout, the
+// device error word and the host-buffer decode step.
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -23,18 +21,6 @@ constexpr int kMaxDevices = 64;
 int* g_err_ptr[kMaxDevices] = {nullptr};
 std::mutex g_err_mu;
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
 }  // namespace
 
 pkv_status fail(pkv_status st, const char* fmt, ...) {
@@ -66,32 +52,6 @@ int* device_error_word() {
     return g_err_ptr[dev];
 }
 
-// 4-D tiled map over a cache [NB, bs, Hkv, D]: dims (D, Hkv, bs, NB), box
-// (128 bytes of D, 1 head, 16 tokens, 1 block), 128-byte swizzle.
-static pkv_status encode_cache_map(CUtensorMap* map, const void* base, pkv_dtype dt, int64_t nb,
-                                   int bs, int hkv, int d) {
-    auto fn = encode_fn();
-    if (!fn) return fail(PKV_ECUDA, "cuTensorMapEncodeTiled unavailable");
-    const int es = dtype_bytes(dt);
-    CUtensorMapDataType t;
-    switch (dt) {
-    case PKV_F32: t = CU_TENSOR_MAP_DATA_TYPE_FLOAT32; break;
-    case PKV_F16: t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16; break;
-    case PKV_BF16: t = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; break;
-    default: t = CU_TENSOR_MAP_DATA_TYPE_UINT8; break;
-    }
-    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)hkv, (cuuint64_t)bs, (cuuint64_t)nb};
-    const cuuint64_t strides[3] = {(cuuint64_t)d * es, (cuuint64_t)hkv * d * es,
-                                   (cuuint64_t)bs * hkv * d * es};
-    const cuuint32_t box[4] = {(cuuint32_t)(128 / es), 1u, (cuuint32_t)kTileTokens, 1u};
-    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-    const CUresult r = fn(map, t, 4, const_cast<void*>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(PKV_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-    return PKV_OK;
-}
-
 static int default_ctas() {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -113,7 +73,8 @@ static bool ws_layout(int num_seqs, int num_heads, int num_kv_heads, int head_di
     if (w->grid <= 0) return false;
     w->nch = (g + kHeadsPerUnit - 1) / kHeadsPerUnit;
     w->hpu = g < kHeadsPerUnit ? g : kHeadsPerUnit;
-    const size_t segs = (size_t)w->grid + (size_t)num_seqs * num_kv_heads * w->nch;
+    // one segment per worker (up to kMaxWarpsPerCta warps per CTA) plus one per unit
+    const size_t segs = (size_t)w->grid * kMaxWarpsPerCta + (size_t)num_seqs * num_kv_heads * w->nch;
     w->o_bytes = segs * w->hpu * head_dim * sizeof(float);
     w->ml_off = (w->o_bytes + 255) & ~(size_t)255;
     w->total = w->ml_off + segs * w->hpu * sizeof(float2);
@@ -180,18 +141,11 @@ extern "C" pkv_status pkv_paged_attention_decode(void* out, const void* query, p
     int* err = device_error_word();
     if (!err) return fail(PKV_ECUDA, "device error word unavailable");
 
-    CUtensorMap tmk, tmv;
-    pkv_status st;
-    if ((st = encode_cache_map(&tmk, key_cache, cache_dtype, num_blocks, block_size, num_kv_heads,
-                               head_dim)) != PKV_OK)
-        return st;
-    if ((st = encode_cache_map(&tmv, value_cache, cache_dtype, num_blocks, block_size, num_kv_heads,
-                               head_dim)) != PKV_OK)
-        return st;
-
     DecodeParams p;
     p.out = out;
     p.q = query;
+    p.key_cache = static_cast<const uint8_t*>(key_cache);
+    p.value_cache = static_cast<const uint8_t*>(value_cache);
     p.block_tables = block_tables;
     p.seq_lens = seq_lens;
     p.k_scale = cache_dtype == PKV_FP8_E4M3 ? k_scale : nullptr;
@@ -209,7 +163,7 @@ extern "C" pkv_status pkv_paged_attention_decode(void* out, const void* query, p
     p.block_size = block_size;
     p.num_blocks = (int)num_blocks;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
-    DecodeLaunchArgs a{&p, &tmk, &tmv, w.grid};
+    DecodeLaunchArgs a{&p, w.grid};
     return launch(a, reinterpret_cast<cudaStream_t>(stream));
 }
 

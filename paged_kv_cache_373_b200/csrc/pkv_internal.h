@@ -23,9 +23,7 @@ struct DecodeParams;  // paged_attention.cuh
 
 struct DecodeLaunchArgs {
     const DecodeParams* params;
-    const CUtensorMap* tmk;
-    const CUtensorMap* tmv;
-    int grid;
+    int grid;  // CTAs of the persistent grid
 };
 
 // One launcher per kernel variant (attn_*.cu).
