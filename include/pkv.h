@@ -176,6 +176,45 @@ pkv_status pkv_paged_attention_decode(void* out, const void* query, pkv_dtype q_
                                       void* workspace, size_t workspace_bytes, int num_ctas,
                                       pkv_stream_t stream);
 
+/* Size of the static scratch used by pkv_paged_attention_decode_noalloc. */
+#define PKV_STATIC_WORKSPACE_BYTES (8u * 1024u * 1024u)
+
+/*
+ * pkv_paged_attention_decode_noalloc -- pkv_paged_attention_decode with no
+ * workspace argument.  The pages have no counterpart: this entry point is for
+ * callers that cannot allocate device memory at the point where they decode,
+ * e.g. a serving engine that reserved (nearly) all device memory for its KV
+ * block pool before the first step, a plugin that has no access to its host
+ * framework's allocator, or a latency-critical decode loop where cudaMalloc /
+ * cudaFree would synchronise the device and stall every other stream.
+ *
+ * Same arguments, semantics and results as pkv_paged_attention_decode; the
+ * split-merge scratch is one file-scope device array of
+ * PKV_STATIC_WORKSPACE_BYTES (8 MiB) that every GPU loading this library holds
+ * until the process exits.  The call allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library routine).
+ *   - Limit: if pkv_paged_attention_workspace_bytes(num_seqs, num_heads,
+ *     num_kv_heads, head_dim, num_ctas) exceeds PKV_STATIC_WORKSPACE_BYTES the
+ *     call returns PKV_EINVAL and launches nothing.
+ *   - Set-up: the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress with that device current); make that first call
+ *     before any stream capture.
+ *   - Sharing: every call on a device uses the same array, which keeps the
+ *     last call's contents.  Nothing in it has to start at zero (every value
+ *     read is written earlier by the same call), but calls that overlap on the
+ *     GPU (different streams, or threads that do not order their calls) race
+ *     on it and give wrong results: order them.
+ */
+pkv_status pkv_paged_attention_decode_noalloc(void* out, const void* query, pkv_dtype q_dtype,
+                                              const void* key_cache, const void* value_cache,
+                                              pkv_dtype cache_dtype, const int32_t* block_tables,
+                                              int max_blocks_per_seq, const int32_t* seq_lens,
+                                              int num_seqs, int num_heads, int num_kv_heads,
+                                              int head_dim, int block_size, int64_t num_blocks,
+                                              float scale, const float* k_scale,
+                                              const float* v_scale, int num_ctas,
+                                              pkv_stream_t stream);
+
 /*
  * pkv_decode_step_host -- one whole decode step driven from host buffers:
  * copies the step's inputs host -> device, runs copy_blocks (if

@@ -7,6 +7,7 @@ are not on a CUDA device, the call raises.
 
 Names follow the C entry points without their ``pkv_`` prefix:
   reshape_and_cache, copy_blocks, paged_attention_decode,
+  paged_attention_decode_noalloc,
   paged_attention_workspace_bytes, default_num_ctas, decode_step_host,
   get_device_error, status_string
 """
@@ -29,7 +30,8 @@ _DTYPES = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_B
            torch.uint8: PKV_FP8_E4M3, torch.float8_e4m3fn: PKV_FP8_E4M3}
 
 EXPORTED = ("pkv_reshape_and_cache", "pkv_copy_blocks", "pkv_paged_attention_workspace_bytes",
-            "pkv_default_num_ctas", "pkv_paged_attention_decode", "pkv_decode_step_host",
+            "pkv_default_num_ctas", "pkv_paged_attention_decode",
+            "pkv_paged_attention_decode_noalloc", "pkv_decode_step_host",
             "pkv_get_device_error", "pkv_status_string", "pkv_last_error_message")
 
 
@@ -88,6 +90,10 @@ def lib() -> ctypes.CDLL:
     L.pkv_paged_attention_decode.argtypes = [vp, vp, c_int, vp, vp, c_int, vp, c_int, vp, c_int,
                                              c_int, c_int, c_int, c_int, i64, ctypes.c_float, vp,
                                              vp, vp, ctypes.c_size_t, c_int, vp]
+    L.pkv_paged_attention_decode_noalloc.restype = c_int
+    L.pkv_paged_attention_decode_noalloc.argtypes = [vp, vp, c_int, vp, vp, c_int, vp, c_int, vp,
+                                                     c_int, c_int, c_int, c_int, c_int, i64,
+                                                     ctypes.c_float, vp, vp, c_int, vp]
     L.pkv_decode_step_host.restype = c_int
     L.pkv_decode_step_host.argtypes = [ctypes.POINTER(DecodeStepArgs), vp]
     L.pkv_get_device_error.restype = c_int
@@ -185,6 +191,23 @@ def paged_attention_decode(out, query, key_cache, value_cache, block_tables, seq
         dtype_code(key_cache), _dev(block_tables), block_tables.shape[1], _dev(seq_lens), S, Hq,
         Hkv, D, bs, NB, float(scale), _dev(k_scale), _dev(v_scale), _dev(workspace),
         workspace.numel() * workspace.element_size(), int(num_ctas), _stream(stream)))
+    return out
+
+
+STATIC_WORKSPACE_BYTES = 8 * 1024 * 1024   # PKV_STATIC_WORKSPACE_BYTES
+
+
+def paged_attention_decode_noalloc(out, query, key_cache, value_cache, block_tables, seq_lens,
+                                   scale, k_scale=None, v_scale=None, num_ctas: int = 0,
+                                   stream=None) -> torch.Tensor:
+    """Like paged_attention_decode, with the library's static scratch instead of
+    a workspace (see pkv_paged_attention_decode_noalloc)."""
+    S, Hq, D = query.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    _check(lib().pkv_paged_attention_decode_noalloc(
+        _dev(out), _dev(query), dtype_code(query), _dev(key_cache), _dev(value_cache),
+        dtype_code(key_cache), _dev(block_tables), block_tables.shape[1], _dev(seq_lens), S, Hq,
+        Hkv, D, bs, NB, float(scale), _dev(k_scale), _dev(v_scale), int(num_ctas), _stream(stream)))
     return out
 
 
