@@ -60,10 +60,15 @@ def barrier(world: int):
 
 
 # ---------------------------------------------------------------- workload
-def make_workload(name: str, rank: int):
+def make_workload(name: str, rank: int, num_seqs: int = 0):
     from paged_kv_cache_373_b200 import workloads as W
     cfg = WORKLOADS[name]
-    wl = W.make_config(cfg)
+    kw = {}
+    if num_seqs and cfg in (2, 3, 4):
+        kw["num_seqs"] = num_seqs
+    elif num_seqs and cfg == 5:
+        kw["num_prompts"] = max(1, num_seqs // 8)
+    wl = W.make_config(cfg, **kw)
     if rank:
         # a different, equally shaped batch per rank
         import math
@@ -196,7 +201,7 @@ def run_reference(args):
     rank, world, local = dist_env()
     if rank != 0:
         return 0
-    wl = make_workload(args.workload, 0)
+    wl = make_workload(args.workload, 0, args.num_seqs)
     # each step is a bounded sample so the whole run stays within a few minutes
     smp = OracleSample(wl, budget_s=max(0.5, min(args.ref_budget, 120.0 / max(1, args.steps))))
     rates = [smp.rate() for _ in range(args.steps)]
@@ -232,7 +237,7 @@ def run_ours(args):
     else:
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
-    wl = make_workload(args.workload, rank)
+    wl = make_workload(args.workload, rank, args.num_seqs)
 
     # ---- resident device state
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -409,6 +414,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="cfg2", choices=sorted(WORKLOADS))
     ap.add_argument("--num-ctas", type=int, default=0)
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="override the workload's batch (profiling a smaller case)")
     ap.add_argument("--spinup-ms", type=float, default=400.0,
                     help="minimum untimed warm-up time (clock ramp-up)")
     ap.add_argument("--ref-budget", type=float, default=15.0)

@@ -73,7 +73,7 @@ typedef enum {
 #define PKV_DEVERR_SLOT     0x2   /* slot_mapping entry >= num_blocks * block_size */
 #define PKV_DEVERR_SEQ_LEN  0x4   /* seq_len < 0 or > max_blocks_per_seq * block_size */
 #define PKV_DEVERR_COPY_ID  0x8   /* copy_blocks src/dst outside [0, num_blocks) */
-#define PKV_DEVERR_TIMEOUT  0x10  /* a pipeline wait gave up (about 2 s); results invalid */
+#define PKV_DEVERR_TIMEOUT  0x10  /* reserved: no kernel of this version waits on another */
 
 /*
  * pkv_reshape_and_cache -- store the K/V of new tokens in their cache slots.
