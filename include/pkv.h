@@ -123,7 +123,7 @@ pkv_status pkv_copy_blocks(void* const* key_caches, void* const* value_caches, i
 
 /*
  * Workspace for pkv_paged_attention_decode: fp32 partial results of the
- * split units, (8 * num_ctas + units) x heads_per_unit x (head_dim + 2)
+ * split units, (12 * num_ctas + units) x heads_per_unit x (head_dim + 2)
  * floats, where units = num_seqs * num_kv_heads * ceil(g / 8),
  * g = num_heads / num_kv_heads and heads_per_unit = min(g, 8).  num_ctas = 0 means the default grid of the
  * current device (pkv_default_num_ctas).  Returns 0 for invalid shapes.
@@ -177,7 +177,7 @@ pkv_status pkv_paged_attention_decode(void* out, const void* query, pkv_dtype q_
                                       pkv_stream_t stream);
 
 /* Size of the static scratch used by pkv_paged_attention_decode_noalloc. */
-#define PKV_STATIC_WORKSPACE_BYTES (8u * 1024u * 1024u)
+#define PKV_STATIC_WORKSPACE_BYTES (16u * 1024u * 1024u)
 
 /*
  * pkv_paged_attention_decode_noalloc -- pkv_paged_attention_decode with no
@@ -190,7 +190,7 @@ pkv_status pkv_paged_attention_decode(void* out, const void* query, pkv_dtype q_
  *
  * Same arguments, semantics and results as pkv_paged_attention_decode; the
  * split-merge scratch is one file-scope device array of
- * PKV_STATIC_WORKSPACE_BYTES (8 MiB) that every GPU loading this library holds
+ * PKV_STATIC_WORKSPACE_BYTES (16 MiB) that every GPU loading this library holds
  * until the process exits.  The call allocates nothing (no cudaMalloc,
  * cudaFree or allocating library routine).
  *   - Limit: if pkv_paged_attention_workspace_bytes(num_seqs, num_heads,

@@ -194,7 +194,7 @@ def paged_attention_decode(out, query, key_cache, value_cache, block_tables, seq
     return out
 
 
-STATIC_WORKSPACE_BYTES = 8 * 1024 * 1024   # PKV_STATIC_WORKSPACE_BYTES
+STATIC_WORKSPACE_BYTES = 16 * 1024 * 1024   # PKV_STATIC_WORKSPACE_BYTES
 
 
 def paged_attention_decode_noalloc(out, query, key_cache, value_cache, block_tables, seq_lens,

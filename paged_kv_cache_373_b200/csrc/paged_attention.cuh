@@ -40,7 +40,7 @@ namespace pkv {
 
 constexpr int kTileTokens = 16;    // tokens per pipeline tile
 constexpr int kHeadsPerUnit = 8;   // q heads served by one KV read (one mma N tile)
-constexpr int kMaxWarpsPerCta = 8; // workspace is sized for this many workers per CTA
+constexpr int kMaxWarpsPerCta = 12; // workspace is sized for this many workers per CTA
 constexpr int kSubBytes = kTileTokens * 128;  // one 128-byte-wide column of a tile
 
 struct DecodeParams {

@@ -43,15 +43,15 @@ def test_status_strings(L):
 
 
 def test_workspace_size_formula(L):
-    # (8 workers per CTA x G + S*Hkv*ceil(g/8)) segments x min(g,8) heads
+    # (12 workers per CTA x G + S*Hkv*ceil(g/8)) segments x min(g,8) heads
     # x (D floats + one float2), 256-aligned split
     G, S, Hq, Hkv, D = 148, 64, 32, 32, 128
-    segs = 8 * G + S * Hkv * 1
+    segs = 12 * G + S * Hkv * 1
     o = segs * 1 * D * 4
     want = ((o + 255) // 256) * 256 + segs * 1 * 8
     assert pkv.paged_attention_workspace_bytes(S, Hq, Hkv, D, G) == want
     # g = 16 -> two head chunks of 8
-    segs = 8 * G + 4 * 2 * 2
+    segs = 12 * G + 4 * 2 * 2
     o = segs * 8 * 128 * 4
     assert pkv.paged_attention_workspace_bytes(4, 32, 2, 128, G) == ((o + 255) // 256) * 256 + segs * 8 * 8
     assert pkv.paged_attention_workspace_bytes(4, 30, 8, 128, G) == 0     # 30 % 8 != 0
