@@ -108,7 +108,10 @@ def recorded_traffic(workload: str):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampling of SM clocks and throttle reasons.  Started before
+    the warm-up (nvidia-smi needs a few hundred ms to start); summary() keeps
+    the samples whose timestamps fall inside the timed window."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -116,8 +119,9 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.window = None
 
-    def __enter__(self):
+    def start(self):
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -130,7 +134,7 @@ class ClockSampler:
             self.proc = None
         return self
 
-    def __exit__(self, *a):
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -142,26 +146,32 @@ class ClockSampler:
     def summary(self):
         if not self.path or not os.path.exists(self.path):
             return None
-        sm, mx, reasons = [], None, set()
+        import datetime
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
             for ln in f:
                 parts = [x.strip() for x in ln.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    mx = float(parts[2])
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(parts[2]), float(parts[3]),
+                                 {n for n, v in zip(names, parts[6:10]) if v.lower() == "active"}))
                 except ValueError:
                     continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
         os.unlink(self.path)
-        if not sm:
+        if not rows:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        t0, t1 = self.window or (rows[0][0], rows[-1][0])
+        inside = [r for r in rows if t0 - 0.02 <= r[0] <= t1 + 0.02]
+        scope = "timed region"
+        if not inside:  # region shorter than the sampling period: nearest samples
+            inside = sorted(rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))[:2]
+            scope = "nearest to the timed region"
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": inside[0][2],
+                "reasons": sorted(set().union(*[r[3] for r in inside])), "samples": len(inside),
+                "scope": scope}
 
 
 # ---------------------------------------------------------------- oracle leg
@@ -267,6 +277,7 @@ def run_ours(args):
 
     # warm-up: at least W steps and at least --spinup-ms of GPU work, so the SM
     # clock has left its idle state before the timed region
+    clk = ClockSampler(dev.index).start()
     warm = 0
     t0 = time.perf_counter()
     while warm < args.warmup or (time.perf_counter() - t0) * 1000.0 < args.spinup_ms:
@@ -284,18 +295,20 @@ def run_ours(args):
           for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clk:
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(stream)
-        for i in range(K):
-            if flush:
-                scratch.fill_(i & 0xff)     # evict the small workload from L2 (outside the step events)
-            ev[i][0].record(stream)
-            step(ev[i][1], ev[i][2])
-            ev[i][3].record(stream)
-        t_end.record(stream)
-        torch.cuda.synchronize()
+    wall0 = time.time()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(K):
+        if flush:
+            scratch.fill_(i & 0xff)     # evict the small workload from L2 (outside the step events)
+        ev[i][0].record(stream)
+        step(ev[i][1], ev[i][2])
+        ev[i][3].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk.window = (wall0, time.time())
+    clk.stop()
     barrier(world)
     step_ms = [a.elapsed_time(d) for a, _, _, d in ev]
     attn_ms = [b.elapsed_time(c) for _, b, c, _ in ev]
