@@ -25,11 +25,12 @@ pkv_status launch_decode(const DecodeLaunchArgs& a, cudaStream_t st) {
         if (e != cudaSuccess) return fail(PKV_ECUDA, "smem opt-in: %s", cudaGetErrorString(e));
         configured.fetch_or(bit);
     }
-    pkv_decode_kernel<C><<<a.grid, C::kWarps * 32, C::kSmemBytes, st>>>(*a.params);
+    const DecodeParams& p = *a.params;
+    pkv_decode_kernel<C><<<a.grid, C::kWarps * 32, C::kSmemBytes, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "decode launch: %s", cudaGetErrorString(e));
     const int64_t workers = (int64_t)a.grid * C::kWarps;
-    pkv_merge_kernel<typename C::q_t, C::D><<<(unsigned)((workers + 7) / 8), 256, 0, st>>>(*a.params, workers);
+    pkv_merge_kernel<typename C::q_t, C::D, C::kTT><<<(unsigned)((workers + 7) / 8), 256, 0, st>>>(p, workers);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "merge launch: %s", cudaGetErrorString(e));
     return PKV_OK;

@@ -38,10 +38,9 @@
 
 namespace pkv {
 
-constexpr int kTileTokens = 16;    // tokens per pipeline tile
+constexpr int kTileTokens = 16;    // tokens per pipeline tile (32 for FP8 caches with 32-token blocks)
 constexpr int kHeadsPerUnit = 8;   // q heads served by one KV read (one mma N tile)
 constexpr int kMaxWarpsPerCta = 12; // workspace is sized for this many workers per CTA
-constexpr int kSubBytes = kTileTokens * 128;  // one 128-byte-wide column of a tile
 
 struct DecodeParams {
     void* out;
@@ -64,10 +63,12 @@ struct DecodeParams {
 };
 
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
-__device__ __forceinline__ int ntiles_of(int L) { return (L + kTileTokens - 1) / kTileTokens; }
+template <int TT>
+__device__ __forceinline__ int ntiles_of(int L) { return (L + TT - 1) / TT; }
 
 // Warp-collective: total tiles W = units_per_seq * sum_s ceil(L_s / 16);
 // *bad_len is set when some length is negative or overruns its table row.
+template <int TT>
 __device__ inline int64_t total_tiles(const int32_t* seq_lens, int S, int units, int cap,
                                       bool* bad_len = nullptr) {
     const int lane = threadIdx.x & 31;
@@ -81,7 +82,7 @@ __device__ inline int64_t total_tiles(const int32_t* seq_lens, int S, int units,
             if (s < S) {
                 const int L = __ldg(seq_lens + s);
                 bad |= (L < 0 || L > cap);
-                part += ntiles_of(clamp_len(L, cap));
+                part += ntiles_of<TT>(clamp_len(L, cap));
             }
         }
 #pragma unroll
@@ -99,6 +100,7 @@ struct SeqHit {
 };
 
 // Warp-collective: the sequence whose tiles contain global tile P.
+template <int TT>
 __device__ inline SeqHit find_seq(const int32_t* seq_lens, int S, int units, int cap, int64_t P) {
     const int lane = threadIdx.x & 31;
     int64_t base = 0;
@@ -108,7 +110,7 @@ __device__ inline SeqHit find_seq(const int32_t* seq_lens, int S, int units, int
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const int s = s0 + lane * 8 + k;
-            w[k] = (s < S) ? (int64_t)ntiles_of(clamp_len(__ldg(seq_lens + s), cap)) * units : 0;
+            w[k] = (s < S) ? (int64_t)ntiles_of<TT>(clamp_len(__ldg(seq_lens + s), cap)) * units : 0;
             part += w[k];
         }
         int64_t incl = part;
@@ -139,7 +141,8 @@ __device__ inline SeqHit find_seq(const int32_t* seq_lens, int S, int units, int
     return SeqHit{S, base, 0};
 }
 
-// Walk over a worker's tiles in order: (sequence, unit j, tile i).
+// Walk over a worker's tiles (TT tokens each) in order: (sequence, unit j, tile i).
+template <int TT>
 struct Walk {
     int s, L, nt, j, i, seg_i0, ord;
     int64_t T, te;
@@ -152,10 +155,10 @@ struct Walk {
         ord = 0;
         s = 0; L = 0; nt = 1; j = 0; i = 0; seg_i0 = 0;
         if (done) return;
-        const SeqHit h = find_seq(seq_lens, S, units, cap, tb);
+        const SeqHit h = find_seq<TT>(seq_lens, S, units, cap, tb);
         s = h.s;
         L = h.L;
-        nt = ntiles_of(L);
+        nt = ntiles_of<TT>(L);
         j = (int)((tb - h.base) / nt);
         i = (int)((tb - h.base) % nt);
         seg_i0 = i;
@@ -173,8 +176,8 @@ struct Walk {
                 j = 0;
                 do {  // a later non-empty sequence exists because T < te <= W
                     ++s;
-                    L = (s < S) ? clamp_len(__ldg(seq_lens + s), cap) : kTileTokens;
-                    nt = ntiles_of(L);
+                    L = (s < S) ? clamp_len(__ldg(seq_lens + s), cap) : TT;
+                    nt = ntiles_of<TT>(L);
                 } while (nt == 0);
             }
         }
@@ -186,7 +189,7 @@ struct Walk {
 // ----------------------------------------------------------------------------
 enum class Path { kMma16, kFp8, kF32 };
 
-template <typename KvT, typename QT, int D_, Path P_, int kWarps_, int kStages_>
+template <typename KvT, typename QT, int D_, Path P_, int kWarps_, int kStages_, int kTT_ = kTileTokens>
 struct Cfg {
     using kv_t = KvT;
     using q_t = QT;
@@ -194,6 +197,8 @@ struct Cfg {
     static constexpr int D = D_;
     static constexpr int kWarps = kWarps_;
     static constexpr int kStages = kStages_;
+    static constexpr int kTT = kTT_;                    // tokens per tile
+    static constexpr int kSubBytes = kTT * 128;         // one 128-byte-wide column of a tile
     static constexpr int kKvBytes = (int)sizeof(KvT);
     static constexpr int kQBytes = (int)sizeof(QT);
     static constexpr int kRowBytes = D * kKvBytes;
@@ -205,6 +210,7 @@ struct Cfg {
     static constexpr int kSmemBytes = kWarps * kWarpBytes + 1024;  // + alignment slack
     static constexpr int kChunksPerRow = kRowBytes / 16;
     static constexpr int kRowsPerInst = 32 / kChunksPerRow;         // rows one warp-wide cp.async covers
+    static_assert(kTT == 16 || (kTT == 32 && P_ != Path::kF32), "tile sizes");
     static_assert(kRowBytes % 128 == 0, "rows must be whole 128-byte columns");
     static_assert(kStageBytes % 1024 == 0 && kQSlot % 1024 == 0, "1024-byte stage alignment");
     static_assert(kWarps <= kMaxWarpsPerCta, "workspace sizing");
@@ -221,9 +227,10 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // Zero rows [valid, 16) of a V tile (NSUB columns of 16 x 128 B).  Used on a
 // sequence's last tile so the unused slots (never written, any bits) cannot
 // reach the tensor-core P.V product.
-template <int kNSub>
+template <int kNSub, int TT>
 __device__ __forceinline__ void zero_tail_rows(uint8_t* tile, int valid, int lane) {
-    const int rows = kTileTokens - valid;
+    constexpr int kSubBytes = TT * 128;
+    const int rows = TT - valid;
     const int per_sub = rows * 8;  // 16-byte chunks
     for (int idx = lane; idx < kNSub * per_sub; idx += 32) {
         const int sub = idx / per_sub, rem = idx % per_sub;
@@ -236,8 +243,9 @@ __device__ __forceinline__ void zero_tail_rows(uint8_t* tile, int valid, int lan
 // Swizzled byte offset of 16-byte chunk `c` (of the whole row) of token row t
 // in a tile: column c/8, line t, chunk (c%8) XOR (t%8) -- conflict-free for
 // the ldmatrix / 16-byte shared loads below and for the cp.async writes.
+template <int TT = kTileTokens>
 __device__ __forceinline__ uint32_t sw_off(int t, int c) {
-    return (uint32_t)((c >> 3) * kSubBytes + t * 128 + ((((c & 7) ^ t) & 7) << 4));
+    return (uint32_t)((c >> 3) * (TT * 128) + t * 128 + ((((c & 7) ^ t) & 7) << 4));
 }
 
 // Output / workspace sink of one unit segment.
@@ -323,46 +331,59 @@ struct MmaConsumer {
         }
     }
 
+    // One tile of TT = 16 * NM tokens: S^T per 16-token m-tile, one online
+    // softmax step over the whole tile, then P.V with one k-step per m-tile.
     __device__ void tile(uint8_t* kt, uint8_t* vt, int valid) {
+        constexpr int TT = C::kTT, NM = TT / 16;
         const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
-        if (valid < kTileTokens) zero_tail_rows<C::kNSub>(vt, valid, lane);
+        if (valid < TT) zero_tail_rows<C::kNSub, TT>(vt, valid, lane);
         const uint32_t kb = smem_u32(kt), vb = smem_u32(vt);
-        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (!kFp8) {
-            const int r = lane & 7, mtx = lane >> 3;
-            const int t = r + ((mtx & 1) << 3);
+        float x[NM][4];
 #pragma unroll
-            for (int kk = 0; kk < KS; ++kk) {
-                uint32_t a[4];
-                ldsm_x4(a, kb + sw_off(t, 2 * kk + (mtx >> 1)));
-                if (kk & 1) mma16816<kOpBf16>(sb, a, qf[kk][0], qf[kk][1]);
-                else        mma16816<kOpBf16>(sa, a, qf[kk][0], qf[kk][1]);
-            }
-        } else {
-            // K rows gid and gid+8, bytes [32*tig, 32*tig+32): two chunks each.
-            const uint4 r0a = *reinterpret_cast<const uint4*>(kt + sw_off(gid, 2 * tig));
-            const uint4 r0b = *reinterpret_cast<const uint4*>(kt + sw_off(gid, 2 * tig + 1));
-            const uint4 r1a = *reinterpret_cast<const uint4*>(kt + sw_off(gid + 8, 2 * tig));
-            const uint4 r1b = *reinterpret_cast<const uint4*>(kt + sw_off(gid + 8, 2 * tig + 1));
-            const uint32_t w0[8] = {r0a.x, r0a.y, r0a.z, r0a.w, r0b.x, r0b.y, r0b.z, r0b.w};
-            const uint32_t w1[8] = {r1a.x, r1a.y, r1a.z, r1a.w, r1b.x, r1b.y, r1b.z, r1b.w};
+        for (int m = 0; m < NM; ++m) {
+            float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+            if constexpr (!kFp8) {
+                const int r = lane & 7, mtx = lane >> 3;
+                const int t = 16 * m + r + ((mtx & 1) << 3);
 #pragma unroll
-            for (int kk = 0; kk < KS; ++kk) {
-                uint32_t a[4];
-                a[0] = e4m3x2_to_f16x2((uint16_t)(w0[kk] & 0xffffu));
-                a[1] = e4m3x2_to_f16x2((uint16_t)(w1[kk] & 0xffffu));
-                a[2] = e4m3x2_to_f16x2((uint16_t)(w0[kk] >> 16));
-                a[3] = e4m3x2_to_f16x2((uint16_t)(w1[kk] >> 16));
-                if (kk & 1) mma16816<false>(sb, a, qf[kk][0], qf[kk][1]);
-                else        mma16816<false>(sa, a, qf[kk][0], qf[kk][1]);
+                for (int kk = 0; kk < KS; ++kk) {
+                    uint32_t a[4];
+                    ldsm_x4(a, kb + sw_off<TT>(t, 2 * kk + (mtx >> 1)));
+                    if (kk & 1) mma16816<kOpBf16>(sb, a, qf[kk][0], qf[kk][1]);
+                    else        mma16816<kOpBf16>(sa, a, qf[kk][0], qf[kk][1]);
+                }
+            } else {
+                // K rows gid and gid+8 of the m-tile, bytes [32*tig, 32*tig+32).
+                const int t0 = 16 * m + gid, t1 = t0 + 8;
+                const uint4 r0a = *reinterpret_cast<const uint4*>(kt + sw_off<TT>(t0, 2 * tig));
+                const uint4 r0b = *reinterpret_cast<const uint4*>(kt + sw_off<TT>(t0, 2 * tig + 1));
+                const uint4 r1a = *reinterpret_cast<const uint4*>(kt + sw_off<TT>(t1, 2 * tig));
+                const uint4 r1b = *reinterpret_cast<const uint4*>(kt + sw_off<TT>(t1, 2 * tig + 1));
+                const uint32_t w0[8] = {r0a.x, r0a.y, r0a.z, r0a.w, r0b.x, r0b.y, r0b.z, r0b.w};
+                const uint32_t w1[8] = {r1a.x, r1a.y, r1a.z, r1a.w, r1b.x, r1b.y, r1b.z, r1b.w};
+#pragma unroll
+                for (int kk = 0; kk < KS; ++kk) {
+                    uint32_t a[4];
+                    a[0] = e4m3x2_to_f16x2((uint16_t)(w0[kk] & 0xffffu));
+                    a[1] = e4m3x2_to_f16x2((uint16_t)(w1[kk] & 0xffffu));
+                    a[2] = e4m3x2_to_f16x2((uint16_t)(w0[kk] >> 16));
+                    a[3] = e4m3x2_to_f16x2((uint16_t)(w1[kk] >> 16));
+                    if (kk & 1) mma16816<false>(sb, a, qf[kk][0], qf[kk][1]);
+                    else        mma16816<false>(sa, a, qf[kk][0], qf[kk][1]);
+                }
             }
+            // scores S^T[token][head]: (gid, 2tig), (gid, 2tig+1), (gid+8, 2tig), (gid+8, 2tig+1)
+            x[m][0] = (sa[0] + sb[0]) * sl0; x[m][1] = (sa[1] + sb[1]) * sl1;
+            x[m][2] = (sa[2] + sb[2]) * sl0; x[m][3] = (sa[3] + sb[3]) * sl1;
+            if (16 * m + gid >= valid) x[m][0] = x[m][1] = -INFINITY;
+            if (16 * m + gid + 8 >= valid) x[m][2] = x[m][3] = -INFINITY;
         }
-        // scores S^T[token][head]: (gid, 2tig), (gid, 2tig+1), (gid+8, 2tig), (gid+8, 2tig+1)
-        float x0 = (sa[0] + sb[0]) * sl0, x1 = (sa[1] + sb[1]) * sl1;
-        float x2 = (sa[2] + sb[2]) * sl0, x3 = (sa[3] + sb[3]) * sl1;
-        if (gid >= valid) x0 = x1 = -INFINITY;
-        if (gid + 8 >= valid) x2 = x3 = -INFINITY;
-        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+        float mx0 = fmaxf(x[0][0], x[0][2]), mx1 = fmaxf(x[0][1], x[0][3]);
+#pragma unroll
+        for (int m = 1; m < NM; ++m) {
+            mx0 = fmaxf(mx0, fmaxf(x[m][0], x[m][2]));
+            mx1 = fmaxf(mx1, fmaxf(x[m][1], x[m][3]));
+        }
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
             mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o));
@@ -377,63 +398,74 @@ struct MmaConsumer {
         // hi + lo bf16 parts (two products, ~16 significant bits): the P.V sum
         // then matches fp32 P to well inside the tolerance.  f16 (11 bits) and
         // the FP8 path (f16) use one part.
-        const float e0 = ex2(x0 - mn0), e1 = ex2(x1 - mn1), e2 = ex2(x2 - mn0), e3 = ex2(x3 - mn1);
-        const uint32_t X0 = pack2<kOpBf16>(e0, e1);
-        const uint32_t X1 = pack2<kOpBf16>(e2, e3);
-        uint32_t c0 = 0, c1 = 0;
-        if constexpr (kOpBf16) {
-            const float2 h0 = unpack2<true>(X0), h1 = unpack2<true>(X1);
-            const uint32_t Y0 = pack2<true>(e0 - h0.x, e1 - h0.y);
-            const uint32_t Y1 = pack2<true>(e2 - h1.x, e3 - h1.y);
-            c0 = movm_trans(Y0);
-            c1 = movm_trans(Y1);
-            l0 = l0 * al0 + (e0 + e2);
-            l1 = l1 * al1 + (e1 + e3);
-        } else {
-            const float2 p0 = unpack2<false>(X0), p1 = unpack2<false>(X1);
-            l0 = l0 * al0 + p0.x + p1.x;  // normaliser from the rounded P actually used
-            l1 = l1 * al1 + p0.y + p1.y;
+        uint32_t b0[NM], b1[NM], c0[NM], c1[NM];
+        float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+        for (int m = 0; m < NM; ++m) {
+            const float e0 = ex2(x[m][0] - mn0), e1 = ex2(x[m][1] - mn1);
+            const float e2 = ex2(x[m][2] - mn0), e3 = ex2(x[m][3] - mn1);
+            const uint32_t X0 = pack2<kOpBf16>(e0, e1);
+            const uint32_t X1 = pack2<kOpBf16>(e2, e3);
+            if constexpr (kOpBf16) {
+                const float2 h0 = unpack2<true>(X0), h1 = unpack2<true>(X1);
+                c0[m] = movm_trans(pack2<true>(e0 - h0.x, e1 - h0.y));
+                c1[m] = movm_trans(pack2<true>(e2 - h1.x, e3 - h1.y));
+                ls0 += e0 + e2;
+                ls1 += e1 + e3;
+            } else {
+                const float2 p0 = unpack2<false>(X0), p1 = unpack2<false>(X1);
+                ls0 += p0.x + p1.x;  // normaliser from the rounded P actually used
+                ls1 += p0.y + p1.y;
+                c0[m] = c1[m] = 0u;
+            }
+            b0[m] = movm_trans(X0);  // P^T as mma B
+            b1[m] = movm_trans(X1);
         }
-        const uint32_t b0 = movm_trans(X0), b1 = movm_trans(X1);  // P^T as mma B
+        l0 = l0 * al0 + ls0;
+        l1 = l1 * al1 + ls1;
 #pragma unroll
         for (int mi = 0; mi < MT; ++mi) {
             acc[mi][0] *= al0; acc[mi][1] *= al1; acc[mi][2] *= al0; acc[mi][3] *= al1;
         }
-        if constexpr (!kFp8) {
-            const int r = lane & 7, mtx = lane >> 3;
-            const int t = r + ((mtx >> 1) << 3);
 #pragma unroll
-            for (int mi = 0; mi < MT; ++mi) {
-                uint32_t a[4];
-                ldsm_x4_trans(a, vb + sw_off(t, 2 * mi + (mtx & 1)));
-                mma16816<kOpBf16>(acc[mi], a, b0, b1);
-                if constexpr (kOpBf16) mma16816<true>(acc[mi], a, c0, c1);
-            }
-        } else {
-            // V^T fragments: thread gid owns d in [16*gid, 16*gid+16) (one chunk),
-            // rows t = 2tig, 2tig+1, 2tig+8, 2tig+9; m-tile mi covers
-            // d = 16*gid + 2*mi (row gid) and 16*gid + 2*mi + 1 (row gid+8).
-            const uint4 R0 = *reinterpret_cast<const uint4*>(vt + sw_off(2 * tig, gid));
-            const uint4 R1 = *reinterpret_cast<const uint4*>(vt + sw_off(2 * tig + 1, gid));
-            const uint4 R8 = *reinterpret_cast<const uint4*>(vt + sw_off(2 * tig + 8, gid));
-            const uint4 R9 = *reinterpret_cast<const uint4*>(vt + sw_off(2 * tig + 9, gid));
-            const uint32_t q0[4] = {R0.x, R0.y, R0.z, R0.w}, q1[4] = {R1.x, R1.y, R1.z, R1.w};
-            const uint32_t q8[4] = {R8.x, R8.y, R8.z, R8.w}, q9[4] = {R9.x, R9.y, R9.z, R9.w};
+        for (int m = 0; m < NM; ++m) {
+            if constexpr (!kFp8) {
+                const int r = lane & 7, mtx = lane >> 3;
+                const int t = 16 * m + r + ((mtx >> 1) << 3);
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const uint32_t X = prmt(q0[w], q1[w], 0x5140), Y = prmt(q0[w], q1[w], 0x7362);
-                const uint32_t X8 = prmt(q8[w], q9[w], 0x5140), Y8 = prmt(q8[w], q9[w], 0x7362);
-                uint32_t a[4];
-                a[0] = e4m3x2_to_f16x2((uint16_t)(X & 0xffffu));
-                a[1] = e4m3x2_to_f16x2((uint16_t)(X >> 16));
-                a[2] = e4m3x2_to_f16x2((uint16_t)(X8 & 0xffffu));
-                a[3] = e4m3x2_to_f16x2((uint16_t)(X8 >> 16));
-                mma16816<false>(acc[2 * w], a, b0, b1);
-                a[0] = e4m3x2_to_f16x2((uint16_t)(Y & 0xffffu));
-                a[1] = e4m3x2_to_f16x2((uint16_t)(Y >> 16));
-                a[2] = e4m3x2_to_f16x2((uint16_t)(Y8 & 0xffffu));
-                a[3] = e4m3x2_to_f16x2((uint16_t)(Y8 >> 16));
-                mma16816<false>(acc[2 * w + 1], a, b0, b1);
+                for (int mi = 0; mi < MT; ++mi) {
+                    uint32_t a[4];
+                    ldsm_x4_trans(a, vb + sw_off<TT>(t, 2 * mi + (mtx & 1)));
+                    mma16816<kOpBf16>(acc[mi], a, b0[m], b1[m]);
+                    if constexpr (kOpBf16) mma16816<true>(acc[mi], a, c0[m], c1[m]);
+                }
+            } else {
+                // V^T fragments: thread gid owns d in [16*gid, 16*gid+16) (one chunk),
+                // rows 2tig, 2tig+1, 2tig+8, 2tig+9 of the m-tile; m-tile mi covers
+                // d = 16*gid + 2*mi (row gid) and 16*gid + 2*mi + 1 (row gid+8).
+                const int tb = 16 * m + 2 * tig;
+                const uint4 R0 = *reinterpret_cast<const uint4*>(vt + sw_off<TT>(tb, gid));
+                const uint4 R1 = *reinterpret_cast<const uint4*>(vt + sw_off<TT>(tb + 1, gid));
+                const uint4 R8 = *reinterpret_cast<const uint4*>(vt + sw_off<TT>(tb + 8, gid));
+                const uint4 R9 = *reinterpret_cast<const uint4*>(vt + sw_off<TT>(tb + 9, gid));
+                const uint32_t q0[4] = {R0.x, R0.y, R0.z, R0.w}, q1[4] = {R1.x, R1.y, R1.z, R1.w};
+                const uint32_t q8[4] = {R8.x, R8.y, R8.z, R8.w}, q9[4] = {R9.x, R9.y, R9.z, R9.w};
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const uint32_t X = prmt(q0[w], q1[w], 0x5140), Y = prmt(q0[w], q1[w], 0x7362);
+                    const uint32_t X8 = prmt(q8[w], q9[w], 0x5140), Y8 = prmt(q8[w], q9[w], 0x7362);
+                    uint32_t a[4];
+                    a[0] = e4m3x2_to_f16x2((uint16_t)(X & 0xffffu));
+                    a[1] = e4m3x2_to_f16x2((uint16_t)(X >> 16));
+                    a[2] = e4m3x2_to_f16x2((uint16_t)(X8 & 0xffffu));
+                    a[3] = e4m3x2_to_f16x2((uint16_t)(X8 >> 16));
+                    mma16816<false>(acc[2 * w], a, b0[m], b1[m]);
+                    a[0] = e4m3x2_to_f16x2((uint16_t)(Y & 0xffffu));
+                    a[1] = e4m3x2_to_f16x2((uint16_t)(Y >> 16));
+                    a[2] = e4m3x2_to_f16x2((uint16_t)(Y8 & 0xffffu));
+                    a[3] = e4m3x2_to_f16x2((uint16_t)(Y8 >> 16));
+                    mma16816<false>(acc[2 * w + 1], a, b0[m], b1[m]);
+                }
             }
         }
     }
@@ -617,11 +649,11 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // Issue the async loads of the walk's current tile (and, on a unit's first
 // tile, of its q rows) into stage `stg` / q slot `qslot`.
 template <class C>
-__device__ __forceinline__ void issue_tile(const DecodeParams& p, const Walk& w, TablePrefetch& tp,
+__device__ __forceinline__ void issue_tile(const DecodeParams& p, const Walk<C::kTT>& w, TablePrefetch& tp,
                                            uint8_t* stg, uint8_t* qslot) {
     const int lane = threadIdx.x & 31;
     const int kh = w.j / p.nch, c = w.j % p.nch;
-    const int tok = w.i * kTileTokens;
+    const int tok = w.i * C::kTT;
     const int nblk = (w.L + p.block_size - 1) / p.block_size;
     int phys = tp.get(p, w.s, tok / p.block_size, nblk, lane);
     if (phys < 0 || phys >= p.num_blocks) {
@@ -636,10 +668,10 @@ __device__ __forceinline__ void issue_tile(const DecodeParams& p, const Walk& w,
     const uint32_t kdst = smem_u32(stg), vdst = smem_u32(stg + C::kTensorTile);
     const int cr = lane % C::kChunksPerRow, r0 = lane / C::kChunksPerRow;
 #pragma unroll
-    for (int it = 0; it < kTileTokens / C::kRowsPerInst; ++it) {
+    for (int it = 0; it < C::kTT / C::kRowsPerInst; ++it) {
         const int t = it * C::kRowsPerInst + r0;
         const int64_t off = t * row_stride + cr * 16;
-        const uint32_t so = sw_off(t, cr);
+        const uint32_t so = sw_off<C::kTT>(t, cr);
         cp_async16(kdst + so, ksrc + off);
         cp_async16(vdst + so, vsrc + off);
     }
@@ -670,13 +702,13 @@ pkv_decode_kernel(const DecodeParams p) {
     const int64_t workers = (int64_t)gridDim.x * C::kWarps;
     const int64_t wid = (int64_t)blockIdx.x * C::kWarps + warp;
     bool bad_len = false;
-    const int64_t W = total_tiles(p.seq_lens, p.num_seqs, units, cap, &bad_len);
+    const int64_t W = total_tiles<C::kTT>(p.seq_lens, p.num_seqs, units, cap, &bad_len);
     if (bad_len && wid == 0 && lane == 0) raise_error(p.err, PKV_DEVERR_SEQ_LEN);
     const int64_t chunk = (W + workers - 1) / workers;
     const int64_t tb = min(W, wid * chunk), te = min(W, tb + chunk);
     if (tb >= te) return;
 
-    Walk iw, cw;  // issue walk (runs kStages-1 tiles ahead) and compute walk
+    Walk<C::kTT> iw, cw;  // issue walk (runs kStages-1 tiles ahead) and compute walk
     iw.init(p.seq_lens, p.num_seqs, units, cap, tb, te);
     cw = iw;
     TablePrefetch tp;
@@ -706,7 +738,7 @@ pkv_decode_kernel(const DecodeParams p) {
             cs.reset();
         }
         uint8_t* kt = stages + (n % C::kStages) * C::kStageBytes;
-        cs.tile(kt, kt + C::kTensorTile, min(kTileTokens, cw.L - cw.i * kTileTokens));
+        cs.tile(kt, kt + C::kTensorTile, min(C::kTT, cw.L - cw.i * C::kTT));
         if (cw.last()) {
             Sink k;
             k.split = (cw.seg_i0 != 0) || (cw.i != cw.nt - 1);
@@ -728,7 +760,7 @@ pkv_decode_kernel(const DecodeParams p) {
 // boundary b if that is the unit's first interior boundary; warp 0 zeroes the
 // empty sequences.  Partials are combined in worker order.
 // ----------------------------------------------------------------------------
-template <typename QT, int D>
+template <typename QT, int D, int TT>
 __global__ void __launch_bounds__(256)
 pkv_merge_kernel(const DecodeParams p, int64_t workers) {
     const int lane = threadIdx.x & 31;
@@ -744,12 +776,12 @@ pkv_merge_kernel(const DecodeParams p, int64_t workers) {
         return;
     }
     if (b >= workers) return;
-    const int64_t W = total_tiles(p.seq_lens, p.num_seqs, units, cap);
+    const int64_t W = total_tiles<TT>(p.seq_lens, p.num_seqs, units, cap);
     const int64_t chunk = (W + workers - 1) / workers;
     const int64_t P = b * chunk;
     if (P >= W) return;
-    const SeqHit hit = find_seq(p.seq_lens, p.num_seqs, units, cap, P);
-    const int nt = ntiles_of(hit.L);
+    const SeqHit hit = find_seq<TT>(p.seq_lens, p.num_seqs, units, cap, P);
+    const int nt = ntiles_of<TT>(hit.L);
     const int j = (int)((P - hit.base) / nt);
     const int off = (int)((P - hit.base) % nt);
     const int64_t T0 = hit.base + (int64_t)j * nt;
