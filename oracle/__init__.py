@@ -50,6 +50,9 @@ def lib():
                                                ctypes.c_float, ctypes.c_float]
         L.oracle_copy_blocks.restype = c_int
         L.oracle_copy_blocks.argtypes = [c_void, c_void, c_int, c_void, c_i64, c_i64, c_i64]
+        L.oracle_swap_blocks.restype = c_int
+        L.oracle_swap_blocks.argtypes = [c_void, c_void, c_i64, c_void, c_void, c_i64, c_int, c_void,
+                                         c_i64, c_i64]
         L.oracle_paged_attention_decode.restype = c_int
         L.oracle_paged_attention_decode.argtypes = [
             c_void, c_void, c_int, c_void, c_void, c_int, c_void, c_int, c_void, c_int, c_int,
@@ -137,6 +140,21 @@ def copy_blocks(key_caches, value_caches, block_mapping) -> None:
                                   bm.shape[0], block_bytes, NB)
     if rc != 0:
         raise ValueError(f"oracle_copy_blocks failed: {rc}")
+
+
+def swap_blocks(dst_key_caches, dst_value_caches, src_key_caches, src_value_caches,
+                block_mapping) -> None:
+    """dst pools modified in place; every pool a list (per layer) of CPU tensors [NB, ...]."""
+    n = len(dst_key_caches)
+    arr = lambda ts: (ctypes.c_void_p * n)(*[_ptr(t) for t in ts])
+    dk, dv, sk, sv = arr(dst_key_caches), arr(dst_value_caches), arr(src_key_caches), arr(src_value_caches)
+    bm = block_mapping.to(torch.int64).contiguous()
+    block_bytes = src_key_caches[0][0].numel() * src_key_caches[0].element_size()
+    rc = lib().oracle_swap_blocks(ctypes.addressof(dk), ctypes.addressof(dv), dst_key_caches[0].shape[0],
+                                  ctypes.addressof(sk), ctypes.addressof(sv), src_key_caches[0].shape[0],
+                                  n, _ptr(bm), bm.shape[0], block_bytes)
+    if rc != 0:
+        raise ValueError(f"oracle_swap_blocks failed: {rc}")
 
 
 def paged_attention_decode(query, key_cache, value_cache, block_tables, seq_lens, scale,

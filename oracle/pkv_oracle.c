@@ -249,6 +249,28 @@ int oracle_copy_blocks(void* const* key_caches, void* const* value_caches, int n
 }
 
 /* ------------------------------------------------------------------------- */
+/* swap_blocks: whole blocks from one pool to another (zwxr.cn 4.3, swapping   */
+/* a preempted sequence's KV blocks out to host memory and back in)           */
+/* ------------------------------------------------------------------------- */
+int oracle_swap_blocks(void* const* dst_key_caches, void* const* dst_value_caches,
+                       int64_t dst_num_blocks, void* const* src_key_caches,
+                       void* const* src_value_caches, int64_t src_num_blocks, int num_layers,
+                       const int64_t* block_mapping, int64_t num_pairs, int64_t block_bytes)
+{
+    for (int64_t p = 0; p < num_pairs; ++p) {
+        int64_t src = block_mapping[2 * p], dst = block_mapping[2 * p + 1];
+        if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) return OR_ERANGE;
+        for (int l = 0; l < num_layers; ++l) {
+            memcpy((char*)dst_key_caches[l] + dst * block_bytes,
+                   (const char*)src_key_caches[l] + src * block_bytes, (size_t)block_bytes);
+            memcpy((char*)dst_value_caches[l] + dst * block_bytes,
+                   (const char*)src_value_caches[l] + src * block_bytes, (size_t)block_bytes);
+        }
+    }
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------------------- */
 /* decode attention (thinkmoon.cn pseudocode, masked to the logical length)   */
 /* ------------------------------------------------------------------------- */
 
