@@ -264,14 +264,29 @@ def run_ours(args):
     flush = kv_bytes < 2 * L2_BYTES
     scratch = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if flush else None
 
+    if args.cascade:
+        from paged_kv_cache_373_b200 import workloads as W
+        goff, gmem, gpre, gmax = (t.to(dev) if torch.is_tensor(t) else t for t in W.cascade_groups(wl))
+        cws = torch.empty(pkv.paged_attention_cascade_workspace_bytes(
+            wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, gpre.shape[0], gmax,
+            args.num_ctas), dtype=torch.uint8, device=dev)
+
+    def attend():
+        if args.cascade:
+            pkv.paged_attention_decode_cascade(out, g["q"], g["kc"], g["vc"], g["tables"], g["lens"],
+                                               goff, gmem, gpre, gmax, wl.scale, g["ks"], g["vs"],
+                                               workspace=cws, num_ctas=args.num_ctas)
+        else:
+            pkv.paged_attention_decode(out, g["q"], g["kc"], g["vc"], g["tables"], g["lens"], wl.scale,
+                                       g["ks"], g["vs"], workspace=ws, num_ctas=args.num_ctas)
+
     def step(ev_a0=None, ev_a1=None):
         if has_pairs:
             pkv.copy_blocks([g["kc"]], [g["vc"]], g["pairs"])
         pkv.reshape_and_cache(g["nk"], g["nv"], g["kc"], g["vc"], g["slots"], g["ks"], g["vs"])
         if ev_a0 is not None:
             ev_a0.record(stream)
-        pkv.paged_attention_decode(out, g["q"], g["kc"], g["vc"], g["tables"], g["lens"], wl.scale,
-                                   g["ks"], g["vs"], workspace=ws, num_ctas=args.num_ctas)
+        attend()
         if ev_a1 is not None:
             ev_a1.record(stream)
 
@@ -336,7 +351,7 @@ def run_ours(args):
                "sample": f"first {smp.k} of {wl.num_seqs} sequences of the same workload, "
                          f"fp64 C oracle, {smp.cores} OpenMP threads"}
 
-    launches_per_step = (1 if has_pairs else 0) + 1 + 2
+    launches_per_step = (1 if has_pairs else 0) + 1 + (6 if args.cascade else 2)
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "seq-steps/s", "n_gpus": world,
@@ -346,7 +361,8 @@ def run_ours(args):
             "dtype": {True: "fp8_e4m3 kv / fp32 accum", False: str(wl.kv_dtype).replace("torch.", "")
                       + " kv / fp32 accum"}[wl.is_fp8],
             "data": "synthetic",
-            "config": {"workload": wl.name, "num_seqs": wl.num_seqs, "num_heads": wl.num_heads,
+            "config": {"workload": wl.name + ("_cascade" if args.cascade else ""),
+                       "num_seqs": wl.num_seqs, "num_heads": wl.num_heads,
                        "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                        "block_size": wl.block_size, "num_blocks": wl.num_blocks,
                        "max_seq_len": wl.max_seq_len, "cow_pairs": int(wl.cow_pairs.shape[0]),
@@ -433,6 +449,8 @@ def main():
                     help="minimum untimed warm-up time (clock ramp-up)")
     ap.add_argument("--ref-budget", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cascade", action="store_true",
+                    help="prefix-sharing workloads: read each shared prefix once per group")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps

@@ -7,6 +7,8 @@
  * and 3.2).  This library implements the device side of one decode step:
  *
  *   pkv_copy_blocks            copy-on-write copies of shared blocks (3.4)
+ *   pkv_swap_blocks            block moves between device and page-locked host
+ *                              pools (preemption by swapping, 4.3)
  *   pkv_reshape_and_cache      write each new token's K/V into its slot (3.1)
  *   pkv_paged_attention_decode single-token attention through the block
  *                              table with the block-wise softmax merge (3.3)
@@ -65,7 +67,8 @@ typedef enum {
     PKV_EINVAL = 1,       /* bad argument (null pointer, bad shape, bad alignment) */
     PKV_EUNSUPPORTED = 2, /* valid but not implemented (e.g. head_dim 96) */
     PKV_ECUDA = 3,        /* a CUDA runtime call failed */
-    PKV_EDEVICE = 4       /* the device error word is non-zero */
+    PKV_EDEVICE = 4,      /* the device error word is non-zero */
+    PKV_ENOBLOCKS = 5     /* host block manager: the pool cannot supply the blocks */
 } pkv_status;
 
 /* Bits of the device error word. */
@@ -122,6 +125,34 @@ pkv_status pkv_copy_blocks(void* const* key_caches, void* const* value_caches, i
                            size_t block_bytes, pkv_stream_t stream);
 
 /*
+ * pkv_swap_blocks -- whole-block copies from one block pool to another, where
+ * each pool lives in device memory of the current device or in page-locked
+ * host memory (cudaHostAlloc / cudaHostRegister, torch pin_memory), which the
+ * kernel reads and writes directly through unified addressing.  This is the
+ * data movement of preemption by swapping (zwxr.cn section 4.3): the blocks
+ * of a preempted sequence go to host memory, and later come back to whatever
+ * device blocks are free (its block table is rewritten by the caller).
+ *
+ * For every pair p and every layer l:
+ *   dst_key_caches[l] block block_mapping[p][1] = src_key_caches[l] block block_mapping[p][0]
+ * (same for values); blocks are block_bytes contiguous bytes (a multiple of
+ * 16), pools 16-byte aligned.  dst/src_*_caches: HOST arrays of num_layers
+ * pool pointers (num_layers in [1, 128]); block_mapping: int64 [num_pairs, 2]
+ * in device or page-locked host memory.  A source id outside
+ * [0, src_num_blocks) or destination id outside [0, dst_num_blocks) skips the
+ * pair and sets PKV_DEVERR_COPY_ID.  Destinations must be distinct and must
+ * not overlap a source block (otherwise the result is unspecified).
+ * Returns PKV_EINVAL for pageable host memory or a pointer CUDA does not
+ * know, and PKV_EUNSUPPORTED for memory of another device; the caller keeps
+ * host pools alive and unmodified until the stream has passed the copy.
+ */
+pkv_status pkv_swap_blocks(void* const* dst_key_caches, void* const* dst_value_caches,
+                           int64_t dst_num_blocks, const void* const* src_key_caches,
+                           const void* const* src_value_caches, int64_t src_num_blocks,
+                           int num_layers, const int64_t* block_mapping, int64_t num_pairs,
+                           size_t block_bytes, pkv_stream_t stream);
+
+/*
  * Workspace for pkv_paged_attention_decode: fp32 partial results of the
  * split units, (12 * num_ctas + units) x heads_per_unit x (head_dim + 2)
  * floats, where units = num_seqs * num_kv_heads * ceil(g / 8),
@@ -175,6 +206,51 @@ pkv_status pkv_paged_attention_decode(void* out, const void* query, pkv_dtype q_
                                       float scale, const float* k_scale, const float* v_scale,
                                       void* workspace, size_t workspace_bytes, int num_ctas,
                                       pkv_stream_t stream);
+
+/*
+ * pkv_paged_attention_decode_cascade -- decode attention for batches in which
+ * groups of sequences share a prompt prefix through shared physical blocks
+ * (copy-on-write sharing: zwxr.cn section 3.4; ttlab.hopto.org section 2,
+ * parallel sampling and beam search).  The shared prefix blocks of a group are
+ * read from memory once per kv head for all members, instead of once per
+ * member; the result is the same attention as pkv_paged_attention_decode
+ * (prefix and suffix are two partial softmaxes merged exactly with the
+ * block-wise (m, l) rule of zwxr.cn section 3.3).
+ *
+ * Groups (all DEVICE int32 arrays):
+ *   group_offsets [num_groups + 1]  CSR offsets; group i's members are
+ *                                   group_members[group_offsets[i] .. group_offsets[i+1])
+ *   group_members                   sequence ids; a sequence in at most one group
+ *   group_prefix_lens [num_groups]  requested shared prefix length (tokens)
+ *   max_group_size                  upper bound on members per group (host)
+ * The prefix actually shared by group i is computed on the device: the
+ * longest run of leading table entries that all members have in common,
+ * capped by group_prefix_lens[i] and by every member's length, in whole
+ * blocks (a request longer than a member's length sets PKV_DEVERR_SEQ_LEN, as
+ * does a group with more than max_group_size members, which is then not
+ * shared).  group_offsets must be a valid non-decreasing CSR index.
+ * Sequences outside every group, groups of one member and cache dtypes other
+ * than f16/bf16 take the ordinary decode path.
+ * workspace: >= pkv_paged_attention_cascade_workspace_bytes(...) bytes, no
+ * initialisation needed.  Other arguments as pkv_paged_attention_decode.
+ */
+size_t pkv_paged_attention_cascade_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
+                                                   int head_dim, int num_groups,
+                                                   int max_group_size, int num_ctas);
+
+pkv_status pkv_paged_attention_decode_cascade(void* out, const void* query, pkv_dtype q_dtype,
+                                              const void* key_cache, const void* value_cache,
+                                              pkv_dtype cache_dtype, const int32_t* block_tables,
+                                              int max_blocks_per_seq, const int32_t* seq_lens,
+                                              int num_seqs, const int32_t* group_offsets,
+                                              const int32_t* group_members,
+                                              const int32_t* group_prefix_lens, int num_groups,
+                                              int max_group_size, int num_heads, int num_kv_heads,
+                                              int head_dim, int block_size, int64_t num_blocks,
+                                              float scale, const float* k_scale,
+                                              const float* v_scale, void* workspace,
+                                              size_t workspace_bytes, int num_ctas,
+                                              pkv_stream_t stream);
 
 /* Size of the static scratch used by pkv_paged_attention_decode_noalloc. */
 #define PKV_STATIC_WORKSPACE_BYTES (16u * 1024u * 1024u)

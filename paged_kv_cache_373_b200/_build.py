@@ -1,4 +1,5 @@
-"""Build libpkv.so in-tree: every csrc/*.cu compiled for sm_100a with nvcc.
+"""Build libpkv.so in-tree: every csrc/*.cu compiled for sm_100a with nvcc,
+and the host-only csrc/*.cpp (block manager) through nvcc's host compiler.
 
 The library links the shared CUDA runtime (libcudart.so.12) so that, inside a
 process that already loaded PyTorch, it shares torch's runtime instance and
@@ -25,7 +26,7 @@ CFLAGS = ARCH + ["-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
 
 
 def _sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _deps():
@@ -41,7 +42,7 @@ def up_to_date() -> bool:
 
 
 def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + ".o")
+    obj = os.path.join(OBJ_DIR, os.path.splitext(os.path.basename(src))[0] + ".o")
     cmd = [NVCC] + CFLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:

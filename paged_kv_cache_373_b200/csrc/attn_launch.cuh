@@ -12,28 +12,35 @@
 
 namespace pkv {
 
-template <class C>
-pkv_status launch_decode(const DecodeLaunchArgs& a, cudaStream_t st) {
+template <class C, bool kSuffix>
+pkv_status launch_decode_k(const DecodeLaunchArgs& a, cudaStream_t st) {
     static std::atomic<unsigned long long> configured{0};  // bit per device (< 64)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(PKV_ECUDA, "cudaGetDevice");
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(configured.load() & bit)) {
-        const cudaError_t e = cudaFuncSetAttribute(pkv_decode_kernel<C>,
+        const cudaError_t e = cudaFuncSetAttribute(pkv_decode_kernel<C, kSuffix>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    C::kSmemBytes);
         if (e != cudaSuccess) return fail(PKV_ECUDA, "smem opt-in: %s", cudaGetErrorString(e));
         configured.fetch_or(bit);
     }
     const DecodeParams& p = *a.params;
-    pkv_decode_kernel<C><<<a.grid, C::kWarps * 32, C::kSmemBytes, st>>>(p);
+    pkv_decode_kernel<C, kSuffix><<<a.grid, C::kWarps * 32, C::kSmemBytes, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "decode launch: %s", cudaGetErrorString(e));
     const int64_t workers = (int64_t)a.grid * C::kWarps;
-    pkv_merge_kernel<typename C::q_t, C::D, C::kTT><<<(unsigned)((workers + 7) / 8), 256, 0, st>>>(p, workers);
+    pkv_merge_kernel<typename C::q_t, C::D, C::kTT, kSuffix>
+        <<<(unsigned)workers, 32 * p.hpu, 0, st>>>(p, workers);  // a warp per head row
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "merge launch: %s", cudaGetErrorString(e));
     return PKV_OK;
+}
+
+// Plain decode, or the cascade suffix pass when the call asks for it.
+template <class C>
+pkv_status launch_decode(const DecodeLaunchArgs& a, cudaStream_t st) {
+    return a.suffix ? launch_decode_k<C, true>(a, st) : launch_decode_k<C, false>(a, st);
 }
 
 }  // namespace pkv

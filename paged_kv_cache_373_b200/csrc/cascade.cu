@@ -1,0 +1,182 @@
+// cascade.cu -- host side of pkv_paged_attention_decode_cascade: workspace
+// layout, validation, and the launch sequence of the passes in cascade.cuh.
+#include <atomic>
+
+#include "cascade.cuh"
+#include "pkv_internal.h"
+
+namespace pkv {
+namespace {
+
+constexpr int kMaxSmem = 227 * 1024;
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct CascadeLayout {
+    int g, rows, nt, row_chunks;
+    size_t dec, pre_seg_o, pre_seg_ml, seq_start, member_info, prefix_eff, suf_o, suf_ml, pre_o, pre_ml,
+        total;
+};
+
+bool cascade_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int num_groups,
+                    int max_group_size, int num_ctas, CascadeLayout* L) {
+    if (num_groups < 0 || max_group_size < 1 || num_kv_heads <= 0 || num_heads % num_kv_heads) return false;
+    const size_t dec = decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, num_ctas);
+    if (dec == 0) return false;
+    int grid = num_ctas;
+    if (grid == 0 && (cudaGetDevice(&grid) != cudaSuccess ||
+                      cudaDeviceGetAttribute(&grid, cudaDevAttrMultiProcessorCount, grid) != cudaSuccess))
+        return false;
+    L->g = num_heads / num_kv_heads;
+    L->rows = max_group_size * L->g;
+    L->nt = L->rows > 8 ? 4 : 2;
+    const int rpu = 8 * L->nt;
+    L->row_chunks = (L->rows + rpu - 1) / rpu;
+    const size_t units = (size_t)num_groups * num_kv_heads * L->row_chunks;
+    const size_t segs = (size_t)grid * kMaxWarpsPerCta + units;
+    size_t off = align256(dec);
+    L->dec = dec;
+    L->pre_seg_o = off;  off = align256(off + segs * rpu * head_dim * sizeof(float));
+    L->pre_seg_ml = off; off = align256(off + segs * rpu * sizeof(float2));
+    L->seq_start = off;  off = align256(off + (size_t)num_seqs * sizeof(int32_t));
+    L->member_info = off; off = align256(off + (size_t)num_seqs * sizeof(int4));
+    L->prefix_eff = off; off = align256(off + (size_t)num_groups * sizeof(int32_t));
+    L->suf_o = off;      off = align256(off + (size_t)num_seqs * num_heads * head_dim * sizeof(float));
+    L->suf_ml = off;     off = align256(off + (size_t)num_seqs * num_heads * sizeof(float2));
+    const size_t prows = (size_t)num_groups * num_kv_heads * L->rows;
+    L->pre_o = off;      off = align256(off + prows * head_dim * sizeof(float));
+    L->pre_ml = off;     off = align256(off + prows * sizeof(float2));
+    L->total = off;
+    return true;
+}
+
+template <class C, int NT>
+pkv_status launch_prefix(const DecodeParams& p, const CascadeParams& c, int grid, cudaStream_t st) {
+    constexpr int kSmem = C::kWarps * C::kStages * (C::kStageBytes + 8 * NT * C::kRowBytes) + 1024;
+    static_assert(kSmem <= kMaxSmem, "prefix kernel shared memory");
+    static std::atomic<unsigned long long> configured{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(PKV_ECUDA, "cudaGetDevice");
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured.load() & bit)) {
+        const cudaError_t e = cudaFuncSetAttribute(pkv_prefix_kernel<C, NT>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        if (e != cudaSuccess) return fail(PKV_ECUDA, "prefix smem opt-in: %s", cudaGetErrorString(e));
+        configured.fetch_or(bit);
+    }
+    pkv_prefix_kernel<C, NT><<<grid, C::kWarps * 32, kSmem, st>>>(p, c);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PKV_ECUDA, "prefix launch: %s", cudaGetErrorString(e));
+    const int64_t workers = (int64_t)grid * C::kWarps;
+    pkv_prefix_merge_kernel<C::D, NT><<<dim3((unsigned)workers, NT), 256, 0, st>>>(p, c, workers);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PKV_ECUDA, "prefix merge launch: %s", cudaGetErrorString(e));
+    return PKV_OK;
+}
+
+template <typename T, int D>
+pkv_status launch_prefix_t(const DecodeParams& p, const CascadeParams& c, int nt, int grid, cudaStream_t st) {
+    // 8 warps for two row tiles; 6 for four (their q slots are twice as large)
+    if (nt == 2) return launch_prefix<Cfg<T, T, D, Path::kMma16, 8, 2>, 2>(p, c, grid, st);
+    return launch_prefix<Cfg<T, T, D, Path::kMma16, 6, 2>, 4>(p, c, grid, st);
+}
+
+template <typename QT, int D>
+pkv_status launch_combine(const DecodeParams& p, const CascadeParams& c, cudaStream_t st) {
+    pkv_cascade_combine_kernel<QT, D><<<p.num_seqs, 256, 0, st>>>(p, c);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PKV_ECUDA, "combine launch: %s", cudaGetErrorString(e));
+    return PKV_OK;
+}
+
+}  // namespace
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" size_t pkv_paged_attention_cascade_workspace_bytes(int num_seqs, int num_heads,
+                                                              int num_kv_heads, int head_dim,
+                                                              int num_groups, int max_group_size,
+                                                              int num_ctas) {
+    CascadeLayout L;
+    if (!cascade_layout(num_seqs, num_heads, num_kv_heads, head_dim, num_groups, max_group_size,
+                        num_ctas, &L))
+        return 0;
+    return L.total;
+}
+
+extern "C" pkv_status pkv_paged_attention_decode_cascade(
+    void* out, const void* query, pkv_dtype q_dtype, const void* key_cache, const void* value_cache,
+    pkv_dtype cache_dtype, const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens,
+    int num_seqs, const int32_t* group_offsets, const int32_t* group_members,
+    const int32_t* group_prefix_lens, int num_groups, int max_group_size, int num_heads,
+    int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
+    const float* k_scale, const float* v_scale, void* workspace, size_t workspace_bytes, int num_ctas,
+    pkv_stream_t stream) {
+    if (num_groups < 0 || max_group_size < 1) return fail(PKV_EINVAL, "num_groups < 0 or max_group_size < 1");
+    if (num_groups > 0 && (!group_offsets || !group_members || !group_prefix_lens))
+        return fail(PKV_EINVAL, "null group array");
+    const bool rows_path = (cache_dtype == PKV_F16 || cache_dtype == PKV_BF16) && q_dtype == cache_dtype;
+    CascadeLayout L;
+    if (num_seqs > 0 && !cascade_layout(num_seqs, num_heads, num_kv_heads, head_dim, num_groups,
+                                        max_group_size, num_ctas, &L))
+        return fail(PKV_EINVAL, "invalid shapes");
+    if (num_seqs > 0 && workspace_bytes < L.total)
+        return fail(PKV_EINVAL, "cascade workspace too small: %zu < %zu bytes", workspace_bytes, L.total);
+    // the suffix pass is the ordinary decode path on the first workspace region
+    DecodeParams p;
+    DecodeLauncher launch;
+    int grid = 0;
+    pkv_status st = decode_prepare(&p, &launch, &grid, out, query, q_dtype, key_cache, value_cache,
+                                   cache_dtype, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+                                   num_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                                   k_scale, v_scale, workspace, num_seqs > 0 ? L.dec : 0, num_ctas);
+    if (st != PKV_OK || num_seqs == 0) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    DecodeLaunchArgs a{&p, grid};
+    if (num_groups == 0 || !rows_path) return launch(a, cs);  // no sharing to exploit: plain decode
+
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    CascadeParams c{};
+    c.grp_offsets = group_offsets;
+    c.grp_members = group_members;
+    c.grp_prefix = group_prefix_lens;
+    c.prefix_eff = reinterpret_cast<int32_t*>(base + L.prefix_eff);
+    c.seq_start = reinterpret_cast<int32_t*>(base + L.seq_start);
+    c.member_info = reinterpret_cast<int4*>(base + L.member_info);
+    c.pre_o = reinterpret_cast<float*>(base + L.pre_o);
+    c.pre_ml = reinterpret_cast<float2*>(base + L.pre_ml);
+    c.suf_o = reinterpret_cast<float*>(base + L.suf_o);
+    c.suf_ml = reinterpret_cast<float2*>(base + L.suf_ml);
+    c.num_groups = num_groups;
+    c.rows = L.rows;
+    c.row_chunks = L.row_chunks;
+
+    cudaError_t e = cudaMemsetAsync(c.seq_start, 0, (size_t)num_seqs * sizeof(int32_t), cs);
+    if (e != cudaSuccess) return fail(PKV_ECUDA, "seq_start memset: %s", cudaGetErrorString(e));
+    pkv_cascade_setup_kernel<<<num_groups, 256, 0, cs>>>(p, c);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PKV_ECUDA, "setup launch: %s", cudaGetErrorString(e));
+
+    DecodeParams pp = p;  // prefix pass: its own split segments
+    pp.ws_o = reinterpret_cast<float*>(base + L.pre_seg_o);
+    pp.ws_ml = reinterpret_cast<float2*>(base + L.pre_seg_ml);
+    if (cache_dtype == PKV_F16)
+        st = head_dim == 64 ? launch_prefix_t<__half, 64>(pp, c, L.nt, grid, cs)
+                            : launch_prefix_t<__half, 128>(pp, c, L.nt, grid, cs);
+    else
+        st = head_dim == 64 ? launch_prefix_t<__nv_bfloat16, 64>(pp, c, L.nt, grid, cs)
+                            : launch_prefix_t<__nv_bfloat16, 128>(pp, c, L.nt, grid, cs);
+    if (st != PKV_OK) return st;
+
+    p.seq_start = c.seq_start;  // suffix pass: members from their shared-prefix end
+    p.part_o = c.suf_o;
+    p.part_ml = c.suf_ml;
+    DecodeLaunchArgs sa{&p, grid, true};
+    if ((st = launch(sa, cs)) != PKV_OK) return st;
+
+    if (cache_dtype == PKV_F16)
+        return head_dim == 64 ? launch_combine<__half, 64>(p, c, cs) : launch_combine<__half, 128>(p, c, cs);
+    return head_dim == 64 ? launch_combine<__nv_bfloat16, 64>(p, c, cs)
+                          : launch_combine<__nv_bfloat16, 128>(p, c, cs);
+}

@@ -1,0 +1,460 @@
+// cascade.cuh -- decode attention for sequences that share a prompt prefix
+// (copy-on-write sharing, zwxr.cn section 3.4; ttlab.hopto.org section 2
+// "共享区块"): the shared prefix blocks are streamed once per (group, kv head)
+// and serve the query rows of every member of the group, instead of once per
+// member.  The result is the same attention as pkv_paged_attention_decode:
+// the prefix part and each member's own suffix are two partial softmaxes
+// merged exactly with the block-wise (m, l) rule of zwxr.cn section 3.3.
+//
+// Passes (all on the caller's stream):
+//   1. pkv_cascade_setup_kernel: per group, the effective shared prefix =
+//      the longest run of leading blocks that every member's table shares,
+//      capped by the requested prefix and by every member's length, in whole
+//      blocks; scatter it to the members as their suffix start.
+//   2. pkv_prefix_kernel (+ pkv_prefix_merge_kernel for split units):
+//      work unit = (group, kv head, chunk of 8*NT member query rows); the
+//      same warp-level cp.async streaming as the decode kernel, with NT
+//      tensor-core N tiles so one K/V tile feeds every member row.
+//   3. pkv_decode_kernel with seq_start = the suffix starts and partial
+//      output for members (the ordinary path for everyone else).
+//   4. pkv_cascade_combine_kernel: out = merge(prefix partial, suffix partial).
+#pragma once
+
+#include "paged_attention.cuh"
+
+namespace pkv {
+
+struct CascadeParams {
+    const int32_t* grp_offsets;  // [G + 1] CSR offsets into grp_members
+    const int32_t* grp_members;  // member sequence ids
+    const int32_t* grp_prefix;   // [G] requested shared prefix (tokens)
+    int32_t* prefix_eff;         // [G] effective shared prefix (tokens), written by setup
+    int32_t* seq_start;          // [S] suffix start per sequence, written by setup
+    int4* member_info;           // [S] member slot k < grp_offsets[G]: (sequence, group, index in
+                                 // the group, 1 if the group shares a prefix), written by setup
+    float* pre_o;                // [G * Hkv * R * D] prefix partial o (unnormalised)
+    float2* pre_ml;              // [G * Hkv * R] prefix partial (m, l), log2 domain
+    float* suf_o;                // [S * Hq * D] suffix partial o of members
+    float2* suf_ml;              // [S * Hq]
+    int num_groups;
+    int rows;                    // R = max_group_size * g (member query rows per kv head)
+    int row_chunks;              // ceil(R / (8 * NT))
+};
+
+// Pass 1 (one CTA per group; seq_start zeroed beforehand): the group's
+// effective prefix, scattered to its members as their suffix start.
+__global__ void __launch_bounds__(256)
+pkv_cascade_setup_kernel(const DecodeParams p, const CascadeParams c) {
+    __shared__ int s_min, s_diff, s_bad;
+    const int g = blockIdx.x, tid = threadIdx.x;
+    const int cap = p.max_blocks_per_seq * p.block_size;
+    const int o0 = __ldg(c.grp_offsets + g), o1 = __ldg(c.grp_offsets + g + 1);
+    if (tid == 0) { s_min = cap; s_diff = 0x7fffffff; s_bad = 0; }
+    __syncthreads();
+    int minlen = cap, bad = 0;
+    for (int i = o0 + tid; i < o1; i += blockDim.x) {
+        const int s = __ldg(c.grp_members + i);
+        if (s < 0 || s >= p.num_seqs) bad = 1;
+        else minlen = min(minlen, clamp_len(__ldg(p.seq_lens + s), cap));
+    }
+    if (minlen < cap) atomicMin(&s_min, minlen);
+    if (bad) atomicOr(&s_bad, 1);
+    __syncthreads();
+    int pre = __ldg(c.grp_prefix + g);
+    pre = pre < 0 ? 0 : pre;
+    minlen = s_min;
+    // a request past a member's end, a member id outside [0, num_seqs) or a
+    // group larger than max_group_size (c.rows / g) is flagged; such a group
+    // (and any single-member group) shares nothing
+    const bool fits = (o1 - o0) * p.g <= c.rows;
+    if (tid == 0 && (pre > minlen || s_bad || !fits)) raise_error(p.err, PKV_DEVERR_SEQ_LEN);
+    const bool share = o1 - o0 > 1 && fits && !s_bad;
+    const int nblk = share ? min(pre, minlen) / p.block_size : 0;
+    // longest common run of leading physical blocks: thread per block, the
+    // members' entries loaded independently
+    if (nblk > 0) {
+        const int32_t* first = p.block_tables + (int64_t)__ldg(c.grp_members + o0) * p.max_blocks_per_seq;
+        for (int b = tid; b < nblk; b += blockDim.x) {
+            const int f = __ldg(first + b);
+            bool miss = false;
+#pragma unroll 8
+            for (int i = o0 + 1; i < o1; ++i)
+                miss |= __ldg(p.block_tables + (int64_t)__ldg(c.grp_members + i) * p.max_blocks_per_seq + b) != f;
+            if (miss) { atomicMin(&s_diff, b); break; }
+        }
+    }
+    __syncthreads();
+    const int eff = min(nblk, s_diff) * p.block_size;
+    if (tid == 0) c.prefix_eff[g] = eff;
+    for (int i = o0 + tid; i < o1; i += blockDim.x) {
+        const int s = __ldg(c.grp_members + i);
+        if (eff > 0) c.seq_start[s] = eff;  // eff > 0: every member id is valid
+        if (i < p.num_seqs) c.member_info[i] = make_int4(s, g, i - o0, eff > 0);
+    }
+}
+
+// ---- tile math with NT tensor-core N tiles of 8 member query rows ----------
+template <class C, int NT>
+struct MmaRowsConsumer {
+    static constexpr bool kOpBf16 = std::is_same<typename C::kv_t, __nv_bfloat16>::value;
+    static constexpr int D = C::D;
+    static constexpr int KS = D / 16;
+    static constexpr int MT = D / 16;
+    static constexpr int R = 8 * NT;  // rows per unit
+    static_assert(NT == 2 || NT == 4, "row tiles");
+    static_assert(C::kPath == Path::kMma16 && C::kTT == 16, "16-bit caches, 16-token tiles");
+
+    float acc[MT][NT][4];
+    float m[NT][2], l[NT][2];
+    uint32_t qb;  // shared address of the unit's q rows (swizzled, R rows)
+    float sl;
+
+    __device__ void reset() {
+#pragma unroll
+        for (int i = 0; i < MT; ++i)
+#pragma unroll
+            for (int n = 0; n < NT; ++n) acc[i][n][0] = acc[i][n][1] = acc[i][n][2] = acc[i][n][3] = 0.f;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) m[n][0] = m[n][1] = -INFINITY, l[n][0] = l[n][1] = 0.f;
+    }
+    // rows >= nrows of the slot are zeroed (they hold no member)
+    __device__ void load_q(uint8_t* qs, int nrows, float scale_log2) {
+        const int lane = threadIdx.x & 31;
+        for (int idx = lane; idx < (R - nrows) * (C::kRowBytes / 16); idx += 32) {
+            const int r = nrows + idx / (C::kRowBytes / 16), ch = idx % (C::kRowBytes / 16);
+            *reinterpret_cast<uint4*>(qs + sw_off<R>(r, ch)) = make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+        qb = smem_u32(qs);
+        sl = scale_log2;
+    }
+
+    __device__ void tile(uint8_t* kt, uint8_t* vt, int valid) {
+        const int lane = threadIdx.x & 31, gid = lane >> 2;
+        if (valid < 16) zero_tail_rows<C::kNSub, 16>(vt, valid, lane);
+        const uint32_t kb = smem_u32(kt), vb = smem_u32(vt);
+        const int r = lane & 7, mtx = lane >> 3;
+        float s[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            uint32_t a[4];
+            ldsm_x4(a, kb + sw_off<16>(r + ((mtx & 1) << 3), 2 * kk + (mtx >> 1)));
+#pragma unroll
+            for (int n2 = 0; n2 < NT / 2; ++n2) {
+                uint32_t b[4];  // b0, b1 of n-tile 2*n2 and of 2*n2+1
+                ldsm_x4(b, qb + sw_off<R>(8 * (2 * n2 + (mtx >> 1)) + r, 2 * kk + (mtx & 1)));
+                mma16816<kOpBf16>(s[2 * n2], a, b[0], b[1]);
+                mma16816<kOpBf16>(s[2 * n2 + 1], a, b[2], b[3]);
+            }
+        }
+        uint32_t b0[NT], b1[NT], c0[NT], c1[NT];
+        float al[NT][2];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            float x0 = s[n][0] * sl, x1 = s[n][1] * sl, x2 = s[n][2] * sl, x3 = s[n][3] * sl;
+            if (gid >= valid) x0 = x1 = -INFINITY;
+            if (gid + 8 >= valid) x2 = x3 = -INFINITY;
+            float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, o));
+            }
+            const float mn0 = fmaxf(m[n][0], mx0), mn1 = fmaxf(m[n][1], mx1);
+            al[n][0] = ex2(m[n][0] - mn0);
+            al[n][1] = ex2(m[n][1] - mn1);
+            m[n][0] = mn0;
+            m[n][1] = mn1;
+            const float e0 = ex2(x0 - mn0), e1 = ex2(x1 - mn1), e2 = ex2(x2 - mn0), e3 = ex2(x3 - mn1);
+            const uint32_t X0 = pack2<kOpBf16>(e0, e1), X1 = pack2<kOpBf16>(e2, e3);
+            if constexpr (kOpBf16) {  // P as hi + lo bf16 parts (see MmaConsumer)
+                const float2 h0 = unpack2<true>(X0), h1 = unpack2<true>(X1);
+                c0[n] = movm_trans(pack2<true>(e0 - h0.x, e1 - h0.y));
+                c1[n] = movm_trans(pack2<true>(e2 - h1.x, e3 - h1.y));
+                l[n][0] = l[n][0] * al[n][0] + (e0 + e2);
+                l[n][1] = l[n][1] * al[n][1] + (e1 + e3);
+            } else {
+                const float2 p0 = unpack2<false>(X0), p1 = unpack2<false>(X1);
+                l[n][0] = l[n][0] * al[n][0] + p0.x + p1.x;
+                l[n][1] = l[n][1] * al[n][1] + p0.y + p1.y;
+                c0[n] = c1[n] = 0u;
+            }
+            b0[n] = movm_trans(X0);
+            b1[n] = movm_trans(X1);
+        }
+#pragma unroll
+        for (int mi = 0; mi < MT; ++mi) {
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                acc[mi][n][0] *= al[n][0]; acc[mi][n][1] *= al[n][1];
+                acc[mi][n][2] *= al[n][0]; acc[mi][n][3] *= al[n][1];
+            }
+        }
+        const int t = r + ((mtx >> 1) << 3);
+#pragma unroll
+        for (int mi = 0; mi < MT; ++mi) {
+            uint32_t a[4];
+            ldsm_x4_trans(a, vb + sw_off<16>(t, 2 * mi + (mtx & 1)));
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                mma16816<kOpBf16>(acc[mi][n], a, b0[n], b1[n]);
+                if constexpr (kOpBf16) mma16816<true>(acc[mi][n], a, c0[n], c1[n]);
+            }
+        }
+    }
+
+    // Partial (m, l, o) of every valid row: to the workspace segment (split
+    // unit) or straight to the prefix partial rows.
+    __device__ void finish(float* o_rows, float2* ml_rows, int nrows) {
+        const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            float a0 = l[n][0], a1 = l[n][1];
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                a0 += __shfl_xor_sync(kFull, a0, o);
+                a1 += __shfl_xor_sync(kFull, a1, o);
+            }
+            const int h0 = 8 * n + 2 * tig, h1 = h0 + 1;
+#pragma unroll
+            for (int mi = 0; mi < MT; ++mi) {
+                const int d0 = 16 * mi + gid, d1 = d0 + 8;
+                if (h0 < nrows) { o_rows[h0 * D + d0] = acc[mi][n][0]; o_rows[h0 * D + d1] = acc[mi][n][2]; }
+                if (h1 < nrows) { o_rows[h1 * D + d0] = acc[mi][n][1]; o_rows[h1 * D + d1] = acc[mi][n][3]; }
+            }
+            if (gid == 0) {
+                if (h0 < nrows) ml_rows[h0] = make_float2(m[n][0], a0);
+                if (h1 < nrows) ml_rows[h1] = make_float2(m[n][1], a1);
+            }
+        }
+    }
+};
+
+// Pass 2: the shared prefixes, every warp an independent worker over an equal
+// share of all (group, kv head, row chunk) tiles.
+template <class C, int NT>
+__global__ void __launch_bounds__(C::kWarps * 32, 1)
+pkv_prefix_kernel(const DecodeParams p, const CascadeParams c) {
+    constexpr int R = 8 * NT;
+    constexpr int kQSlot = R * C::kRowBytes;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t* stages = smem + warp * C::kStages * (C::kStageBytes + kQSlot);
+    uint8_t* qslots = stages + C::kStages * C::kStageBytes;
+
+    const Lens<false> ln{c.prefix_eff, nullptr, c.num_groups, p.num_kv_heads * c.row_chunks, 0x7fffffff};
+    const int64_t workers = (int64_t)gridDim.x * C::kWarps;
+    const int64_t wid = (int64_t)blockIdx.x * C::kWarps + warp;
+    const int64_t W = total_tiles<16>(ln);
+    const int64_t chunk = (W + workers - 1) / workers;
+    const int64_t tb = min(W, wid * chunk), te = min(W, tb + chunk);
+    if (tb >= te) return;
+
+    // member rows of unit j of group g: rows [R*rc, R*rc + R) of the group's
+    // members x q heads of kv head kh (row = member * g + head)
+    auto unit_rows = [&](int g, int j, int& kh, int& rc, int& nrows, int& o0) {
+        kh = j / c.row_chunks;
+        rc = j % c.row_chunks;
+        o0 = __ldg(c.grp_offsets + g);
+        const int total = (__ldg(c.grp_offsets + g + 1) - o0) * p.g;
+        nrows = max(0, min(R, total - R * rc));
+    };
+    auto issue = [&](const Walk<16>& w, TablePrefetch& tp, uint8_t* stg, uint8_t* qslot) {
+        int kh, rc, nrows, o0;
+        unit_rows(w.s, w.j, kh, rc, nrows, o0);
+        const int first_member = __ldg(c.grp_members + o0);
+        const int tok = w.i * 16;
+        const int nblk = (w.L + p.block_size - 1) / p.block_size;
+        int phys = tp.get(p, first_member, tok / p.block_size, nblk, lane);
+        if (phys < 0 || phys >= p.num_blocks) {
+            if (lane == 0) raise_error(p.err, PKV_DEVERR_BLOCK_ID);
+            phys = 0;
+        }
+        const int tok0 = tok % p.block_size;
+        const int64_t row_stride = (int64_t)p.num_kv_heads * C::kRowBytes;
+        const int64_t base = (((int64_t)phys * p.block_size + tok0) * p.num_kv_heads + kh) * C::kRowBytes;
+        const uint32_t kdst = smem_u32(stg), vdst = smem_u32(stg + C::kTensorTile);
+        const int cr = lane % C::kChunksPerRow, r0 = lane / C::kChunksPerRow;
+#pragma unroll
+        for (int it = 0; it < 16 / C::kRowsPerInst; ++it) {
+            const int t = it * C::kRowsPerInst + r0;
+            const int64_t off = t * row_stride + cr * 16;
+            const uint32_t so = sw_off<16>(t, cr);
+            cp_async16(kdst + so, p.key_cache + base + off);
+            cp_async16(vdst + so, p.value_cache + base + off);
+        }
+        if (w.first()) {
+            constexpr int CPR = C::kRowBytes / 16;
+            for (int idx = lane; idx < nrows * CPR; idx += 32) {
+                const int rr = idx / CPR, ch = idx % CPR;
+                const int row = R * rc + rr;                      // member row within the group
+                const int s = __ldg(c.grp_members + o0 + row / p.g);
+                const uint8_t* src = reinterpret_cast<const uint8_t*>(p.q) +
+                    ((int64_t)s * p.num_heads + (int64_t)kh * p.g + row % p.g) * C::kRowBytes + ch * 16;
+                cp_async16(smem_u32(qslot + sw_off<R>(rr, ch)), src);
+            }
+        }
+    };
+
+    Walk<16> iw, cw;
+    iw.init(ln, tb, te);
+    cw = iw;
+    TablePrefetch tp;
+#pragma unroll 1
+    for (int k = 0; k < C::kStages - 1; ++k) {
+        if (!iw.done) issue(iw, tp, stages + k * C::kStageBytes, qslots + (iw.ord % C::kStages) * kQSlot);
+        cp_async_commit();
+        iw.advance(ln);
+    }
+    MmaRowsConsumer<C, NT> cs;
+#pragma unroll 1
+    for (int n = 0; !cw.done; ++n) {
+        if (!iw.done)
+            issue(iw, tp, stages + ((n + C::kStages - 1) % C::kStages) * C::kStageBytes,
+                  qslots + (iw.ord % C::kStages) * kQSlot);
+        cp_async_commit();
+        iw.advance(ln);
+        cp_async_wait<C::kStages - 1>();
+        __syncwarp();
+        int kh, rc, nrows, o0;
+        unit_rows(cw.s, cw.j, kh, rc, nrows, o0);
+        if (cw.first()) {
+            cs.load_q(qslots + (cw.ord % C::kStages) * kQSlot, nrows, p.scale_log2);
+            cs.reset();
+        }
+        uint8_t* kt = stages + (n % C::kStages) * C::kStageBytes;
+        cs.tile(kt, kt + C::kTensorTile, min(16, cw.L - cw.i * 16));
+        if (cw.last()) {
+            const bool split = (cw.seg_i0 != 0) || (cw.i != cw.nt - 1);
+            const int64_t unit = (int64_t)cw.s * ln.units + cw.j;
+            if (split) {
+                const int64_t seg = wid + unit;
+                cs.finish(p.ws_o + seg * R * C::D, p.ws_ml + seg * R, nrows);
+            } else {
+                const int64_t row0 = ((int64_t)cw.s * p.num_kv_heads + kh) * c.rows + R * rc;
+                cs.finish(c.pre_o + row0 * C::D, c.pre_ml + row0, nrows);
+            }
+        }
+        __syncwarp();
+        cw.advance(ln);
+    }
+    cp_async_wait<0>();
+}
+
+// Merge of the prefix units split between workers (into the prefix partial
+// rows).  Grid (workers, NT): CTA (b >= 1, y) owns rows 8y..8y+7 of the unit
+// cut by worker boundary b if b is the unit's first interior boundary, one
+// warp per row; CTA (0, 0) marks the rows of groups with no shared prefix as
+// empty partials.
+template <int D, int NT>
+__global__ void __launch_bounds__(256)
+pkv_prefix_merge_kernel(const DecodeParams p, const CascadeParams c, int64_t workers) {
+    constexpr int R = 8 * NT;
+    __shared__ int64_t sh[6];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t b = blockIdx.x;
+    const Lens<false> ln{c.prefix_eff, nullptr, c.num_groups, p.num_kv_heads * c.row_chunks, 0x7fffffff};
+    if (b == 0) {
+        if (blockIdx.y != 0) return;
+        for (int g = warp; g < c.num_groups; g += 8) {
+            if (__ldg(c.prefix_eff + g) != 0) continue;
+            const int64_t r0 = (int64_t)g * p.num_kv_heads * c.rows;
+            for (int i = lane; i < p.num_kv_heads * c.rows; i += 32) c.pre_ml[r0 + i] = make_float2(-INFINITY, 0.f);
+        }
+        return;
+    }
+    if (warp == 0) {
+        int64_t flag = 0, unit = 0, bf = 0, bl = 0, row0 = 0, nrows = 0;
+        const int64_t W = total_tiles<16>(ln);
+        const int64_t chunk = (W + workers - 1) / workers;
+        const int64_t P = b * chunk;
+        if (P < W) {
+            const SeqHit hit = find_seq<16>(ln, P);
+            const int nt = ntiles_of<16>(hit.L);
+            const int j = (int)((P - hit.base) / nt);
+            const int off = (int)((P - hit.base) % nt);
+            const int64_t T0 = hit.base + (int64_t)j * nt;
+            if (off != 0 && (b - 1) * chunk <= T0) {
+                const int kh = j / c.row_chunks, rc = j % c.row_chunks;
+                const int o0 = __ldg(c.grp_offsets + hit.s);
+                flag = 1;
+                unit = (int64_t)hit.s * ln.units + j;
+                bf = T0 / chunk;
+                bl = (T0 + nt - 1) / chunk;
+                row0 = ((int64_t)hit.s * p.num_kv_heads + kh) * c.rows + R * rc;
+                nrows = max(0, min(R, (__ldg(c.grp_offsets + hit.s + 1) - o0) * p.g - R * rc));
+            }
+        }
+        if (lane == 0) { sh[0] = flag; sh[1] = unit; sh[2] = bf; sh[3] = bl; sh[4] = row0; sh[5] = nrows; }
+    }
+    __syncthreads();
+    const int h = (int)blockIdx.y * 8 + warp;
+    if (!sh[0] || h >= (int)sh[5]) return;
+    const int64_t unit = sh[1], bf = sh[2], row0 = sh[4];
+    const int n = (int)(sh[3] - bf + 1);  // segments of the unit
+    // (m, l) of the segments, lane-parallel
+    float M = -INFINITY;
+    for (int i = lane; i < n; i += 32) M = fmaxf(M, p.ws_ml[(bf + i + unit) * R + h].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+    float ls = 0.f;
+    for (int i = lane; i < n; i += 32) {
+        const float2 ml = p.ws_ml[(bf + i + unit) * R + h];
+        ls += ml.x == -INFINITY ? 0.f : ml.y * ex2(ml.x - M);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(kFull, ls, o);
+    constexpr int PER = D / 32;
+    float o[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) o[e] = 0.f;
+#pragma unroll 4
+    for (int i = 0; i < n; ++i) {
+        const float2 ml = p.ws_ml[(bf + i + unit) * R + h];
+        const float f = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);
+        const float* src = p.ws_o + ((bf + i + unit) * R + h) * D;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[e] += src[lane + 32 * e] * f;
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) c.pre_o[(row0 + h) * D + lane + 32 * e] = o[e];
+    if (lane == 0) c.pre_ml[row0 + h] = make_float2(M, ls);
+}
+
+// Pass 4: out[s, h] = merge(prefix partial, suffix partial) for every member
+// of a group with a shared prefix (one CTA per member slot, one warp per head).
+template <typename QT, int D>
+__global__ void __launch_bounds__(256)
+pkv_cascade_combine_kernel(const DecodeParams p, const CascadeParams c) {
+    const int k = blockIdx.x;  // member slot
+    const int total = __ldg(c.grp_offsets + c.num_groups);
+    const int4 info = c.member_info[k];  // (s, g, index in group, shared)
+    if (k >= total || !info.w) return;   // no sharing: the suffix pass wrote out
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int s = info.x, g = info.y, mi = info.z;
+    constexpr int PER = D / 32;
+#pragma unroll 2
+    for (int h = warp; h < p.num_heads; h += blockDim.x >> 5) {
+        const int kh = h / p.g;
+        const int64_t pr = ((int64_t)g * p.num_kv_heads + kh) * c.rows + (int64_t)mi * p.g + h % p.g;
+        const int64_t sr = (int64_t)s * p.num_heads + h;
+        const float2 a = c.pre_ml[pr], b = c.suf_ml[sr];
+        const float M = fmaxf(a.x, b.x);
+        const float fa = (a.x == -INFINITY) ? 0.f : ex2(a.x - M);
+        const float fb = (b.x == -INFINITY) ? 0.f : ex2(b.x - M);
+        const float ls = a.y * fa + b.y * fb;
+        QT* out = reinterpret_cast<QT*>(p.out) + sr * D;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int d = lane + 32 * e;
+            const float o = c.pre_o[pr * D + d] * fa + c.suf_o[sr * D + d] * fb;
+            out[d] = from_f32<QT>(ls > 0.f ? o / ls : 0.f);
+        }
+    }
+}
+
+}  // namespace pkv

@@ -60,29 +60,62 @@ struct DecodeParams {
     int hpu;               // heads per unit stride in the workspace = min(8, g)
     int max_blocks_per_seq, block_size, num_blocks;
     float scale_log2;      // scale * log2(e)
+    // Cascade suffix pass only: the first token attended per sequence, and for
+    // sequences with a non-zero start the unnormalised o and (m, l) partials
+    // that replace out.
+    const int32_t* seq_start;  // [num_seqs] or null (all from 0)
+    float* part_o;             // [num_seqs * num_heads * D] or null
+    float2* part_ml;           // [num_seqs * num_heads]
 };
 
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
+
+// Per-sequence token ranges [start_s, L_s) the kernel attends over; kStart
+// false: every range starts at token 0 (start is not read).
+template <bool kStart>
+struct Lens {
+    static constexpr bool kHasStart = kStart;
+    const int32_t* len;
+    const int32_t* start;
+    int S, units, cap;
+    __device__ __forceinline__ int first(int s) const {
+        if constexpr (!kStart) {
+            return 0;
+        } else {
+            const int st = __ldg(start + s);
+            return st < 0 ? 0 : st;
+        }
+    }
+    __device__ __forceinline__ int full(int s) const { return clamp_len(__ldg(len + s), cap); }
+    // attended length (tokens after the start)
+    __device__ __forceinline__ int eff(int s) const {
+        if constexpr (!kStart) {
+            return full(s);
+        } else {
+            const int L = full(s), st = first(s);
+            return st >= L ? 0 : L - st;
+        }
+    }
+};
 template <int TT>
 __device__ __forceinline__ int ntiles_of(int L) { return (L + TT - 1) / TT; }
 
 // Warp-collective: total tiles W = units_per_seq * sum_s ceil(L_s / 16);
 // *bad_len is set when some length is negative or overruns its table row.
-template <int TT>
-__device__ inline int64_t total_tiles(const int32_t* seq_lens, int S, int units, int cap,
-                                      bool* bad_len = nullptr) {
+template <int TT, class LN>
+__device__ inline int64_t total_tiles(const LN& ln, bool* bad_len = nullptr) {
     const int lane = threadIdx.x & 31;
     int64_t tot = 0;
     bool bad = false;
-    for (int s0 = 0; s0 < S; s0 += 256) {
+    for (int s0 = 0; s0 < ln.S; s0 += 256) {
         int part = 0;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const int s = s0 + lane * 8 + k;
-            if (s < S) {
-                const int L = __ldg(seq_lens + s);
-                bad |= (L < 0 || L > cap);
-                part += ntiles_of<TT>(clamp_len(L, cap));
+            if (s < ln.S) {
+                const int L = __ldg(ln.len + s);
+                bad |= (L < 0 || L > ln.cap);
+                part += ntiles_of<TT>(LN::kHasStart ? ln.eff(s) : clamp_len(L, ln.cap));
             }
         }
 #pragma unroll
@@ -90,27 +123,27 @@ __device__ inline int64_t total_tiles(const int32_t* seq_lens, int S, int units,
         tot += part;
     }
     if (bad_len) *bad_len = __any_sync(kFull, bad);
-    return tot * units;
+    return tot * ln.units;
 }
 
 struct SeqHit {
     int s;          // sequence holding tile P (num_seqs if none)
     int64_t base;   // index of its first tile
-    int L;          // its clamped length
+    int L;          // its attended length
 };
 
 // Warp-collective: the sequence whose tiles contain global tile P.
-template <int TT>
-__device__ inline SeqHit find_seq(const int32_t* seq_lens, int S, int units, int cap, int64_t P) {
+template <int TT, class LN>
+__device__ inline SeqHit find_seq(const LN& ln, int64_t P) {
     const int lane = threadIdx.x & 31;
     int64_t base = 0;
-    for (int s0 = 0; s0 < S; s0 += 256) {
+    for (int s0 = 0; s0 < ln.S; s0 += 256) {
         int64_t w[8];
         int64_t part = 0;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const int s = s0 + lane * 8 + k;
-            w[k] = (s < S) ? (int64_t)ntiles_of<TT>(clamp_len(__ldg(seq_lens + s), cap)) * units : 0;
+            w[k] = (s < ln.S) ? (int64_t)ntiles_of<TT>(ln.eff(s)) * ln.units : 0;
             part += w[k];
         }
         int64_t incl = part;
@@ -134,30 +167,37 @@ __device__ inline SeqHit find_seq(const int32_t* seq_lens, int S, int units, int
             }
             found = max(__shfl_sync(kFull, found, src) - 1, 0);
             at = __shfl_sync(kFull, at, src);
-            return SeqHit{found, at, clamp_len(__ldg(seq_lens + found), cap)};
+            return SeqHit{found, at, ln.eff(found)};
         }
         base += __shfl_sync(kFull, incl, 31);
     }
-    return SeqHit{S, base, 0};
+    return SeqHit{ln.S, base, 0};
 }
 
+// First attended token of the walk's current sequence: a field only when
+// ranges may start past token 0.
+template <bool kStart> struct WalkStart { int st; };
+template <> struct WalkStart<false> { static constexpr int st = 0; };
+
 // Walk over a worker's tiles (TT tokens each) in order: (sequence, unit j, tile i).
-template <int TT>
-struct Walk {
-    int s, L, nt, j, i, seg_i0, ord;
+template <int TT, bool kStart = false>
+struct Walk : WalkStart<kStart> {
+    int s, L, nt, j, i, seg_i0, ord;  // L: attended length
     int64_t T, te;
     bool done;
 
-    __device__ void init(const int32_t* seq_lens, int S, int units, int cap, int64_t tb, int64_t te_) {
+    __device__ void init(const Lens<kStart>& ln, int64_t tb, int64_t te_) {
         te = te_;
         T = tb;
         done = tb >= te_;
         ord = 0;
         s = 0; L = 0; nt = 1; j = 0; i = 0; seg_i0 = 0;
+        if constexpr (kStart) this->st = 0;
         if (done) return;
-        const SeqHit h = find_seq<TT>(seq_lens, S, units, cap, tb);
+        const SeqHit h = find_seq<TT>(ln, tb);
         s = h.s;
         L = h.L;
+        if constexpr (kStart) this->st = ln.first(s);
         nt = ntiles_of<TT>(L);
         j = (int)((tb - h.base) / nt);
         i = (int)((tb - h.base) % nt);
@@ -165,20 +205,21 @@ struct Walk {
     }
     __device__ bool first() const { return i == seg_i0; }
     __device__ bool last() const { return i == nt - 1 || T == te - 1; }
-    __device__ void advance(const int32_t* seq_lens, int S, int units, int cap) {
+    __device__ void advance(const Lens<kStart>& ln) {
         if (done) return;
         if (++T >= te) { done = true; return; }
         if (++i == nt) {
             i = 0;
             seg_i0 = 0;
             ++ord;
-            if (++j == units) {
+            if (++j == ln.units) {
                 j = 0;
                 do {  // a later non-empty sequence exists because T < te <= W
                     ++s;
-                    L = (s < S) ? clamp_len(__ldg(seq_lens + s), cap) : TT;
+                    L = (s < ln.S) ? ln.eff(s) : TT;
                     nt = ntiles_of<TT>(L);
                 } while (nt == 0);
+                if constexpr (kStart) this->st = (s < ln.S) ? ln.first(s) : 0;
             }
         }
     }
@@ -251,16 +292,20 @@ __device__ __forceinline__ uint32_t sw_off(int t, int c) {
 // Output / workspace sink of one unit segment.
 struct Sink {
     bool split;
+    bool part;     // whole unit, result to part_o / part_ml (read only when kPart)
     int64_t seg;   // workspace segment (split only)
     int64_t row0;  // output row (s * Hq + first head of the chunk)
     int nh;
 };
 
-template <typename QT>
+// kPart: the cascade suffix pass, whose whole units may be partials.
+template <typename QT, bool kPart>
 __device__ __forceinline__ void sink_write(const DecodeParams& p, const Sink& k, int D, int h, int d,
                                            float o, float l, float vscale) {
     if (h >= k.nh) return;
-    if (!k.split) {
+    if (kPart && k.part) {
+        p.part_o[(k.row0 + h) * D + d] = o * vscale;
+    } else if (!k.split) {
         QT* out = reinterpret_cast<QT*>(p.out) + (k.row0 + h) * D + d;
         *out = from_f32<QT>(l > 0.f ? o * vscale / l : 0.f);
     } else {
@@ -471,6 +516,7 @@ struct MmaConsumer {
     }
 
     // End of a unit segment: the output (whole unit) or a partial (split).
+    template <bool kPart>
     __device__ void finish(const DecodeParams& p, const Sink& k, float vscale) {
         using QT = typename C::q_t;
         const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
@@ -486,12 +532,18 @@ struct MmaConsumer {
             int d0, d1;
             if constexpr (!kFp8) { d0 = 16 * mi + gid; d1 = d0 + 8; }
             else { d0 = 16 * gid + 2 * mi; d1 = d0 + 1; }
-            sink_write<QT>(p, k, D, h0, d0, acc[mi][0], a0, vscale);
-            sink_write<QT>(p, k, D, h1, d0, acc[mi][1], a1, vscale);
-            sink_write<QT>(p, k, D, h0, d1, acc[mi][2], a0, vscale);
-            sink_write<QT>(p, k, D, h1, d1, acc[mi][3], a1, vscale);
+            sink_write<QT, kPart>(p, k, D, h0, d0, acc[mi][0], a0, vscale);
+            sink_write<QT, kPart>(p, k, D, h1, d0, acc[mi][1], a1, vscale);
+            sink_write<QT, kPart>(p, k, D, h0, d1, acc[mi][2], a0, vscale);
+            sink_write<QT, kPart>(p, k, D, h1, d1, acc[mi][3], a1, vscale);
         }
-        if (k.split && gid == 0) {
+        if constexpr (kPart) {
+            if (gid == 0 && (k.split || k.part)) {
+                float2* ml = k.part ? p.part_ml + k.row0 : p.ws_ml + k.seg * p.hpu;
+                if (h0 < k.nh) ml[h0] = make_float2(m0, a0);
+                if (h1 < k.nh) ml[h1] = make_float2(m1, a1);
+            }
+        } else if (k.split && gid == 0) {
             if (h0 < k.nh) p.ws_ml[k.seg * p.hpu + h0] = make_float2(m0, a0);
             if (h1 < k.nh) p.ws_ml[k.seg * p.hpu + h1] = make_float2(m1, a1);
         }
@@ -589,6 +641,7 @@ struct F32Consumer {
             }
         }
     }
+    template <bool kPart>
     __device__ void finish(const DecodeParams& p, const Sink& k, float vscale) {
         const int lane = threadIdx.x & 31, c = lane % CPR, rh = lane / CPR;
 #pragma unroll
@@ -602,12 +655,15 @@ struct F32Consumer {
                 a.z += __shfl_xor_sync(kFull, a.z, 16); a.w += __shfl_xor_sync(kFull, a.w, 16);
             }
             if (rh == 0) {
-                sink_write<float>(p, k, D, h, 4 * c + 0, a.x, ls, vscale);
-                sink_write<float>(p, k, D, h, 4 * c + 1, a.y, ls, vscale);
-                sink_write<float>(p, k, D, h, 4 * c + 2, a.z, ls, vscale);
-                sink_write<float>(p, k, D, h, 4 * c + 3, a.w, ls, vscale);
+                sink_write<float, kPart>(p, k, D, h, 4 * c + 0, a.x, ls, vscale);
+                sink_write<float, kPart>(p, k, D, h, 4 * c + 1, a.y, ls, vscale);
+                sink_write<float, kPart>(p, k, D, h, 4 * c + 2, a.z, ls, vscale);
+                sink_write<float, kPart>(p, k, D, h, 4 * c + 3, a.w, ls, vscale);
             }
-            if (k.split && lane == 0 && h < k.nh) p.ws_ml[k.seg * p.hpu + h] = make_float2(m[h], ls);
+            if (lane == 0 && h < k.nh) {
+                if (kPart && k.part) p.part_ml[k.row0 + h] = make_float2(m[h], ls);
+                else if (k.split) p.ws_ml[k.seg * p.hpu + h] = make_float2(m[h], ls);
+            }
         }
     }
 };
@@ -648,13 +704,13 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 // Issue the async loads of the walk's current tile (and, on a unit's first
 // tile, of its q rows) into stage `stg` / q slot `qslot`.
-template <class C>
-__device__ __forceinline__ void issue_tile(const DecodeParams& p, const Walk<C::kTT>& w, TablePrefetch& tp,
+template <class C, bool kStart>
+__device__ __forceinline__ void issue_tile(const DecodeParams& p, const Walk<C::kTT, kStart>& w, TablePrefetch& tp,
                                            uint8_t* stg, uint8_t* qslot) {
     const int lane = threadIdx.x & 31;
     const int kh = w.j / p.nch, c = w.j % p.nch;
-    const int tok = w.i * C::kTT;
-    const int nblk = (w.L + p.block_size - 1) / p.block_size;
+    const int tok = w.st + w.i * C::kTT;  // absolute token of the tile's first row
+    const int nblk = (w.st + w.L + p.block_size - 1) / p.block_size;
     int phys = tp.get(p, w.s, tok / p.block_size, nblk, lane);
     if (phys < 0 || phys >= p.num_blocks) {
         if (lane == 0) raise_error(p.err, PKV_DEVERR_BLOCK_ID);
@@ -687,7 +743,9 @@ __device__ __forceinline__ void issue_tile(const DecodeParams& p, const Walk<C::
 // ----------------------------------------------------------------------------
 // The kernel: every warp is an independent worker.
 // ----------------------------------------------------------------------------
-template <class C>
+// kSuffix: the cascade suffix pass (per-sequence start tokens, partial
+// output); false compiles the plain decode path without either.
+template <class C, bool kSuffix>
 __global__ void __launch_bounds__(C::kWarps * 32, 1)
 pkv_decode_kernel(const DecodeParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -697,19 +755,19 @@ pkv_decode_kernel(const DecodeParams p) {
     uint8_t* stages = smem + warp * C::kWarpBytes;
     uint8_t* qslots = stages + C::kStages * C::kStageBytes;
 
-    const int units = p.num_kv_heads * p.nch;
-    const int cap = p.max_blocks_per_seq * p.block_size;
+    const Lens<kSuffix> ln{p.seq_lens, p.seq_start, p.num_seqs, p.num_kv_heads * p.nch,
+                           p.max_blocks_per_seq * p.block_size};
     const int64_t workers = (int64_t)gridDim.x * C::kWarps;
     const int64_t wid = (int64_t)blockIdx.x * C::kWarps + warp;
     bool bad_len = false;
-    const int64_t W = total_tiles<C::kTT>(p.seq_lens, p.num_seqs, units, cap, &bad_len);
+    const int64_t W = total_tiles<C::kTT>(ln, &bad_len);
     if (bad_len && wid == 0 && lane == 0) raise_error(p.err, PKV_DEVERR_SEQ_LEN);
     const int64_t chunk = (W + workers - 1) / workers;
     const int64_t tb = min(W, wid * chunk), te = min(W, tb + chunk);
     if (tb >= te) return;
 
-    Walk<C::kTT> iw, cw;  // issue walk (runs kStages-1 tiles ahead) and compute walk
-    iw.init(p.seq_lens, p.num_seqs, units, cap, tb, te);
+    Walk<C::kTT, kSuffix> iw, cw;  // issue walk (runs kStages-1 tiles ahead) and compute walk
+    iw.init(ln, tb, te);
     cw = iw;
     TablePrefetch tp;
 #pragma unroll 1
@@ -717,7 +775,7 @@ pkv_decode_kernel(const DecodeParams p) {
         if (!iw.done)
             issue_tile<C>(p, iw, tp, stages + k * C::kStageBytes, qslots + (iw.ord % C::kStages) * C::kQSlot);
         cp_async_commit();
-        iw.advance(p.seq_lens, p.num_seqs, units, cap);
+        iw.advance(ln);
     }
     const float kscale = (C::kPath == Path::kFp8 && p.k_scale) ? __ldg(p.k_scale) : 1.f;
     const float vscale = (C::kPath == Path::kFp8 && p.v_scale) ? __ldg(p.v_scale) : 1.f;
@@ -728,7 +786,7 @@ pkv_decode_kernel(const DecodeParams p) {
             issue_tile<C>(p, iw, tp, stages + ((n + C::kStages - 1) % C::kStages) * C::kStageBytes,
                           qslots + (iw.ord % C::kStages) * C::kQSlot);
         cp_async_commit();
-        iw.advance(p.seq_lens, p.num_seqs, units, cap);
+        iw.advance(ln);
         cp_async_wait<C::kStages - 1>();
         __syncwarp();
         const int kh = cw.j / p.nch, c = cw.j % p.nch;
@@ -742,13 +800,14 @@ pkv_decode_kernel(const DecodeParams p) {
         if (cw.last()) {
             Sink k;
             k.split = (cw.seg_i0 != 0) || (cw.i != cw.nt - 1);
+            k.part = kSuffix && !k.split && cw.st > 0;
             k.seg = wid + ((int64_t)cw.s * p.num_kv_heads + kh) * p.nch + c;
             k.row0 = (int64_t)cw.s * p.num_heads + (int64_t)kh * p.g + kHeadsPerUnit * c;
             k.nh = nh;
-            cs.finish(p, k, vscale);
+            cs.template finish<kSuffix>(p, k, vscale);
         }
         __syncwarp();  // every lane is done with this stage before it is refilled
-        cw.advance(p.seq_lens, p.num_seqs, units, cap);
+        cw.advance(ln);
     }
     cp_async_wait<0>();
 }
@@ -756,31 +815,46 @@ pkv_decode_kernel(const DecodeParams p) {
 // ----------------------------------------------------------------------------
 // Exact merge of split units (zwxr.cn 3.3: M = max m_p,
 // out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p) and zero output for
-// empty sequences.  Warp b >= 1 (global) owns the unit cut by worker
-// boundary b if that is the unit's first interior boundary; warp 0 zeroes the
-// empty sequences.  Partials are combined in worker order.
+// empty sequences.  CTA b >= 1 (hpu warps) owns the unit cut by worker
+// boundary b if that is the unit's first interior boundary, one warp per head
+// row; CTA 0 zeroes the empty sequences.  Partials are folded in worker order, four segments
+// per step (their loads in flight together, M updated once per step).
 // ----------------------------------------------------------------------------
-template <typename QT, int D, int TT>
+template <typename QT, int D, int TT, bool kSuffix>
 __global__ void __launch_bounds__(256)
 pkv_merge_kernel(const DecodeParams p, int64_t workers) {
-    const int lane = threadIdx.x & 31;
-    const int64_t b = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int units = p.num_kv_heads * p.nch;
-    const int cap = p.max_blocks_per_seq * p.block_size;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t b = blockIdx.x;
+    const Lens<kSuffix> ln{p.seq_lens, p.seq_start, p.num_seqs, p.num_kv_heads * p.nch,
+                           p.max_blocks_per_seq * p.block_size};
     if (b == 0) {
-        for (int s = 0; s < p.num_seqs; ++s) {
-            if (clamp_len(__ldg(p.seq_lens + s), cap) != 0) continue;
-            QT* out = reinterpret_cast<QT*>(p.out) + (int64_t)s * p.num_heads * D;
-            for (int i = lane; i < p.num_heads * D; i += 32) out[i] = from_f32<QT>(0.f);
+        // sequences with nothing to attend: zero output (or an empty partial
+        // (m, l) = (-inf, 0) for a cascade suffix); warps scan 32 at a time
+        for (int s0 = warp * 32; s0 < p.num_seqs; s0 += blockDim.x) {
+            const int sl = s0 + lane;
+            unsigned empty = __ballot_sync(kFull, sl < p.num_seqs && ln.eff(sl) == 0);
+            while (empty) {
+                const int s = s0 + __ffs(empty) - 1;
+                empty &= empty - 1;
+                if (kSuffix && ln.first(s) > 0) {
+                    for (int i = lane; i < p.num_heads * D; i += 32) p.part_o[(int64_t)s * p.num_heads * D + i] = 0.f;
+                    for (int h = lane; h < p.num_heads; h += 32)
+                        p.part_ml[(int64_t)s * p.num_heads + h] = make_float2(-INFINITY, 0.f);
+                    continue;
+                }
+                QT* out = reinterpret_cast<QT*>(p.out) + (int64_t)s * p.num_heads * D;
+                for (int i = lane; i < p.num_heads * D; i += 32) out[i] = from_f32<QT>(0.f);
+            }
         }
         return;
     }
     if (b >= workers) return;
-    const int64_t W = total_tiles<TT>(p.seq_lens, p.num_seqs, units, cap);
+    // every warp locates the boundary's unit itself (no block barrier)
+    const int64_t W = total_tiles<TT>(ln);
     const int64_t chunk = (W + workers - 1) / workers;
     const int64_t P = b * chunk;
     if (P >= W) return;
-    const SeqHit hit = find_seq<TT>(p.seq_lens, p.num_seqs, units, cap, P);
+    const SeqHit hit = find_seq<TT>(ln, P);
     const int nt = ntiles_of<TT>(hit.L);
     const int j = (int)((P - hit.base) / nt);
     const int off = (int)((P - hit.base) % nt);
@@ -789,27 +863,57 @@ pkv_merge_kernel(const DecodeParams p, int64_t workers) {
     const int64_t bf = T0 / chunk, bl = (T0 + nt - 1) / chunk;
     const int kh = j / p.nch, c = j % p.nch;
     const int nh = min(kHeadsPerUnit, p.g - kHeadsPerUnit * c);
+    const int h = warp;
+    if (h >= nh) return;
     const int64_t u = ((int64_t)hit.s * p.num_kv_heads + kh) * p.nch + c;
     const int64_t row0 = (int64_t)hit.s * p.num_heads + (int64_t)kh * p.g + kHeadsPerUnit * c;
     constexpr int PER = D / 32;
-    for (int h = 0; h < nh; ++h) {
-        float M = -INFINITY;
-        for (int64_t w = bf; w <= bl; ++w) M = fmaxf(M, p.ws_ml[(w + u) * p.hpu + h].x);
-        float ls = 0.f, o[PER];
+    constexpr int kBatch = 4;
+    float M = -INFINITY, ls = 0.f, o[PER];
 #pragma unroll
-        for (int e = 0; e < PER; ++e) o[e] = 0.f;
-        for (int64_t w = bf; w <= bl; ++w) {
-            const float2 ml = p.ws_ml[(w + u) * p.hpu + h];
-            const float f = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M);
-            ls += ml.y * f;
-            const float* src = p.ws_o + ((w + u) * p.hpu + h) * D;
+    for (int e = 0; e < PER; ++e) o[e] = 0.f;
+    for (int64_t w0 = bf; w0 <= bl; w0 += kBatch) {
+        float2 ml[kBatch];
+        float v[kBatch][PER];
 #pragma unroll
-            for (int e = 0; e < PER; ++e) o[e] += src[lane + 32 * e] * f;
+        for (int k = 0; k < kBatch; ++k) {
+            const int64_t w = w0 + k;
+            ml[k] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+            for (int e = 0; e < PER; ++e) v[k][e] = 0.f;
+            if (w <= bl) {
+                ml[k] = p.ws_ml[(w + u) * p.hpu + h];
+                const float* src = p.ws_o + ((w + u) * p.hpu + h) * D;
+#pragma unroll
+                for (int e = 0; e < PER; ++e) v[k][e] = src[lane + 32 * e];
+            }
         }
-        QT* out = reinterpret_cast<QT*>(p.out) + (row0 + h) * D;
+        float Mb = M;
 #pragma unroll
-        for (int e = 0; e < PER; ++e) out[lane + 32 * e] = from_f32<QT>(ls > 0.f ? o[e] / ls : 0.f);
+        for (int k = 0; k < kBatch; ++k) Mb = fmaxf(Mb, ml[k].x);
+        if (Mb == -INFINITY) continue;  // nothing attended yet
+        const float fo = M == -INFINITY ? 0.f : ex2(M - Mb);
+        ls *= fo;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[e] *= fo;
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            const float f = ml[k].x == -INFINITY ? 0.f : ex2(ml[k].x - Mb);
+            ls += ml[k].y * f;
+#pragma unroll
+            for (int e = 0; e < PER; ++e) o[e] += v[k][e] * f;
+        }
+        M = Mb;
     }
+    if (kSuffix && ln.first(hit.s) > 0) {   // cascade suffix: keep the partial
+#pragma unroll
+        for (int e = 0; e < PER; ++e) p.part_o[(row0 + h) * D + lane + 32 * e] = o[e];
+        if (lane == 0) p.part_ml[row0 + h] = make_float2(M, ls);
+        return;
+    }
+    QT* out = reinterpret_cast<QT*>(p.out) + (row0 + h) * D;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) out[lane + 32 * e] = from_f32<QT>(ls > 0.f ? o[e] / ls : 0.f);
 }
 
 }  // namespace pkv

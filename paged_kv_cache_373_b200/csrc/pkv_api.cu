@@ -94,15 +94,16 @@ extern "C" size_t pkv_paged_attention_workspace_bytes(int num_seqs, int num_head
     return w.total;
 }
 
-extern "C" pkv_status pkv_paged_attention_decode(void* out, const void* query, pkv_dtype q_dtype,
-                                                 const void* key_cache, const void* value_cache,
-                                                 pkv_dtype cache_dtype, const int32_t* block_tables,
-                                                 int max_blocks_per_seq, const int32_t* seq_lens,
-                                                 int num_seqs, int num_heads, int num_kv_heads,
-                                                 int head_dim, int block_size, int64_t num_blocks,
-                                                 float scale, const float* k_scale, const float* v_scale,
-                                                 void* workspace, size_t workspace_bytes, int num_ctas,
-                                                 pkv_stream_t stream) {
+namespace pkv {
+
+pkv_status decode_prepare(DecodeParams* pp, DecodeLauncher* launch_out, int* grid_out, void* out,
+                          const void* query, pkv_dtype q_dtype, const void* key_cache,
+                          const void* value_cache, pkv_dtype cache_dtype, const int32_t* block_tables,
+                          int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs, int num_heads,
+                          int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
+                          const float* k_scale, const float* v_scale, void* workspace,
+                          size_t workspace_bytes, int num_ctas) {
+    *launch_out = nullptr;
     if (num_seqs < 0) return fail(PKV_EINVAL, "num_seqs < 0");
     if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
         return fail(PKV_EINVAL, "num_heads must be a positive multiple of num_kv_heads");
@@ -114,7 +115,7 @@ extern "C" pkv_status pkv_paged_attention_decode(void* out, const void* query, p
     if (!std::isfinite(scale)) return fail(PKV_EINVAL, "scale must be finite");
     if (num_ctas < 0) return fail(PKV_EINVAL, "num_ctas < 0");
     // dtype combination -> launcher
-    pkv_status (*launch)(const DecodeLaunchArgs&, cudaStream_t) = nullptr;
+    DecodeLauncher launch = nullptr;
     if (cache_dtype == PKV_F32 && q_dtype == PKV_F32)
         launch = head_dim == 64 ? launch_decode_f32_d64 : launch_decode_f32_d128;
     else if (cache_dtype == PKV_F16 && q_dtype == PKV_F16)
@@ -127,7 +128,7 @@ extern "C" pkv_status pkv_paged_attention_decode(void* out, const void* query, p
                              (int)q_dtype, (int)cache_dtype, head_dim);
     if (cache_dtype == PKV_FP8_E4M3 && (!k_scale || !v_scale))
         return fail(PKV_EINVAL, "FP8 cache needs k_scale and v_scale");
-    if (num_seqs == 0) return PKV_OK;
+    if (num_seqs == 0) return PKV_OK;  // nothing to launch
     if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens || !workspace)
         return fail(PKV_EINVAL, "null pointer");
     if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
@@ -141,7 +142,7 @@ extern "C" pkv_status pkv_paged_attention_decode(void* out, const void* query, p
     int* err = device_error_word();
     if (!err) return fail(PKV_ECUDA, "device error word unavailable");
 
-    DecodeParams p;
+    DecodeParams p{};
     p.out = out;
     p.q = query;
     p.key_cache = static_cast<const uint8_t*>(key_cache);
@@ -163,7 +164,38 @@ extern "C" pkv_status pkv_paged_attention_decode(void* out, const void* query, p
     p.block_size = block_size;
     p.num_blocks = (int)num_blocks;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
-    DecodeLaunchArgs a{&p, w.grid};
+    *pp = p;
+    *launch_out = launch;
+    *grid_out = w.grid;
+    return PKV_OK;
+}
+
+size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int num_ctas) {
+    WsLayout w;
+    if (!ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, num_ctas, &w)) return 0;
+    return w.total;
+}
+
+}  // namespace pkv
+
+extern "C" pkv_status pkv_paged_attention_decode(void* out, const void* query, pkv_dtype q_dtype,
+                                                 const void* key_cache, const void* value_cache,
+                                                 pkv_dtype cache_dtype, const int32_t* block_tables,
+                                                 int max_blocks_per_seq, const int32_t* seq_lens,
+                                                 int num_seqs, int num_heads, int num_kv_heads,
+                                                 int head_dim, int block_size, int64_t num_blocks,
+                                                 float scale, const float* k_scale, const float* v_scale,
+                                                 void* workspace, size_t workspace_bytes, int num_ctas,
+                                                 pkv_stream_t stream) {
+    DecodeParams p;
+    DecodeLauncher launch;
+    int grid = 0;
+    const pkv_status st = decode_prepare(&p, &launch, &grid, out, query, q_dtype, key_cache, value_cache,
+                                         cache_dtype, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+                                         num_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                                         k_scale, v_scale, workspace, workspace_bytes, num_ctas);
+    if (st != PKV_OK || num_seqs == 0) return st;
+    DecodeLaunchArgs a{&p, grid};
     return launch(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -244,6 +276,7 @@ extern "C" const char* pkv_status_string(pkv_status s) {
     case PKV_EUNSUPPORTED: return "unsupported combination";
     case PKV_ECUDA: return "CUDA error";
     case PKV_EDEVICE: return "device-side error flag set";
+    case PKV_ENOBLOCKS: return "out of free blocks";
     default: return "unknown status";
     }
 }

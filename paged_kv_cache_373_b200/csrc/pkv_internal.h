@@ -23,8 +23,22 @@ struct DecodeParams;  // paged_attention.cuh
 
 struct DecodeLaunchArgs {
     const DecodeParams* params;
-    int grid;  // CTAs of the persistent grid
+    int grid;            // CTAs of the persistent grid
+    bool suffix = false; // cascade suffix pass (seq_start / partial output in params)
 };
+
+using DecodeLauncher = pkv_status (*)(const DecodeLaunchArgs&, cudaStream_t);
+
+// Validate the arguments of pkv_paged_attention_decode and fill the kernel
+// parameters, the variant's launcher and the grid size (pkv_api.cu).
+pkv_status decode_prepare(DecodeParams* p, DecodeLauncher* launch, int* grid, void* out,
+                          const void* query, pkv_dtype q_dtype, const void* key_cache,
+                          const void* value_cache, pkv_dtype cache_dtype, const int32_t* block_tables,
+                          int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs, int num_heads,
+                          int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
+                          const float* k_scale, const float* v_scale, void* workspace,
+                          size_t workspace_bytes, int num_ctas);
+size_t decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int num_ctas);
 
 // One launcher per kernel variant (attn_*.cu).
 pkv_status launch_decode_f32_d64(const DecodeLaunchArgs&, cudaStream_t);

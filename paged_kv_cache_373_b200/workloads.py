@@ -234,7 +234,8 @@ def config4(num_seqs: int = 32, lo: int = 16384, hi: int = 32768) -> DecodeWorkl
 
 
 def config5(num_prompts: int = 16, samples: int = 8, prefix: int = 3000,
-            tail_lo: int = 32, tail_hi: int = 512) -> DecodeWorkload:
+            tail_lo: int = 32, tail_hi: int = 512, dtype: torch.dtype = torch.bfloat16,
+            num_heads: int = 32, num_kv_heads: int = 8, head_dim: int = 128) -> DecodeWorkload:
     """Shared prompt prefix + copy-on-write of its partially filled last block.
 
     Each prompt's prefix is prefilled once and forked ``samples`` times
@@ -248,7 +249,7 @@ def config5(num_prompts: int = 16, samples: int = 8, prefix: int = 3000,
     that share the copied block take the values the copy brings.  The step
     replays: copy_blocks(cow_pairs) -> reshape_and_cache(new tokens) -> decode.
     """
-    bs, Hq, Hkv, D = 16, 32, 8, 128
+    bs, Hq, Hkv, D = 16, num_heads, num_kv_heads, head_dim
     gen = torch.Generator().manual_seed(_seed(5))
     tails = torch.randint(tail_lo, tail_hi + 1, (num_prompts, samples), generator=gen)
     pblocks = (prefix + bs - 1) // bs
@@ -282,15 +283,16 @@ def config5(num_prompts: int = 16, samples: int = 8, prefix: int = 3000,
         tables[i, :len(t)] = torch.tensor(t, dtype=torch.int32)
         lens.append(bm.seq_len(sid))
     pool_shape = (num_blocks, bs, Hkv, D)
-    kpool = _fill(pool_shape, torch.bfloat16, gen, "normal")
-    vpool = _fill(pool_shape, torch.bfloat16, gen, "normal")
-    query = _fill((S, Hq, D), torch.bfloat16, gen, "normal")
-    new_k = _fill((S, Hkv, D), torch.bfloat16, gen, "normal")
-    new_v = _fill((S, Hkv, D), torch.bfloat16, gen, "normal")
+    kpool = _fill(pool_shape, dtype, gen, "normal")
+    vpool = _fill(pool_shape, dtype, gen, "normal")
+    query = _fill((S, Hq, D), dtype, gen, "normal")
+    new_k = _fill((S, Hkv, D), dtype, gen, "normal")
+    new_v = _fill((S, Hkv, D), dtype, gen, "normal")
+    dname = {torch.bfloat16: "bf16", torch.float16: "fp16", torch.float32: "fp32"}[dtype]
     return DecodeWorkload(
-        name=f"cfg5_prefix_cow_bf16_{num_prompts}x{samples}", num_seqs=S, num_heads=Hq,
+        name=f"cfg5_prefix_cow_{dname}_{num_prompts}x{samples}", num_seqs=S, num_heads=Hq,
         num_kv_heads=Hkv, head_dim=D, block_size=bs, num_blocks=num_blocks,
-        kv_dtype=torch.bfloat16, q_dtype=torch.bfloat16, scale=1.0 / math.sqrt(D),
+        kv_dtype=dtype, q_dtype=dtype, scale=1.0 / math.sqrt(D),
         query=query, key_cache=kpool, value_cache=vpool, block_tables=tables,
         seq_lens=torch.tensor(lens, dtype=torch.int32), new_key=new_k, new_value=new_v,
         slot_mapping=torch.tensor(slots, dtype=torch.int64),
@@ -329,6 +331,18 @@ def with_all_copies(wl: DecodeWorkload) -> DecodeWorkload:
     out.name = wl.name + "_allcopy"
     out.meta = dict(wl.meta, all_copy=True)
     return out
+
+
+def cascade_groups(wl: DecodeWorkload):
+    """Sharing groups of a prefix-sharing workload (one group per prompt, its
+    samples as members, the prompt length as the requested shared prefix):
+    (group_offsets int32 [G+1], group_members int32, prefix_lens int32 [G],
+    max_group_size)."""
+    prompts, samples, prefix = wl.meta["prompts"], wl.meta["samples"], wl.meta["prefix"]
+    offsets = torch.arange(0, prompts * samples + 1, samples, dtype=torch.int32)
+    members = torch.arange(prompts * samples, dtype=torch.int32)
+    prefix_lens = torch.full((prompts,), prefix, dtype=torch.int32)
+    return offsets, members, prefix_lens, samples
 
 
 CONFIGS = {1: config1, 2: config2, 3: config3, 4: config4, 5: config5}

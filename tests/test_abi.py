@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_status_strings(L):
-    for s in range(5):
+    for s in range(6):
         assert pkv.status_string(s)
     assert pkv.status_string(99) == "unknown status"
 

@@ -1,0 +1,103 @@
+"""Cascade (shared-prefix) decode: the shared prefix blocks of a group are read
+once for all members (zwxr.cn 3.4 sharing turned into bandwidth); the result
+must equal ordinary decode attention, so it is checked against the fp64
+oracle with the same tolerances, and against the plain decode path."""
+import pytest
+import torch
+
+import paged_kv_cache_373_b200 as pkv
+from paged_kv_cache_373_b200 import workloads as W
+from pkv_testutil import compare, gpu_inputs, oracle_step
+
+pytestmark = pytest.mark.gpu
+
+
+def _cascade_step(wl, groups=None, num_ctas=0):
+    g = gpu_inputs(wl)
+    if g["pairs"].numel():
+        pkv.copy_blocks([g["kc"]], [g["vc"]], g["pairs"])
+    pkv.reshape_and_cache(g["nk"], g["nv"], g["kc"], g["vc"], g["slots"], g["ks"], g["vs"])
+    off, mem, pre, mgs = groups or W.cascade_groups(wl)
+    out = torch.empty_like(g["q"])
+    pkv.paged_attention_decode_cascade(out, g["q"], g["kc"], g["vc"], g["tables"], g["lens"],
+                                       off.cuda(), mem.cuda(), pre.cuda(), mgs, wl.scale,
+                                       g["ks"], g["vs"], num_ctas=num_ctas)
+    plain = torch.empty_like(g["q"])
+    pkv.paged_attention_decode(plain, g["q"], g["kc"], g["vc"], g["tables"], g["lens"], wl.scale,
+                               g["ks"], g["vs"], num_ctas=num_ctas)
+    return out, plain, pkv.get_device_error()
+
+
+@pytest.mark.parametrize("shape", [(2, 4, 200, 3, 40), (3, 8, 3000, 32, 512), (1, 3, 40, 1, 20)])
+def test_cascade_matches_oracle(shape):
+    prompts, samples, prefix, lo, hi = shape
+    wl = W.config5(num_prompts=prompts, samples=samples, prefix=prefix, tail_lo=lo, tail_hi=hi)
+    out, plain, err = _cascade_step(wl)
+    assert err == 0
+    ref = oracle_step(wl)
+    compare(out, ref, wl)
+    compare(plain, ref, wl)
+
+
+@pytest.mark.parametrize("dtype,heads,d", [(torch.float16, (16, 4), 64), (torch.bfloat16, (24, 2), 128),
+                                           (torch.float16, (8, 8), 128), (torch.float32, (8, 2), 64)])
+def test_cascade_dtypes_and_head_groupings(dtype, heads, d):
+    # f16 / bf16 with g = 4, 12 (two head chunks) and 1; fp32 takes the plain path
+    wl = W.config5(num_prompts=3, samples=5, prefix=333, tail_lo=1, tail_hi=70, dtype=dtype,
+                   num_heads=heads[0], num_kv_heads=heads[1], head_dim=d)
+    out, _, err = _cascade_step(wl)
+    assert err == 0
+    compare(out, oracle_step(wl), wl)
+
+
+def test_cascade_full_config5_sampled():
+    wl = W.config5()
+    out, plain, err = _cascade_step(wl)
+    assert err == 0
+    seqs = [0, 7, 8, 63, 64, 100, 127]
+    compare(out, oracle_step(wl, seqs=seqs), wl, seqs=seqs)
+    d = (out.float() - plain.float()).abs().max().item()
+    assert d < 4e-3, d
+
+
+@pytest.mark.parametrize("num_ctas", [1, 7, 148])
+def test_cascade_split_counts(num_ctas):
+    wl = W.config5(num_prompts=2, samples=5, prefix=700, tail_lo=1, tail_hi=90)
+    out, _, err = _cascade_step(wl, num_ctas=num_ctas)
+    assert err == 0
+    compare(out, oracle_step(wl), wl)
+
+
+def test_cascade_groups_that_share_less_than_declared():
+    # requested prefix longer than what the tables share, a member shorter than
+    # the request, a single-member group and an empty group: still exact
+    wl = W.config5(num_prompts=3, samples=4, prefix=100, tail_lo=1, tail_hi=60)
+    off = torch.tensor([0, 4, 5, 5, 12], dtype=torch.int32)     # groups: 4, 1, 0, 7 members
+    mem = torch.tensor([0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11], dtype=torch.int32)
+    pre = torch.tensor([4096, 96, 0, 64], dtype=torch.int32)
+    out, _, err = _cascade_step(wl, groups=(off, mem, pre, 7))
+    assert err == pkv.DEVERR_SEQ_LEN        # 4096 exceeds the members' lengths: flagged, clamped
+    compare(out, oracle_step(wl), wl)
+
+
+def test_cascade_invalid_member_and_oversize_group_are_flagged_and_unshared():
+    # a member id outside [0, num_seqs) and a group larger than max_group_size:
+    # both flagged, neither group shared, every output still exact
+    wl = W.config5(num_prompts=2, samples=4, prefix=160, tail_lo=1, tail_hi=40)
+    off = torch.tensor([0, 4, 8], dtype=torch.int32)
+    mem = torch.tensor([0, 1, 2, 999, 4, 5, 6, 7], dtype=torch.int32)
+    pre = torch.tensor([160, 160], dtype=torch.int32)
+    out, plain, err = _cascade_step(wl, groups=(off, mem, pre, 3))
+    assert err == pkv.DEVERR_SEQ_LEN
+    compare(out, oracle_step(wl), wl)
+    assert (out.float() - plain.float()).abs().max().item() < 4e-3
+
+
+def test_cascade_without_groups_is_plain_decode():
+    wl = W.build_decode("nogroups", [5, 40, 300], 8, 2, 128, 16, torch.bfloat16, torch.bfloat16, seed=61)
+    wl.meta.update(prompts=0, samples=1, prefix=0)
+    groups = (torch.zeros(1, dtype=torch.int32), torch.zeros(0, dtype=torch.int32),
+              torch.zeros(0, dtype=torch.int32), 1)
+    out, plain, err = _cascade_step(wl, groups=groups)
+    assert err == 0
+    assert torch.equal(out.view(torch.int16), plain.view(torch.int16))
