@@ -50,6 +50,10 @@ def lib():
                                                ctypes.c_float, ctypes.c_float]
         L.oracle_copy_blocks.restype = c_int
         L.oracle_copy_blocks.argtypes = [c_void, c_void, c_int, c_void, c_i64, c_i64, c_i64]
+        L.oracle_paged_prefill.restype = c_int
+        L.oracle_paged_prefill.argtypes = [c_void, c_void, c_int, c_void, c_void, c_int, c_void, c_int,
+                                           c_void, c_void, c_int, c_int, c_int, c_int, c_int, c_i64,
+                                           ctypes.c_double, ctypes.c_float, ctypes.c_float, c_int]
         L.oracle_swap_blocks.restype = c_int
         L.oracle_swap_blocks.argtypes = [c_void, c_void, c_i64, c_void, c_void, c_i64, c_int, c_void,
                                          c_i64, c_i64]
@@ -178,6 +182,27 @@ def paged_attention_decode(query, key_cache, value_cache, block_tables, seq_lens
         float(scale), float(k_scale), float(v_scale), sub_ptr, nsub, int(num_threads))
     if rc != 0:
         raise ValueError(f"oracle_paged_attention_decode failed: {rc}")
+    return out
+
+
+def paged_prefill(query, key_cache, value_cache, block_tables, seq_lens, query_start, scale,
+                  k_scale: float = 1.0, v_scale: float = 1.0, num_threads: int = 0) -> np.ndarray:
+    """Chunked-prefill attention, fp64 [T, Hq, D]: the chunk of sequence s is
+    query rows query_start[s]..query_start[s+1]-1, ending at position seq_lens[s]-1."""
+    T, Hq, D = query.shape
+    NB, bs, Hkv, D2 = key_cache.shape
+    assert D == D2
+    bt = block_tables.to(torch.int32).contiguous()
+    sl = seq_lens.to(torch.int32).contiguous()
+    qs = query_start.to(torch.int32).contiguous()
+    assert int(qs[-1]) == T
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    rc = lib().oracle_paged_prefill(
+        out.ctypes.data, _ptr(query), dtype_code(query), _ptr(key_cache), _ptr(value_cache),
+        dtype_code(key_cache), _ptr(bt), bt.shape[1], _ptr(sl), _ptr(qs), sl.shape[0], Hq, Hkv, D,
+        bs, NB, float(scale), float(k_scale), float(v_scale), int(num_threads))
+    if rc != 0:
+        raise ValueError(f"oracle_paged_prefill failed: {rc}")
     return out
 
 

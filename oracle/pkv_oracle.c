@@ -372,6 +372,69 @@ int oracle_paged_attention_decode(double* out, const void* q, int q_dtype,
 }
 
 /*
+ * Chunked prefill (ttlab.hopto.org "LLM KV cache 02", section 3, "新问题：
+ * 长 Prefill 会暂停解码": a long prompt is cut into chunks processed over
+ * several steps).  Sequence s contributes the C_s = query_start[s+1] -
+ * query_start[s] query rows of its current chunk; its cache already holds
+ * all seq_lens[s] tokens (the context and this chunk), so the chunk's i-th
+ * token sits at position p = seq_lens[s] - C_s + i and attends to the
+ * cached tokens t <= p (causal attention through the block table).
+ * out  : fp64 [T, num_heads, head_dim], T = query_start[num_seqs]
+ * q    : [T, num_heads, head_dim] in q_dtype; other arguments as decode.
+ */
+int oracle_paged_prefill(double* out, const void* q, int q_dtype,
+                         const void* key_cache, const void* value_cache, int cache_dtype,
+                         const int32_t* block_tables, int max_blocks_per_seq,
+                         const int32_t* seq_lens, const int32_t* query_start, int num_seqs,
+                         int num_heads, int num_kv_heads, int head_dim, int block_size,
+                         int64_t num_blocks, double scale, float k_scale, float v_scale,
+                         int num_threads)
+{
+    if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0) return OR_EINVAL;
+    if (dtype_bytes(q_dtype) == 0 || dtype_bytes(cache_dtype) == 0) return OR_EINVAL;
+    int g = num_heads / num_kv_heads;
+    double ks = cache_dtype == OR_FP8_E4M3 ? (double)k_scale : 1.0;
+    double vs = cache_dtype == OR_FP8_E4M3 ? (double)v_scale : 1.0;
+    int status = OR_OK;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int s = 0; s < num_seqs; ++s) {
+        int L = seq_lens[s];
+        int C = query_start[s + 1] - query_start[s];
+        if (L < 0 || C < 0 || C > L ||
+            (int64_t)(L + block_size - 1) / block_size > max_blocks_per_seq) {
+            status = OR_ERANGE;
+            continue;
+        }
+        double* K = (double*)malloc(sizeof(double) * ((size_t)L * head_dim + 1));
+        double* V = (double*)malloc(sizeof(double) * ((size_t)L * head_dim + 1));
+        double* score = (double*)malloc(sizeof(double) * ((size_t)L + 1));
+        double* qh = (double*)malloc(sizeof(double) * (size_t)head_dim);
+        for (int kvh = 0; kvh < num_kv_heads; ++kvh) {
+            if (gather_sequence(K, V, key_cache, value_cache, cache_dtype,
+                                block_tables + (int64_t)s * max_blocks_per_seq, L, block_size,
+                                num_blocks, num_kv_heads, kvh, head_dim, ks, vs) != OR_OK) {
+                status = OR_ERANGE;
+                break;
+            }
+            for (int i = 0; i < C; ++i) {
+                int64_t row = (int64_t)query_start[s] + i;
+                int pos = L - C + i;                      /* the token's position */
+                for (int h = kvh * g; h < (kvh + 1) * g; ++h) {
+                    int64_t qo = (row * num_heads + h) * head_dim;
+                    for (int d = 0; d < head_dim; ++d) qh[d] = load_elem(q, qo + d, q_dtype);
+                    attend(out + qo, qh, K, V, pos + 1, head_dim, scale, score);  /* t <= pos */
+                }
+            }
+        }
+        free(K); free(V); free(score); free(qh);
+    }
+    return status;
+}
+
+/*
  * Block-wise softmax (zwxr.cn 3.3): the L rows are cut into partitions of
  * `part` tokens; each partition keeps its own max m_p, normaliser
  * l_p = sum exp(s - m_p) and unnormalised o_p = sum exp(s - m_p) v; the
