@@ -345,6 +345,116 @@ def cascade_groups(wl: DecodeWorkload):
     return offsets, members, prefix_lens, samples
 
 
+# ----------------------------------------------------------------------------
+# Chunked prefill (ttlab.hopto.org "LLM KV cache 02", section 3: a long prompt
+# is cut into chunks that share each step's token budget with decode tokens).
+@dataclass
+class PrefillWorkload:
+    name: str
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    kv_dtype: torch.dtype
+    scale: float
+    query: torch.Tensor              # [T, Hq, D] the chunks' query rows, sequence after sequence
+    query_start: torch.Tensor        # int32 [S+1]
+    key_cache: torch.Tensor          # [NB, bs, Hkv, D] context tokens filled, chunk slots not yet
+    value_cache: torch.Tensor
+    block_tables: torch.Tensor       # int32 [S, max_blocks]
+    seq_lens: torch.Tensor           # int32 [S] context + chunk
+    new_key: torch.Tensor            # [T, Hkv, D] the chunks' K/V
+    new_value: torch.Tensor
+    slot_mapping: torch.Tensor       # int64 [T]
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def num_seqs(self) -> int:
+        return int(self.seq_lens.shape[0])
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.query.shape[0])
+
+    @property
+    def max_query_len(self) -> int:
+        qs = self.query_start
+        return int((qs[1:] - qs[:-1]).max()) if self.num_seqs else 0
+
+    def causal_pairs(self) -> int:
+        """(query token, attended token) pairs per head: sum over chunk tokens of position + 1."""
+        tot = 0
+        for s in range(self.num_seqs):
+            L = int(self.seq_lens[s])
+            C = int(self.query_start[s + 1] - self.query_start[s])
+            tot += C * (L - C) + C * (C + 1) // 2
+        return tot
+
+    def flops(self) -> int:
+        """4 flops per (pair, q head, dim): q.k and p.v, multiply + add."""
+        return 4 * self.causal_pairs() * self.num_heads * self.head_dim
+
+
+def build_prefill(name: str, ctx_lens: Sequence[int], chunk_lens: Sequence[int], num_heads: int,
+                  num_kv_heads: int, head_dim: int, block_size: int, dtype: torch.dtype, seed: int,
+                  slack: float = 0.10) -> PrefillWorkload:
+    """Sequence s has ctx_lens[s] tokens cached and a chunk of chunk_lens[s]
+    new tokens: their K/V go to the cache through slot_mapping, then the
+    chunk's query rows attend causally over all ctx + chunk tokens."""
+    gen = torch.Generator().manual_seed(seed)
+    ctx = [int(c) for c in ctx_lens]
+    ch = [int(c) for c in chunk_lens]
+    lens = [a + b for a, b in zip(ctx, ch)]
+    need = sum((L + block_size - 1) // block_size for L in lens)
+    num_blocks = max(need + int(math.ceil(need * slack)), 1)
+    bm = BlockManager(num_blocks, block_size, torch.randperm(num_blocks, generator=gen).tolist())
+    slots: List[int] = []
+    tables = []
+    for c, n in zip(ctx, ch):
+        sid = bm.add_sequence(c)
+        for _ in range(n):
+            slots.append(bm.append_slot(sid)[0])
+        tables.append(bm.block_table(sid))
+    mb = max([len(t) for t in tables] + [1])
+    bt = torch.full((len(lens), mb), -1, dtype=torch.int32)
+    for i, t in enumerate(tables):
+        bt[i, :len(t)] = torch.tensor(t, dtype=torch.int32)
+    T = sum(ch)
+    shape = (num_blocks, block_size, num_kv_heads, head_dim)
+    kc = _fill(shape, dtype, gen, "normal")
+    vc = _fill(shape, dtype, gen, "normal")
+    q = _fill((T, num_heads, head_dim), dtype, gen, "normal")
+    nk = _fill((T, num_kv_heads, head_dim), dtype, gen, "normal")
+    nv = _fill((T, num_kv_heads, head_dim), dtype, gen, "normal")
+    qs = torch.tensor([0] + list(torch.tensor(ch).cumsum(0).tolist()), dtype=torch.int32)
+    return PrefillWorkload(
+        name=name, num_heads=num_heads, num_kv_heads=num_kv_heads, head_dim=head_dim,
+        block_size=block_size, num_blocks=num_blocks, kv_dtype=dtype, scale=1.0 / math.sqrt(head_dim),
+        query=q, query_start=qs, key_cache=kc, value_cache=vc, block_tables=bt,
+        seq_lens=torch.tensor(lens, dtype=torch.int32), new_key=nk, new_value=nv,
+        slot_mapping=torch.tensor(slots, dtype=torch.int64), meta={"ctx": ctx, "chunks": ch})
+
+
+def prefill_config(budget: int = 8192) -> PrefillWorkload:
+    """A chunked-prefill step of the ttlab.hopto.org experiment (Qwen3-1.7B
+    layer shape: 16 q / 8 kv heads, D=128, bf16, bs=16): three 3,500-token
+    inputs arrive while one request decodes; the step's token budget goes to
+    the decode token first, then to the inputs' chunks in arrival order.
+      budget 8192: two whole inputs (ctx 0, 3500 tokens each), the first 1191
+                   tokens of the third, one decode row at length 4500
+      budget 2048: the first input's second chunk (ctx 2047, 1453 tokens), the
+                   second input's first 594 tokens, one decode row"""
+    if budget == 8192:
+        ctx, ch = [4499, 0, 0, 0], [1, 3500, 3500, 1191]
+    elif budget == 2048:
+        ctx, ch = [4499, 2047, 0], [1, 1453, 594]
+    else:
+        raise ValueError("budget must be 2048 or 8192")
+    return build_prefill(f"prefill_qwen3_1p7b_bf16_budget{budget}", ctx, ch, 16, 8, 128, 16,
+                         torch.bfloat16, _seed(6) + budget)
+
+
 CONFIGS = {1: config1, 2: config2, 3: config3, 4: config4, 5: config5}
 
 
