@@ -6,6 +6,8 @@ reshape_and_cache (one new token per sequence) -> paged_attention_decode.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload cfg2]
     python bench.py --impl reference ...     # the fp64 CPU oracle, bounded sample
+    python bench.py --measure swap           # swap_blocks: HBM <-> page-locked host GB/s
+    python bench.py --measure block_manager  # host block manager, decode steps/s (no GPU)
 
 Multi-GPU (torchrun): every rank runs its own batch of the same workload
 (sequences are independent; no data-path collective) -> weak scaling; the
@@ -388,6 +390,191 @@ def run_ours(args):
     return 0
 
 
+# ---------------------------------------------------------------- swap leg
+SWAP_METRIC = "swap_blocks GB/s (KV blocks between HBM and page-locked host memory)"
+
+
+def run_swap(args):
+    """Preemption by swapping on cfg5-shaped blocks (16 tokens x 8 kv heads x
+    128 x bf16 = 32 KB per K or V block): swap out `--swap-blocks` scattered
+    device blocks to a pinned host pool, then swap them back into other
+    scattered device blocks.  One step = out + in.  The peak is one
+    contiguous cudaMemcpyAsync of the same bytes each way in the same run (the
+    copy engines over the host link); the per-block copy loop is the
+    one-DMA-call-per-block pattern, timed beside it."""
+    import paged_kv_cache_373_b200 as pkv
+    from paged_kv_cache_373_b200 import _build
+    _build.build()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator().manual_seed(373)
+    nb_dev, n = 16384, args.swap_blocks
+    shape = (16, 8, 128)
+    dk = torch.randn((nb_dev,) + shape, generator=gen, dtype=torch.float32).to(torch.bfloat16).to(dev)
+    dv = torch.randn((nb_dev,) + shape, generator=gen, dtype=torch.float32).to(torch.bfloat16).to(dev)
+    hk = torch.empty((n,) + shape, dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty((n,) + shape, dtype=torch.bfloat16).pin_memory()
+    perm = torch.randperm(nb_dev, generator=gen)
+    out_map = torch.stack([perm[:n], torch.arange(n)], 1).to(dev)
+    in_map = torch.stack([torch.arange(n), perm[n:2 * n]], 1).to(dev)
+    block_bytes = hk[0].numel() * 2
+    moved = 2 * n * block_bytes                     # K and V, one direction
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, k):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(k):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / k
+
+    out_ms = timed(lambda: pkv.swap_blocks([hk], [hv], [dk], [dv], out_map), args.steps)
+    in_ms = timed(lambda: pkv.swap_blocks([dk], [dv], [hk], [hv], in_map), args.steps)
+    if pkv.get_device_error() != 0:
+        raise RuntimeError("device error in swap_blocks")
+    # peaks: one contiguous copy of the same bytes each way (K and V pools)
+    dflat = dk[:n].view(-1)
+    hflat = hk.view(-1)
+    d2h_ms = timed(lambda: (hflat.copy_(dflat, non_blocking=True), hv.view(-1).copy_(dv[:n].view(-1), non_blocking=True)), args.steps)
+    h2d_ms = timed(lambda: (dflat.copy_(hflat, non_blocking=True), dv[:n].view(-1).copy_(hv.view(-1), non_blocking=True)), args.steps)
+    # one cudaMemcpyAsync per block (torch's copy_ per block row)
+    idx_out = perm[:n].tolist()
+
+    def per_block_out():
+        for i, b in enumerate(idx_out[:256]):
+            hk[i].copy_(dk[b], non_blocking=True)
+            hv[i].copy_(dv[b], non_blocking=True)
+    pb_ms = timed(per_block_out, max(3, args.steps // 10)) * n / 256
+    # CPU baseline: the oracle's swap (memcpy per block) on host copies of the pools
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        sk, sv = [dk[perm[:n]].cpu()], [dv[perm[:n]].cpu()]
+        ok, ov = [torch.empty_like(sk[0])], [torch.empty_like(sv[0])]
+        m = torch.stack([torch.arange(n), torch.arange(n)], 1)
+        t0 = time.perf_counter()
+        reps = 0
+        while time.perf_counter() - t0 < min(args.ref_budget, 10.0) or reps == 0:
+            oracle.swap_blocks(ok, ov, sk, sv, m)
+            reps += 1
+        dt = (time.perf_counter() - t0) / reps
+        cpu = {"value": moved / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{n} blocks x K,V host-to-host memcpy per block, {reps} reps"}
+    out_gbs, in_gbs = moved / out_ms / 1e6, moved / in_ms / 1e6
+    d2h_gbs, h2d_gbs = moved / d2h_ms / 1e6, moved / h2d_ms / 1e6
+    value = 2 * moved / (out_ms + in_ms) / 1e6
+    peak = 2 * moved / (d2h_ms + h2d_ms) / 1e6
+    line = {
+        "metric": SWAP_METRIC, "value": value, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": out_ms + in_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bytes (bf16 blocks)", "data": "synthetic",
+        "config": {"workload": f"swap_{n}_blocks_of_32KB_x2", "blocks": n, "block_bytes": block_bytes,
+                   "device_pool_blocks": nb_dev, "bytes_per_direction": moved},
+        "swap_out_gbs": out_gbs, "swap_in_gbs": in_gbs,
+        "contiguous_copy_gbs": {"d2h": d2h_gbs, "h2d": h2d_gbs},
+        "per_block_memcpy_out_gbs": moved / pb_ms / 1e6,
+        "roofline": {"bound": "host link", "achieved": value, "peak": peak, "unit": "GB/s",
+                     "frac": value / peak, "peak_kind": "contiguous cudaMemcpyAsync of the same bytes, "
+                                                      "measured in this run", "traffic": None},
+        "gpu_launches": 2 * args.steps, "e2e": None, "cpu_baseline": cpu,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------- host block manager leg
+BM_METRIC = "host block manager decode-step bookkeeping, seq-steps/s"
+
+
+def run_block_manager(args):
+    """The serving-side bookkeeping of cfg5 (16 prompts x 8 samples, 3000-token
+    shared prefix, prefix caching on): admit the prompts (key chain, cache
+    hits for samples forked from them), then per decode step one batched
+    append for all 128 sequences (slot mapping + copy-on-write pairs) and the
+    batch's block tables.  Host only; the oracle is timed on the same steps."""
+    import paged_kv_cache_373_b200 as pkv
+    from paged_kv_cache_373_b200 import _build
+    _build.build()
+    prompts, samples, prefix, bs = 16, 8, 3000, 16
+    nblocks = prompts * (prefix // bs + 1) + prompts * samples * 40 + 64
+    gen = torch.Generator().manual_seed(373 + 5)
+    toks = torch.randint(0, 32000, (prompts, prefix), generator=gen).tolist()
+
+    def admit(bm):
+        sids = []
+        for p in range(prompts):
+            parent, _ = bm.add_sequence(toks[p])
+            sids += [bm.fork(parent) for _ in range(samples)]
+            bm.free_sequence(parent)
+        return sids
+
+    K = args.steps
+    new_tok = torch.randint(0, 32000, (K + args.warmup, prompts * samples), generator=gen).tolist()
+    mbps = (prefix + K + args.warmup) // bs + 2
+    bm = pkv.HostBlockManager(nblocks, bs)
+    t0 = time.perf_counter()
+    sids = admit(bm)
+    admit_s = time.perf_counter() - t0
+    for i in range(args.warmup):
+        bm.append_batch(sids, new_tok[i])
+    t0 = time.perf_counter()
+    cows = 0
+    for i in range(K):
+        slots, pairs = bm.append_batch(sids, new_tok[args.warmup + i])
+        tables, lens = bm.batch_tables(sids, mbps)
+        cows += pairs.shape[0]
+    dt = time.perf_counter() - t0
+    value = K * len(sids) / dt
+    cpu = None
+    if not args.no_cpu_baseline:
+        from oracle.block_manager import OracleBlockManager
+        ob = OracleBlockManager(nblocks, bs)
+        sids_o = admit(_OracleAdapter(ob))
+        for i in range(args.warmup):
+            for s, t in zip(sids_o, new_tok[i]):
+                ob.append_token(s, t)
+        k_o, t0 = 0, time.perf_counter()
+        while k_o < K and time.perf_counter() - t0 < min(args.ref_budget, 10.0):
+            for s, t in zip(sids_o, new_tok[args.warmup + k_o]):
+                ob.append_token(s, t)
+            _ = [ob.block_table(s) for s in sids_o]
+            k_o += 1
+        cpu = {"value": k_o * len(sids_o) / (time.perf_counter() - t0), "unit": "seq-steps/s", "cores": 1,
+               "kind": "oracle", "sample": f"{k_o} of {K} decode steps, pure-Python oracle"}
+    line = {
+        "metric": BM_METRIC, "value": value, "unit": "seq-steps/s", "n_gpus": 0, "steps": K,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * dt / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int32 ids / sha256 keys", "data": "synthetic",
+        "config": {"workload": "cfg5_serving_bookkeeping_16x8", "num_seqs": len(sids), "block_size": bs,
+                   "num_blocks": nblocks, "prefix_tokens": prefix, "prefix_cache": True},
+        "admit_ms": 1000.0 * admit_s, "stats": bm.stats(), "cow_pairs_in_timed_steps": cows,
+        "roofline": None, "gpu_launches": 0, "e2e": None, "cpu_baseline": cpu,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+class _OracleAdapter:
+    """The oracle block manager behind the native binding's method names."""
+
+    def __init__(self, ob):
+        self.ob = ob
+
+    def add_sequence(self, tokens, extras=b""):
+        return self.ob.add_sequence(tokens, extras)
+
+    def fork(self, parent):
+        return self.ob.fork(parent)
+
+    def free_sequence(self, sid):
+        self.ob.free_sequence(sid)
+
+
 def e2e_leg(pkv, wl, g, ws, args, dev):
     """decode_step_host: pinned host inputs -> H2D -> step -> D2H -> sync."""
     pin = lambda t: t.contiguous().pin_memory()
@@ -452,8 +639,15 @@ def main():
     ap.add_argument("--cascade", action="store_true",
                     help="prefix-sharing workloads: read each shared prefix once per group")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--measure", default="decode", choices=["decode", "swap", "block_manager"],
+                    help="decode (the hot path), or a widened row: swap_blocks / host block manager")
+    ap.add_argument("--swap-blocks", type=int, default=4096)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    if args.measure == "swap":
+        return run_swap(args)
+    if args.measure == "block_manager":
+        return run_block_manager(args)
     return run_reference(args) if args.impl == "reference" else run_ours(args)
 
 

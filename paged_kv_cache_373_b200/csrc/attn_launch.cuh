@@ -26,12 +26,14 @@ pkv_status launch_decode_k(const DecodeLaunchArgs& a, cudaStream_t st) {
         configured.fetch_or(bit);
     }
     const DecodeParams& p = *a.params;
-    pkv_decode_kernel<C, kSuffix><<<a.grid, C::kWarps * 32, C::kSmemBytes, st>>>(p);
+    SuffixArg<kSuffix> sx{};
+    if constexpr (kSuffix) sx = SuffixArg<true>{a.seq_start, a.part_o, a.part_ml};
+    pkv_decode_kernel<C, kSuffix><<<a.grid, C::kWarps * 32, C::kSmemBytes, st>>>(p, sx);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "decode launch: %s", cudaGetErrorString(e));
     const int64_t workers = (int64_t)a.grid * C::kWarps;
     pkv_merge_kernel<typename C::q_t, C::D, C::kTT, kSuffix>
-        <<<(unsigned)workers, 32 * p.hpu, 0, st>>>(p, workers);  // a warp per head row
+        <<<(unsigned)workers, 32 * p.hpu, 0, st>>>(p, workers, sx);  // a warp per head row
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "merge launch: %s", cudaGetErrorString(e));
     return PKV_OK;

@@ -169,10 +169,8 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
                             : launch_prefix_t<__nv_bfloat16, 128>(pp, c, L.nt, grid, cs);
     if (st != PKV_OK) return st;
 
-    p.seq_start = c.seq_start;  // suffix pass: members from their shared-prefix end
-    p.part_o = c.suf_o;
-    p.part_ml = c.suf_ml;
-    DecodeLaunchArgs sa{&p, grid, true};
+    // suffix pass: members from their shared-prefix end, partial outputs
+    DecodeLaunchArgs sa{&p, grid, true, c.seq_start, c.suf_o, c.suf_ml};
     if ((st = launch(sa, cs)) != PKV_OK) return st;
 
     if (cache_dtype == PKV_F16)

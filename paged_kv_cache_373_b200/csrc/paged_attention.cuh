@@ -60,11 +60,19 @@ struct DecodeParams {
     int hpu;               // heads per unit stride in the workspace = min(8, g)
     int max_blocks_per_seq, block_size, num_blocks;
     float scale_log2;      // scale * log2(e)
-    // Cascade suffix pass only: the first token attended per sequence, and for
-    // sequences with a non-zero start the unnormalised o and (m, l) partials
-    // that replace out.
-    const int32_t* seq_start;  // [num_seqs] or null (all from 0)
-    float* part_o;             // [num_seqs * num_heads * D] or null
+};
+// (DecodeParams is kept at 128 bytes: growing it changed the code generated
+// for the decode kernel and cost 3-4% of its bandwidth.)
+
+// Cascade suffix pass only (a second kernel argument, empty otherwise): the
+// first token attended per sequence, and for sequences with a non-zero start
+// the unnormalised o and (m, l) partials that replace out.
+template <bool kSuffix> struct SuffixArg {
+    static constexpr const int32_t* seq_start = nullptr;
+};
+template <> struct SuffixArg<true> {
+    const int32_t* seq_start;  // [num_seqs]
+    float* part_o;             // [num_seqs * num_heads * D]
     float2* part_ml;           // [num_seqs * num_heads]
 };
 
@@ -300,12 +308,16 @@ struct Sink {
 
 // kPart: the cascade suffix pass, whose whole units may be partials.
 template <typename QT, bool kPart>
-__device__ __forceinline__ void sink_write(const DecodeParams& p, const Sink& k, int D, int h, int d,
-                                           float o, float l, float vscale) {
+__device__ __forceinline__ void sink_write(const DecodeParams& p, const SuffixArg<kPart>& sx, const Sink& k,
+                                           int D, int h, int d, float o, float l, float vscale) {
     if (h >= k.nh) return;
-    if (kPart && k.part) {
-        p.part_o[(k.row0 + h) * D + d] = o * vscale;
-    } else if (!k.split) {
+    if constexpr (kPart) {
+        if (k.part) {
+            sx.part_o[(k.row0 + h) * D + d] = o * vscale;
+            return;
+        }
+    }
+    if (!k.split) {
         QT* out = reinterpret_cast<QT*>(p.out) + (k.row0 + h) * D + d;
         *out = from_f32<QT>(l > 0.f ? o * vscale / l : 0.f);
     } else {
@@ -517,7 +529,7 @@ struct MmaConsumer {
 
     // End of a unit segment: the output (whole unit) or a partial (split).
     template <bool kPart>
-    __device__ void finish(const DecodeParams& p, const Sink& k, float vscale) {
+    __device__ void finish(const DecodeParams& p, const SuffixArg<kPart>& sx, const Sink& k, float vscale) {
         using QT = typename C::q_t;
         const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
         float a0 = l0, a1 = l1;
@@ -532,14 +544,14 @@ struct MmaConsumer {
             int d0, d1;
             if constexpr (!kFp8) { d0 = 16 * mi + gid; d1 = d0 + 8; }
             else { d0 = 16 * gid + 2 * mi; d1 = d0 + 1; }
-            sink_write<QT, kPart>(p, k, D, h0, d0, acc[mi][0], a0, vscale);
-            sink_write<QT, kPart>(p, k, D, h1, d0, acc[mi][1], a1, vscale);
-            sink_write<QT, kPart>(p, k, D, h0, d1, acc[mi][2], a0, vscale);
-            sink_write<QT, kPart>(p, k, D, h1, d1, acc[mi][3], a1, vscale);
+            sink_write<QT, kPart>(p, sx, k, D, h0, d0, acc[mi][0], a0, vscale);
+            sink_write<QT, kPart>(p, sx, k, D, h1, d0, acc[mi][1], a1, vscale);
+            sink_write<QT, kPart>(p, sx, k, D, h0, d1, acc[mi][2], a0, vscale);
+            sink_write<QT, kPart>(p, sx, k, D, h1, d1, acc[mi][3], a1, vscale);
         }
         if constexpr (kPart) {
             if (gid == 0 && (k.split || k.part)) {
-                float2* ml = k.part ? p.part_ml + k.row0 : p.ws_ml + k.seg * p.hpu;
+                float2* ml = k.part ? sx.part_ml + k.row0 : p.ws_ml + k.seg * p.hpu;
                 if (h0 < k.nh) ml[h0] = make_float2(m0, a0);
                 if (h1 < k.nh) ml[h1] = make_float2(m1, a1);
             }
@@ -642,7 +654,7 @@ struct F32Consumer {
         }
     }
     template <bool kPart>
-    __device__ void finish(const DecodeParams& p, const Sink& k, float vscale) {
+    __device__ void finish(const DecodeParams& p, const SuffixArg<kPart>& sx, const Sink& k, float vscale) {
         const int lane = threadIdx.x & 31, c = lane % CPR, rh = lane / CPR;
 #pragma unroll
         for (int h = 0; h < kHeadsPerUnit; ++h) {
@@ -655,14 +667,18 @@ struct F32Consumer {
                 a.z += __shfl_xor_sync(kFull, a.z, 16); a.w += __shfl_xor_sync(kFull, a.w, 16);
             }
             if (rh == 0) {
-                sink_write<float, kPart>(p, k, D, h, 4 * c + 0, a.x, ls, vscale);
-                sink_write<float, kPart>(p, k, D, h, 4 * c + 1, a.y, ls, vscale);
-                sink_write<float, kPart>(p, k, D, h, 4 * c + 2, a.z, ls, vscale);
-                sink_write<float, kPart>(p, k, D, h, 4 * c + 3, a.w, ls, vscale);
+                sink_write<float, kPart>(p, sx, k, D, h, 4 * c + 0, a.x, ls, vscale);
+                sink_write<float, kPart>(p, sx, k, D, h, 4 * c + 1, a.y, ls, vscale);
+                sink_write<float, kPart>(p, sx, k, D, h, 4 * c + 2, a.z, ls, vscale);
+                sink_write<float, kPart>(p, sx, k, D, h, 4 * c + 3, a.w, ls, vscale);
             }
-            if (lane == 0 && h < k.nh) {
-                if (kPart && k.part) p.part_ml[k.row0 + h] = make_float2(m[h], ls);
-                else if (k.split) p.ws_ml[k.seg * p.hpu + h] = make_float2(m[h], ls);
+            if constexpr (kPart) {
+                if (lane == 0 && h < k.nh) {
+                    if (k.part) sx.part_ml[k.row0 + h] = make_float2(m[h], ls);
+                    else if (k.split) p.ws_ml[k.seg * p.hpu + h] = make_float2(m[h], ls);
+                }
+            } else if (k.split && lane == 0 && h < k.nh) {
+                p.ws_ml[k.seg * p.hpu + h] = make_float2(m[h], ls);
             }
         }
     }
@@ -747,7 +763,7 @@ __device__ __forceinline__ void issue_tile(const DecodeParams& p, const Walk<C::
 // output); false compiles the plain decode path without either.
 template <class C, bool kSuffix>
 __global__ void __launch_bounds__(C::kWarps * 32, 1)
-pkv_decode_kernel(const DecodeParams p) {
+pkv_decode_kernel(const DecodeParams p, const SuffixArg<kSuffix> sx) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -755,7 +771,7 @@ pkv_decode_kernel(const DecodeParams p) {
     uint8_t* stages = smem + warp * C::kWarpBytes;
     uint8_t* qslots = stages + C::kStages * C::kStageBytes;
 
-    const Lens<kSuffix> ln{p.seq_lens, p.seq_start, p.num_seqs, p.num_kv_heads * p.nch,
+    const Lens<kSuffix> ln{p.seq_lens, sx.seq_start, p.num_seqs, p.num_kv_heads * p.nch,
                            p.max_blocks_per_seq * p.block_size};
     const int64_t workers = (int64_t)gridDim.x * C::kWarps;
     const int64_t wid = (int64_t)blockIdx.x * C::kWarps + warp;
@@ -804,7 +820,7 @@ pkv_decode_kernel(const DecodeParams p) {
             k.seg = wid + ((int64_t)cw.s * p.num_kv_heads + kh) * p.nch + c;
             k.row0 = (int64_t)cw.s * p.num_heads + (int64_t)kh * p.g + kHeadsPerUnit * c;
             k.nh = nh;
-            cs.template finish<kSuffix>(p, k, vscale);
+            cs.template finish<kSuffix>(p, sx, k, vscale);
         }
         __syncwarp();  // every lane is done with this stage before it is refilled
         cw.advance(ln);
@@ -822,10 +838,10 @@ pkv_decode_kernel(const DecodeParams p) {
 // ----------------------------------------------------------------------------
 template <typename QT, int D, int TT, bool kSuffix>
 __global__ void __launch_bounds__(256)
-pkv_merge_kernel(const DecodeParams p, int64_t workers) {
+pkv_merge_kernel(const DecodeParams p, int64_t workers, const SuffixArg<kSuffix> sx) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t b = blockIdx.x;
-    const Lens<kSuffix> ln{p.seq_lens, p.seq_start, p.num_seqs, p.num_kv_heads * p.nch,
+    const Lens<kSuffix> ln{p.seq_lens, sx.seq_start, p.num_seqs, p.num_kv_heads * p.nch,
                            p.max_blocks_per_seq * p.block_size};
     if (b == 0) {
         // sequences with nothing to attend: zero output (or an empty partial
@@ -836,11 +852,14 @@ pkv_merge_kernel(const DecodeParams p, int64_t workers) {
             while (empty) {
                 const int s = s0 + __ffs(empty) - 1;
                 empty &= empty - 1;
-                if (kSuffix && ln.first(s) > 0) {
-                    for (int i = lane; i < p.num_heads * D; i += 32) p.part_o[(int64_t)s * p.num_heads * D + i] = 0.f;
-                    for (int h = lane; h < p.num_heads; h += 32)
-                        p.part_ml[(int64_t)s * p.num_heads + h] = make_float2(-INFINITY, 0.f);
-                    continue;
+                if constexpr (kSuffix) {
+                    if (ln.first(s) > 0) {
+                        for (int i = lane; i < p.num_heads * D; i += 32)
+                            sx.part_o[(int64_t)s * p.num_heads * D + i] = 0.f;
+                        for (int h = lane; h < p.num_heads; h += 32)
+                            sx.part_ml[(int64_t)s * p.num_heads + h] = make_float2(-INFINITY, 0.f);
+                        continue;
+                    }
                 }
                 QT* out = reinterpret_cast<QT*>(p.out) + (int64_t)s * p.num_heads * D;
                 for (int i = lane; i < p.num_heads * D; i += 32) out[i] = from_f32<QT>(0.f);
@@ -905,11 +924,13 @@ pkv_merge_kernel(const DecodeParams p, int64_t workers) {
         }
         M = Mb;
     }
-    if (kSuffix && ln.first(hit.s) > 0) {   // cascade suffix: keep the partial
+    if constexpr (kSuffix) {
+        if (ln.first(hit.s) > 0) {   // cascade suffix: keep the partial
 #pragma unroll
-        for (int e = 0; e < PER; ++e) p.part_o[(row0 + h) * D + lane + 32 * e] = o[e];
-        if (lane == 0) p.part_ml[row0 + h] = make_float2(M, ls);
-        return;
+            for (int e = 0; e < PER; ++e) sx.part_o[(row0 + h) * D + lane + 32 * e] = o[e];
+            if (lane == 0) sx.part_ml[row0 + h] = make_float2(M, ls);
+            return;
+        }
     }
     QT* out = reinterpret_cast<QT*>(p.out) + (row0 + h) * D;
 #pragma unroll
