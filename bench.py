@@ -8,6 +8,7 @@ reshape_and_cache (one new token per sequence) -> paged_attention_decode.
     python bench.py --impl reference ...     # the fp64 CPU oracle, bounded sample
     python bench.py --measure swap           # swap_blocks: HBM <-> page-locked host GB/s
     python bench.py --measure block_manager  # host block manager, decode steps/s (no GPU)
+    python bench.py --measure prefill        # chunked-prefill attention, TFLOP/s
 
 Multi-GPU (torchrun): every rank runs its own batch of the same workload
 (sequences are independent; no data-path collective) -> weak scaling; the
@@ -487,6 +488,106 @@ def run_swap(args):
     return 0
 
 
+# ---------------------------------------------------------------- prefill leg
+PREFILL_METRIC = "chunked-prefill attention TFLOP/s (causal, paged KV)"
+
+
+def run_prefill(args):
+    """One step of chunked prefill: reshape_and_cache of the chunks' K/V, then
+    paged_prefill over all chunk rows (the budget-8192 step of the
+    ttlab.hopto.org experiment by default).  FLOPs = 4 * causal pairs * Hq * D;
+    the dominant kernel is bound by the tensor cores (bf16 mma.sync), peak =
+    the measured cuBLAS bf16 burst figure."""
+    import paged_kv_cache_373_b200 as pkv
+    from paged_kv_cache_373_b200 import _build, workloads as W
+    _build.build()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    wl = W.prefill_config(args.prefill_budget)
+    kc, vc = wl.key_cache.to(dev), wl.value_cache.to(dev)
+    q, nk, nv = wl.query.to(dev), wl.new_key.to(dev), wl.new_value.to(dev)
+    slots, tables = wl.slot_mapping.to(dev), wl.block_tables.to(dev)
+    lens, qs = wl.seq_lens.to(dev), wl.query_start.to(dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    scratch = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step(e0=None, e1=None):
+        pkv.reshape_and_cache(nk, nv, kc, vc, slots)
+        if e0 is not None:
+            e0.record(stream)
+        pkv.paged_prefill(out, q, kc, vc, tables, lens, qs, wl.scale)
+        if e1 is not None:
+            e1.record(stream)
+
+    clk = ClockSampler(dev.index).start()
+    t0 = time.perf_counter()
+    warm = 0
+    while warm < args.warmup or (time.perf_counter() - t0) * 1000.0 < args.spinup_ms:
+        step()
+        warm += 1
+    torch.cuda.synchronize()
+    if pkv.get_device_error() != 0:
+        raise RuntimeError("device error in prefill warm-up")
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    wall0 = time.time()
+    for i in range(K):
+        scratch.fill_(i & 0xff)          # cold L2 for every step (outside the step events)
+        ev[i][0].record(stream)
+        step(ev[i][1], ev[i][2])
+        ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    clk.window = (wall0, time.time())
+    clk.stop()
+    if pkv.get_device_error() != 0:
+        raise RuntimeError("device error in prefill")
+    step_ms = statistics.mean(a.elapsed_time(d) for a, _, _, d in ev)
+    attn_ms = statistics.mean(b.elapsed_time(c) for _, b, c, _ in ev)
+    flops = wl.flops()
+    achieved = flops / (attn_ms / 1000.0) / 1e12
+    peak, kind = 1590.0, "fallback bf16 burst"
+    pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pp):
+        with open(pp) as f:
+            peak, kind = float(json.load(f)["bf16_tflops"]), "measured cuBLAS bf16 burst"
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        kc_h, vc_h = wl.key_cache.clone(), wl.value_cache.clone()
+        oracle.reshape_and_cache(wl.new_key, wl.new_value, kc_h, vc_h, wl.slot_mapping)
+        # the decode row and the last chunk (the oracle's bounded sample)
+        qsl = wl.query_start.tolist()
+        sub = [0, wl.num_seqs - 1]
+        rows = torch.cat([wl.query[qsl[s]:qsl[s + 1]] for s in sub])
+        qsub = torch.tensor([0] + list(torch.tensor([qsl[s + 1] - qsl[s] for s in sub]).cumsum(0).tolist()),
+                            dtype=torch.int32)
+        sw = W.build_prefill("sample", [int(wl.seq_lens[s]) - (qsl[s + 1] - qsl[s]) for s in sub],
+                             [qsl[s + 1] - qsl[s] for s in sub], wl.num_heads, wl.num_kv_heads,
+                             wl.head_dim, wl.block_size, wl.kv_dtype, 1)
+        t0 = time.perf_counter()
+        oracle.paged_prefill(rows, kc_h, vc_h, wl.block_tables[sub], wl.seq_lens[sub], qsub, wl.scale,
+                             num_threads=oracle.num_threads_available())
+        dt = time.perf_counter() - t0
+        cpu = {"value": sw.flops() / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads_available(),
+               "kind": "oracle", "sample": f"sequences {sub} of the step ({sw.num_tokens} chunk rows), fp64 C oracle"}
+    line = {
+        "metric": PREFILL_METRIC, "value": achieved, "unit": "TFLOP/s", "n_gpus": 1, "steps": K,
+        "warmup": warm, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 / fp32 accum", "data": "synthetic",
+        "config": {"workload": wl.name, "num_seqs": wl.num_seqs, "chunk_tokens": wl.num_tokens,
+                   "seq_lens": wl.seq_lens.tolist(), "num_heads": wl.num_heads,
+                   "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": wl.block_size,
+                   "flops": flops, "l2": "flushed between steps"},
+        "prefill_ms": attn_ms,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_kind": kind, "traffic": None},
+        "clocks": clk.summary(), "gpu_launches": 2 * K, "e2e": None, "cpu_baseline": cpu,
+    }
+    print(json.dumps(line))
+    return 0
+
+
 # ---------------------------------------------------------------- host block manager leg
 BM_METRIC = "host block manager decode-step bookkeeping, seq-steps/s"
 
@@ -639,15 +740,18 @@ def main():
     ap.add_argument("--cascade", action="store_true",
                     help="prefix-sharing workloads: read each shared prefix once per group")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--measure", default="decode", choices=["decode", "swap", "block_manager"],
+    ap.add_argument("--measure", default="decode", choices=["decode", "swap", "block_manager", "prefill"],
                     help="decode (the hot path), or a widened row: swap_blocks / host block manager")
     ap.add_argument("--swap-blocks", type=int, default=4096)
+    ap.add_argument("--prefill-budget", type=int, default=8192, choices=[2048, 8192])
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
     if args.measure == "swap":
         return run_swap(args)
     if args.measure == "block_manager":
         return run_block_manager(args)
+    if args.measure == "prefill":
+        return run_prefill(args)
     return run_reference(args) if args.impl == "reference" else run_ours(args)
 
 

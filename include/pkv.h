@@ -12,6 +12,12 @@
  *   pkv_reshape_and_cache      write each new token's K/V into its slot (3.1)
  *   pkv_paged_attention_decode single-token attention through the block
  *                              table with the block-wise softmax merge (3.3)
+ *   pkv_paged_attention_decode_cascade  decode with shared prompt prefixes
+ *                              read once per group (3.4)
+ *   pkv_paged_prefill          chunked-prefill (causal, multi-token) attention
+ *                              through the block table
+ * and, in pkv_block_manager.h, the host block manager that produces the
+ * tables, slots and copy-on-write pairs.
  *
  * Conventions for every call
  *   - The caller owns all memory.  Pointers named d_* or documented as
@@ -251,6 +257,36 @@ pkv_status pkv_paged_attention_decode_cascade(void* out, const void* query, pkv_
                                               const float* v_scale, void* workspace,
                                               size_t workspace_bytes, int num_ctas,
                                               pkv_stream_t stream);
+
+/*
+ * pkv_paged_prefill -- chunked-prefill attention over the paged cache
+ * (ttlab.hopto.org "LLM KV cache 02", section 3: a long prompt is cut into
+ * chunks that share each step's token budget with decode tokens).
+ *
+ * Sequence s contributes the chunk rows query[query_start[s] .. query_start[s+1])
+ * (C_s = query_start[s+1] - query_start[s] tokens; C_s = 1 is a decode row).
+ * The cache already holds all seq_lens[s] tokens of the sequence, the
+ * chunk's own K/V included (pkv_reshape_and_cache first), so chunk token i is
+ * at position p = seq_lens[s] - C_s + i and
+ *   out[query_start[s] + i, h, :] = softmax_t<=p(scale * q . K[t, h / g]) . V
+ * (causal attention through the block table; g = num_heads / num_kv_heads).
+ * query, out: [num_query_tokens, num_heads, head_dim] (device, 16-byte
+ * aligned); query_start: DEVICE int32 [num_seqs + 1], non-decreasing, with
+ * query_start[num_seqs] == num_query_tokens (host-known, sizes the grid);
+ * caches, tables, seq_lens as pkv_paged_attention_decode.
+ * Supported: f16 or bf16 caches with q and out of the same dtype,
+ * head_dim in {64, 128}, block_size in {16, 32}, g in {1, 2, 4, 8, 16}
+ * (otherwise PKV_EUNSUPPORTED).  A seq_len shorter than its chunk or longer
+ * than its table row, or a decreasing query_start, sets PKV_DEVERR_SEQ_LEN
+ * (those rows are not written); an out-of-range block id reads zeros and
+ * sets PKV_DEVERR_BLOCK_ID.  No workspace.
+ */
+pkv_status pkv_paged_prefill(void* out, const void* query, pkv_dtype q_dtype, const void* key_cache,
+                             const void* value_cache, pkv_dtype cache_dtype,
+                             const int32_t* block_tables, int max_blocks_per_seq,
+                             const int32_t* seq_lens, const int32_t* query_start, int num_seqs,
+                             int64_t num_query_tokens, int num_heads, int num_kv_heads, int head_dim,
+                             int block_size, int64_t num_blocks, float scale, pkv_stream_t stream);
 
 /* Size of the static scratch used by pkv_paged_attention_decode_noalloc. */
 #define PKV_STATIC_WORKSPACE_BYTES (16u * 1024u * 1024u)

@@ -6,7 +6,7 @@ kernels.  There is no CPU fallback; if the library is missing or the tensors
 are not on a CUDA device, the call raises.
 
 Names follow the C entry points without their ``pkv_`` prefix:
-  reshape_and_cache, copy_blocks, swap_blocks, paged_attention_decode,
+  reshape_and_cache, copy_blocks, swap_blocks, paged_attention_decode, paged_prefill,
   paged_attention_decode_noalloc, paged_attention_decode_cascade,
   paged_attention_workspace_bytes, default_num_ctas, decode_step_host,
   get_device_error, status_string
@@ -32,7 +32,7 @@ _DTYPES = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_B
 EXPORTED = ("pkv_reshape_and_cache", "pkv_copy_blocks", "pkv_swap_blocks", "pkv_paged_attention_workspace_bytes",
             "pkv_default_num_ctas", "pkv_paged_attention_decode",
             "pkv_paged_attention_decode_noalloc", "pkv_paged_attention_cascade_workspace_bytes",
-            "pkv_paged_attention_decode_cascade", "pkv_decode_step_host",
+            "pkv_paged_attention_decode_cascade", "pkv_paged_prefill", "pkv_decode_step_host",
             "pkv_get_device_error", "pkv_status_string", "pkv_last_error_message")
 
 
@@ -104,6 +104,9 @@ def lib() -> ctypes.CDLL:
                                                      vp, vp, vp, c_int, c_int, c_int, c_int, c_int,
                                                      c_int, i64, ctypes.c_float, vp, vp, vp,
                                                      ctypes.c_size_t, c_int, vp]
+    L.pkv_paged_prefill.restype = c_int
+    L.pkv_paged_prefill.argtypes = [vp, vp, c_int, vp, vp, c_int, vp, c_int, vp, vp, c_int, i64, c_int,
+                                    c_int, c_int, c_int, i64, ctypes.c_float, vp]
     L.pkv_decode_step_host.restype = c_int
     L.pkv_decode_step_host.argtypes = [ctypes.POINTER(DecodeStepArgs), vp]
     L.pkv_get_device_error.restype = c_int
@@ -168,6 +171,21 @@ def copy_blocks(key_caches: Sequence[torch.Tensor], value_caches: Sequence[torch
     block_bytes = kc[0].numel() * kc.element_size()
     _check(lib().pkv_copy_blocks(kp, vp, n, _dev(block_mapping), block_mapping.shape[0],
                                  kc.shape[0], block_bytes, _stream(stream)))
+
+
+def paged_prefill(out, query, key_cache, value_cache, block_tables, seq_lens, query_start, scale,
+                  stream=None) -> None:
+    """Chunked-prefill attention: query/out [T, Hq, D]; sequence s owns rows
+    query_start[s]..query_start[s+1]-1, the last of them at position seq_lens[s]-1."""
+    T, Hq, D = query.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    S = seq_lens.shape[0]
+    if query_start.shape[0] != S + 1:
+        raise ValueError("query_start needs num_seqs + 1 entries")
+    _check(lib().pkv_paged_prefill(
+        _dev(out), _dev(query), dtype_code(query), _dev(key_cache), _dev(value_cache),
+        dtype_code(key_cache), _dev(block_tables), block_tables.shape[1], _dev(seq_lens),
+        _dev(query_start), S, T, Hq, Hkv, D, bs, NB, float(scale), _stream(stream)))
 
 
 def _pool(t: torch.Tensor) -> int:

@@ -1,0 +1,139 @@
+"""Chunked-prefill attention on the GPU (ttlab.hopto.org "LLM KV cache 02",
+section 3) against the fp64 oracle: the chunk's K/V go to the cache with
+reshape_and_cache, then every chunk row attends causally through the block
+table.  Tolerance as for decode: 2e-3 max-abs plus half an ulp of the output
+dtype."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_373_b200 as pkv
+from paged_kv_cache_373_b200 import workloads as W
+from pkv_testutil import TOL_16, half_ulp
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_prefill(wl, kc=None, vc=None):
+    kc = wl.key_cache.cuda() if kc is None else kc
+    vc = wl.value_cache.cuda() if vc is None else vc
+    pkv.reshape_and_cache(wl.new_key.cuda(), wl.new_value.cuda(), kc, vc, wl.slot_mapping.cuda())
+    out = torch.full_like(wl.query, float("nan")).cuda()
+    pkv.paged_prefill(out, wl.query.cuda(), kc, vc, wl.block_tables.cuda(), wl.seq_lens.cuda(),
+                      wl.query_start.cuda(), wl.scale)
+    err = pkv.get_device_error()
+    return out, err, kc, vc
+
+
+def oracle_caches(wl):
+    kc, vc = wl.key_cache.clone(), wl.value_cache.clone()
+    oracle.reshape_and_cache(wl.new_key, wl.new_value, kc, vc, wl.slot_mapping)
+    return kc, vc
+
+
+def check(out, ref, dtype, rows=None):
+    g = out.float().cpu().double().numpy()
+    if rows is not None:
+        g = g[rows]
+    assert np.isfinite(g).all(), "non-finite output"
+    err = np.abs(g - ref)
+    worst = float((err - (TOL_16 + half_ulp(ref, dtype))).max())
+    assert worst <= 0.0, f"max|err| {err.max():.3e} exceeds the bound by {worst:.3e}"
+    return float(err.max())
+
+
+CASES = [
+    # name, ctx, chunks, Hq, Hkv, D, bs, dtype
+    ("g2_bf16_d128", [0, 37, 5, 0], [100, 21, 1, 64], 16, 8, 128, 16, torch.bfloat16),
+    ("g1_f16_d128_bs32", [3, 100, 0], [29, 64, 130], 4, 4, 128, 32, torch.float16),
+    ("g4_bf16_d64", [17, 0, 250], [1, 33, 70], 8, 2, 64, 16, torch.bfloat16),
+    ("g8_f16_d64", [0, 64, 1], [65, 63, 16], 16, 2, 64, 16, torch.float16),
+    ("g16_bf16_d128", [5, 0], [9, 40], 16, 1, 128, 32, torch.bfloat16),
+    ("empty_chunks", [10, 20, 0, 30], [0, 5, 0, 1], 8, 4, 128, 16, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_prefill_matches_oracle(case):
+    name, ctx, ch, hq, hkv, d, bs, dt = case
+    wl = W.build_prefill(name, ctx, ch, hq, hkv, d, bs, dt, seed=21)
+    out, err, _, _ = gpu_prefill(wl)
+    assert err == 0
+    kc, vc = oracle_caches(wl)
+    ref = oracle.paged_prefill(wl.query, kc, vc, wl.block_tables, wl.seq_lens, wl.query_start, wl.scale)
+    check(out, ref, dt)
+
+
+def oracle_rows(wl, kc, vc, rows):
+    """The oracle one row at a time: row r of sequence s is a one-token chunk at its position."""
+    qs = wl.query_start.tolist()
+    res = []
+    for r in rows:
+        s = max(i for i in range(wl.num_seqs) if qs[i] <= r)
+        pos = int(wl.seq_lens[s]) - (qs[s + 1] - qs[s]) + (r - qs[s])
+        res.append(oracle.paged_prefill(wl.query[r:r + 1], kc, vc, wl.block_tables[s:s + 1],
+                                        torch.tensor([pos + 1], dtype=torch.int32),
+                                        torch.tensor([0, 1], dtype=torch.int32), wl.scale)[0])
+    return np.stack(res)
+
+
+@pytest.mark.parametrize("budget", [2048, 8192])
+def test_prefill_full_step_sampled(budget):
+    wl = W.prefill_config(budget)
+    out, err, _, _ = gpu_prefill(wl)
+    assert err == 0
+    assert torch.isfinite(out.float()).all()
+    kc, vc = oracle_caches(wl)
+    qs = wl.query_start.tolist()
+    rows = sorted({0, 1, 2, 63, 64, 65, qs[-2], qs[-1] - 1, qs[-2] + 200, qs[1] + 3499 if budget == 8192 else 5,
+                   qs[2] + 1000, qs[-1] // 2})
+    rows = [r for r in rows if 0 <= r < wl.num_tokens]
+    check(out, oracle_rows(wl, kc, vc, rows), wl.kv_dtype, rows)
+
+
+def test_splitting_a_chunk_is_bit_identical():
+    # the same 150 tokens as one chunk, or as chunks of 70 and 80 in two calls
+    wl = W.build_prefill("whole", [40], [150], 8, 4, 128, 16, torch.bfloat16, seed=22)
+    whole, err, kc, vc = gpu_prefill(wl)
+    assert err == 0
+    q = wl.query.cuda()
+    part = torch.empty_like(q)
+    t = wl.block_tables.cuda()
+    for lo, hi in ((0, 70), (70, 150)):
+        pkv.paged_prefill(part[lo:hi], q[lo:hi].contiguous(), kc, vc, t,
+                          torch.tensor([40 + hi], dtype=torch.int32, device="cuda"),
+                          torch.tensor([0, hi - lo], dtype=torch.int32, device="cuda"), wl.scale)
+    assert pkv.get_device_error() == 0
+    assert torch.equal(whole.view(torch.int16), part.view(torch.int16))
+
+
+def test_one_token_chunks_match_decode():
+    lens = [1, 17, 300, 2049]
+    wl = W.build_prefill("decode_rows", [L - 1 for L in lens], [1] * 4, 32, 8, 128, 16, torch.bfloat16, seed=23)
+    out, err, kc, vc = gpu_prefill(wl)
+    assert err == 0
+    dec = torch.empty_like(out)
+    pkv.paged_attention_decode(dec, wl.query.cuda(), kc, vc, wl.block_tables.cuda(), wl.seq_lens.cuda(),
+                               wl.scale)
+    assert (out.float() - dec.float()).abs().max().item() < 4e-3
+
+
+def test_bad_lengths_and_block_ids_are_flagged():
+    wl = W.build_prefill("bad", [10, 20], [5, 5], 8, 4, 64, 16, torch.float16, seed=24)
+    kc, vc = wl.key_cache.cuda(), wl.value_cache.cuda()
+    q = wl.query.cuda()
+    out = torch.zeros_like(q)
+    short = torch.tensor([3, 25], dtype=torch.int32, device="cuda")          # 3 < chunk of 5
+    pkv.paged_prefill(out, q, kc, vc, wl.block_tables.cuda(), short, wl.query_start.cuda(), wl.scale)
+    assert pkv.get_device_error() == pkv.DEVERR_SEQ_LEN
+    tables = wl.block_tables.clone()
+    tables[1, 0] = wl.num_blocks + 7
+    pkv.paged_prefill(out, q, kc, vc, tables.cuda(), wl.seq_lens.cuda(), wl.query_start.cuda(), wl.scale)
+    assert pkv.get_device_error() == pkv.DEVERR_BLOCK_ID
+    with pytest.raises(pkv.PkvError):   # g = 3 is not supported
+        pkv.paged_prefill(torch.zeros(10, 6, 64, dtype=torch.float16, device="cuda"),
+                          torch.zeros(10, 6, 64, dtype=torch.float16, device="cuda"),
+                          torch.zeros(4, 16, 2, 64, dtype=torch.float16, device="cuda"),
+                          torch.zeros(4, 16, 2, 64, dtype=torch.float16, device="cuda"),
+                          wl.block_tables.cuda(), wl.seq_lens.cuda(), wl.query_start.cuda(), 0.125)
