@@ -234,7 +234,9 @@ pkv_status pkv_paged_attention_decode(void* out, const void* query, pkv_dtype q_
  * capped by group_prefix_lens[i] and by every member's length, in whole
  * blocks (a request longer than a member's length sets PKV_DEVERR_SEQ_LEN, as
  * does a group with more than max_group_size members, which is then not
- * shared).  group_offsets must be a valid non-decreasing CSR index.
+ * shared).  A shared run shorter than 32 tokens is not worth a separate pass:
+ * such a group is decoded unshared.  group_offsets must be a valid
+ * non-decreasing CSR index.
  * Sequences outside every group, groups of one member and cache dtypes other
  * than f16/bf16 take the ordinary decode path.
  * workspace: >= pkv_paged_attention_cascade_workspace_bytes(...) bytes, no

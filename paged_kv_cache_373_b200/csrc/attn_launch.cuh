@@ -14,6 +14,7 @@ namespace pkv {
 
 template <class C, bool kSuffix>
 pkv_status launch_decode_k(const DecodeLaunchArgs& a, cudaStream_t st) {
+    static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
     static std::atomic<unsigned long long> configured{0};  // bit per device (< 64)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(PKV_ECUDA, "cudaGetDevice");

@@ -52,7 +52,7 @@ bool cascade_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
 
 template <class C, int NT>
 pkv_status launch_prefix(const DecodeParams& p, const CascadeParams& c, int grid, cudaStream_t st) {
-    constexpr int kSmem = C::kWarps * C::kStages * (C::kStageBytes + 8 * NT * C::kRowBytes) + 1024;
+    constexpr int kSmem = C::kWarps * (C::kStages * C::kStageBytes + 2 * 8 * NT * C::kRowBytes) + 1024;
     static_assert(kSmem <= kMaxSmem, "prefix kernel shared memory");
     static std::atomic<unsigned long long> configured{0};
     int dev = 0;
@@ -65,25 +65,29 @@ pkv_status launch_prefix(const DecodeParams& p, const CascadeParams& c, int grid
         configured.fetch_or(bit);
     }
     pkv_prefix_kernel<C, NT><<<grid, C::kWarps * 32, kSmem, st>>>(p, c);
-    cudaError_t e = cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "prefix launch: %s", cudaGetErrorString(e));
-    const int64_t workers = (int64_t)grid * C::kWarps;
-    pkv_prefix_merge_kernel<C::D, NT><<<dim3((unsigned)workers, NT), 256, 0, st>>>(p, c, workers);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(PKV_ECUDA, "prefix merge launch: %s", cudaGetErrorString(e));
     return PKV_OK;
 }
 
+// warps per CTA of the prefix pass (2-stage K/V rings + 2 query slots): 8
+// for two row tiles; 7 for four (their query slots are twice as large).
+// Measured on cfg5: more warps beat deeper rings (6 warps x 2 stages 68.7 us,
+// 5 x 3 81.6 us).
+constexpr int prefix_warps(int nt) { return nt == 2 ? 8 : 7; }
+constexpr int kPrefixStages = 2;
+
 template <typename T, int D>
 pkv_status launch_prefix_t(const DecodeParams& p, const CascadeParams& c, int nt, int grid, cudaStream_t st) {
-    // 8 warps for two row tiles; 6 for four (their q slots are twice as large)
-    if (nt == 2) return launch_prefix<Cfg<T, T, D, Path::kMma16, 8, 2>, 2>(p, c, grid, st);
-    return launch_prefix<Cfg<T, T, D, Path::kMma16, 6, 2>, 4>(p, c, grid, st);
+    if (nt == 2) return launch_prefix<Cfg<T, T, D, Path::kMma16, prefix_warps(2), kPrefixStages>, 2>(p, c, grid, st);
+    return launch_prefix<Cfg<T, T, D, Path::kMma16, prefix_warps(4), kPrefixStages>, 4>(p, c, grid, st);
 }
 
 template <typename QT, int D>
-pkv_status launch_combine(const DecodeParams& p, const CascadeParams& c, cudaStream_t st) {
-    pkv_cascade_combine_kernel<QT, D><<<p.num_seqs, 256, 0, st>>>(p, c);
+pkv_status launch_combine(const DecodeParams& p, const CascadeParams& c, int nt, cudaStream_t st) {
+    const dim3 grid((unsigned)p.num_seqs, (unsigned)((p.num_heads + 7) / 8));  // a warp per (member, head)
+    if (nt == 2) pkv_cascade_combine_kernel<QT, D, 2><<<grid, 256, 0, st>>>(p, c);
+    else pkv_cascade_combine_kernel<QT, D, 4><<<grid, 256, 0, st>>>(p, c);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "combine launch: %s", cudaGetErrorString(e));
     return PKV_OK;
@@ -151,6 +155,9 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
     c.num_groups = num_groups;
     c.rows = L.rows;
     c.row_chunks = L.row_chunks;
+    c.pre_seg_o = reinterpret_cast<const float*>(base + L.pre_seg_o);
+    c.pre_seg_ml = reinterpret_cast<const float2*>(base + L.pre_seg_ml);
+    c.prefix_workers = (int64_t)grid * prefix_warps(L.nt);
 
     cudaError_t e = cudaMemsetAsync(c.seq_start, 0, (size_t)num_seqs * sizeof(int32_t), cs);
     if (e != cudaSuccess) return fail(PKV_ECUDA, "seq_start memset: %s", cudaGetErrorString(e));
@@ -174,7 +181,8 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
     if ((st = launch(sa, cs)) != PKV_OK) return st;
 
     if (cache_dtype == PKV_F16)
-        return head_dim == 64 ? launch_combine<__half, 64>(p, c, cs) : launch_combine<__half, 128>(p, c, cs);
-    return head_dim == 64 ? launch_combine<__nv_bfloat16, 64>(p, c, cs)
-                          : launch_combine<__nv_bfloat16, 128>(p, c, cs);
+        return head_dim == 64 ? launch_combine<__half, 64>(p, c, L.nt, cs)
+                              : launch_combine<__half, 128>(p, c, L.nt, cs);
+    return head_dim == 64 ? launch_combine<__nv_bfloat16, 64>(p, c, L.nt, cs)
+                          : launch_combine<__nv_bfloat16, 128>(p, c, L.nt, cs);
 }

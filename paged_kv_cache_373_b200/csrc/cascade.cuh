@@ -11,18 +11,25 @@
 //      the longest run of leading blocks that every member's table shares,
 //      capped by the requested prefix and by every member's length, in whole
 //      blocks; scatter it to the members as their suffix start.
-//   2. pkv_prefix_kernel (+ pkv_prefix_merge_kernel for split units):
-//      work unit = (group, kv head, chunk of 8*NT member query rows); the
-//      same warp-level cp.async streaming as the decode kernel, with NT
-//      tensor-core N tiles so one K/V tile feeds every member row.
+//   2. pkv_prefix_kernel: work unit = (group, kv head, chunk of 8*NT member
+//      query rows); the same warp-level cp.async streaming as the decode
+//      kernel, with NT tensor-core N tiles so one K/V tile feeds every member
+//      row.  Whole units write their partial rows; split units leave
+//      segments that pass 4 merges.
 //   3. pkv_decode_kernel with seq_start = the suffix starts and partial
 //      output for members (the ordinary path for everyone else).
-//   4. pkv_cascade_combine_kernel: out = merge(prefix partial, suffix partial).
+//   4. pkv_cascade_combine_kernel: out = merge(prefix partial or segments,
+//      suffix partial).
 #pragma once
 
 #include "paged_attention.cuh"
 
 namespace pkv {
+
+// Shortest prefix shared through the prefix pass, in 16-token tiles (the
+// prefix kernel's query slots rely on it; shorter prefixes are decoded as
+// part of each member's own sequence).
+constexpr int kPrefixMinTiles = 2;
 
 struct CascadeParams {
     const int32_t* grp_offsets;  // [G + 1] CSR offsets into grp_members
@@ -36,6 +43,9 @@ struct CascadeParams {
     float2* pre_ml;              // [G * Hkv * R] prefix partial (m, l), log2 domain
     float* suf_o;                // [S * Hq * D] suffix partial o of members
     float2* suf_ml;              // [S * Hq]
+    const float* pre_seg_o;      // prefix pass's split segments: [segments * R * D]
+    const float2* pre_seg_ml;    // [segments * R]
+    int64_t prefix_workers;      // warps of the prefix pass (its tile split)
     int num_groups;
     int rows;                    // R = max_group_size * g (member query rows per kv head)
     int row_chunks;              // ceil(R / (8 * NT))
@@ -84,7 +94,8 @@ pkv_cascade_setup_kernel(const DecodeParams p, const CascadeParams c) {
         }
     }
     __syncthreads();
-    const int eff = min(nblk, s_diff) * p.block_size;
+    int eff = min(nblk, s_diff) * p.block_size;
+    if (eff < kPrefixMinTiles * 16) eff = 0;  // too short to be worth a shared pass
     if (tid == 0) c.prefix_eff[g] = eff;
     for (int i = o0 + tid; i < o1; i += blockDim.x) {
         const int s = __ldg(c.grp_members + i);
@@ -243,7 +254,13 @@ pkv_prefix_kernel(const DecodeParams p, const CascadeParams c) {
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint8_t* stages = smem + warp * C::kStages * (C::kStageBytes + kQSlot);
+    // per warp: the K/V ring and two query slots used by alternate units.  A
+    // slot is refilled while the issue walk, at most kStages-1 tiles ahead,
+    // starts the unit after next; every unit but a worker's first holds at
+    // least kPrefixMinTiles = kStages-1 tiles (setup shares no shorter
+    // prefix), so the compute walk has left the slot's previous unit by then.
+    static_assert(C::kStages - 1 <= kPrefixMinTiles, "query slots need units of kStages-1 tiles");
+    uint8_t* stages = smem + warp * (C::kStages * C::kStageBytes + 2 * kQSlot);
     uint8_t* qslots = stages + C::kStages * C::kStageBytes;
 
     const Lens<false> ln{c.prefix_eff, nullptr, c.num_groups, p.num_kv_heads * c.row_chunks, 0x7fffffff};
@@ -255,18 +272,27 @@ pkv_prefix_kernel(const DecodeParams p, const CascadeParams c) {
     if (tb >= te) return;
 
     // member rows of unit j of group g: rows [R*rc, R*rc + R) of the group's
-    // members x q heads of kv head kh (row = member * g + head)
-    auto unit_rows = [&](int g, int j, int& kh, int& rc, int& nrows, int& o0) {
-        kh = j / c.row_chunks;
-        rc = j % c.row_chunks;
-        o0 = __ldg(c.grp_offsets + g);
-        const int total = (__ldg(c.grp_offsets + g + 1) - o0) * p.g;
-        nrows = max(0, min(R, total - R * rc));
+    // members x q heads of kv head kh (row = member * g + head).  Looked up
+    // once per unit: per tile, the loads would sit behind the previous
+    // tile's copies (a compiler memory barrier) and stall the issue.
+    struct UnitInfo {
+        int s = -1, j = -1, kh, rc, nrows, o0, first_member;
     };
+    auto unit_rows = [&](const Walk<16>& w, UnitInfo& u) {
+        if (u.s == w.s && u.j == w.j) return;
+        u.s = w.s;
+        u.j = w.j;
+        u.kh = w.j / c.row_chunks;
+        u.rc = w.j % c.row_chunks;
+        u.o0 = __ldg(c.grp_offsets + w.s);
+        const int total = (__ldg(c.grp_offsets + w.s + 1) - u.o0) * p.g;
+        u.nrows = max(0, min(R, total - R * u.rc));
+        u.first_member = __ldg(c.grp_members + u.o0);
+    };
+    UnitInfo iu, cu;  // issue walk's and compute walk's units
     auto issue = [&](const Walk<16>& w, TablePrefetch& tp, uint8_t* stg, uint8_t* qslot) {
-        int kh, rc, nrows, o0;
-        unit_rows(w.s, w.j, kh, rc, nrows, o0);
-        const int first_member = __ldg(c.grp_members + o0);
+        unit_rows(w, iu);
+        const int kh = iu.kh, rc = iu.rc, nrows = iu.nrows, o0 = iu.o0, first_member = iu.first_member;
         const int tok = w.i * 16;
         const int nblk = (w.L + p.block_size - 1) / p.block_size;
         int phys = tp.get(p, first_member, tok / p.block_size, nblk, lane);
@@ -306,7 +332,7 @@ pkv_prefix_kernel(const DecodeParams p, const CascadeParams c) {
     TablePrefetch tp;
 #pragma unroll 1
     for (int k = 0; k < C::kStages - 1; ++k) {
-        if (!iw.done) issue(iw, tp, stages + k * C::kStageBytes, qslots + (iw.ord % C::kStages) * kQSlot);
+        if (!iw.done) issue(iw, tp, stages + k * C::kStageBytes, qslots + (iw.ord & 1) * kQSlot);
         cp_async_commit();
         iw.advance(ln);
     }
@@ -315,15 +341,15 @@ pkv_prefix_kernel(const DecodeParams p, const CascadeParams c) {
     for (int n = 0; !cw.done; ++n) {
         if (!iw.done)
             issue(iw, tp, stages + ((n + C::kStages - 1) % C::kStages) * C::kStageBytes,
-                  qslots + (iw.ord % C::kStages) * kQSlot);
+                  qslots + (iw.ord & 1) * kQSlot);
         cp_async_commit();
         iw.advance(ln);
         cp_async_wait<C::kStages - 1>();
         __syncwarp();
-        int kh, rc, nrows, o0;
-        unit_rows(cw.s, cw.j, kh, rc, nrows, o0);
+        unit_rows(cw, cu);
+        const int kh = cu.kh, rc = cu.rc, nrows = cu.nrows;
         if (cw.first()) {
-            cs.load_q(qslots + (cw.ord % C::kStages) * kQSlot, nrows, p.scale_log2);
+            cs.load_q(qslots + (cw.ord & 1) * kQSlot, nrows, p.scale_log2);
             cs.reset();
         }
         uint8_t* kt = stages + (n % C::kStages) * C::kStageBytes;
@@ -345,116 +371,110 @@ pkv_prefix_kernel(const DecodeParams p, const CascadeParams c) {
     cp_async_wait<0>();
 }
 
-// Merge of the prefix units split between workers (into the prefix partial
-// rows).  Grid (workers, NT): CTA (b >= 1, y) owns rows 8y..8y+7 of the unit
-// cut by worker boundary b if b is the unit's first interior boundary, one
-// warp per row; CTA (0, 0) marks the rows of groups with no shared prefix as
-// empty partials.
-template <int D, int NT>
-__global__ void __launch_bounds__(256)
-pkv_prefix_merge_kernel(const DecodeParams p, const CascadeParams c, int64_t workers) {
-    constexpr int R = 8 * NT;
-    __shared__ int64_t sh[6];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t b = blockIdx.x;
-    const Lens<false> ln{c.prefix_eff, nullptr, c.num_groups, p.num_kv_heads * c.row_chunks, 0x7fffffff};
-    if (b == 0) {
-        if (blockIdx.y != 0) return;
-        for (int g = warp; g < c.num_groups; g += 8) {
-            if (__ldg(c.prefix_eff + g) != 0) continue;
-            const int64_t r0 = (int64_t)g * p.num_kv_heads * c.rows;
-            for (int i = lane; i < p.num_kv_heads * c.rows; i += 32) c.pre_ml[r0 + i] = make_float2(-INFINITY, 0.f);
-        }
-        return;
+// Sum over groups g' < g of the tiles of their units (warp-collective):
+// the index of group g's first tile in the prefix pass's tile sequence.
+__device__ inline int64_t group_tile_base(const Lens<false>& ln, int g) {
+    const int lane = threadIdx.x & 31;
+    int64_t base = 0;
+    for (int g0 = 0; g0 < g; g0 += 32) {
+        const int gi = g0 + lane;
+        int64_t t = gi < g ? (int64_t)ntiles_of<16>(ln.eff(gi)) * ln.units : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(kFull, t, o);
+        base += t;
     }
-    if (warp == 0) {
-        int64_t flag = 0, unit = 0, bf = 0, bl = 0, row0 = 0, nrows = 0;
-        const int64_t W = total_tiles<16>(ln);
-        const int64_t chunk = (W + workers - 1) / workers;
-        const int64_t P = b * chunk;
-        if (P < W) {
-            const SeqHit hit = find_seq<16>(ln, P);
-            const int nt = ntiles_of<16>(hit.L);
-            const int j = (int)((P - hit.base) / nt);
-            const int off = (int)((P - hit.base) % nt);
-            const int64_t T0 = hit.base + (int64_t)j * nt;
-            if (off != 0 && (b - 1) * chunk <= T0) {
-                const int kh = j / c.row_chunks, rc = j % c.row_chunks;
-                const int o0 = __ldg(c.grp_offsets + hit.s);
-                flag = 1;
-                unit = (int64_t)hit.s * ln.units + j;
-                bf = T0 / chunk;
-                bl = (T0 + nt - 1) / chunk;
-                row0 = ((int64_t)hit.s * p.num_kv_heads + kh) * c.rows + R * rc;
-                nrows = max(0, min(R, (__ldg(c.grp_offsets + hit.s + 1) - o0) * p.g - R * rc));
-            }
-        }
-        if (lane == 0) { sh[0] = flag; sh[1] = unit; sh[2] = bf; sh[3] = bl; sh[4] = row0; sh[5] = nrows; }
-    }
-    __syncthreads();
-    const int h = (int)blockIdx.y * 8 + warp;
-    if (!sh[0] || h >= (int)sh[5]) return;
-    const int64_t unit = sh[1], bf = sh[2], row0 = sh[4];
-    const int n = (int)(sh[3] - bf + 1);  // segments of the unit
-    // (m, l) of the segments, lane-parallel
-    float M = -INFINITY;
-    for (int i = lane; i < n; i += 32) M = fmaxf(M, p.ws_ml[(bf + i + unit) * R + h].x);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-    float ls = 0.f;
-    for (int i = lane; i < n; i += 32) {
-        const float2 ml = p.ws_ml[(bf + i + unit) * R + h];
-        ls += ml.x == -INFINITY ? 0.f : ml.y * ex2(ml.x - M);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(kFull, ls, o);
-    constexpr int PER = D / 32;
-    float o[PER];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) o[e] = 0.f;
-#pragma unroll 4
-    for (int i = 0; i < n; ++i) {
-        const float2 ml = p.ws_ml[(bf + i + unit) * R + h];
-        const float f = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);
-        const float* src = p.ws_o + ((bf + i + unit) * R + h) * D;
-#pragma unroll
-        for (int e = 0; e < PER; ++e) o[e] += src[lane + 32 * e] * f;
-    }
-#pragma unroll
-    for (int e = 0; e < PER; ++e) c.pre_o[(row0 + h) * D + lane + 32 * e] = o[e];
-    if (lane == 0) c.pre_ml[row0 + h] = make_float2(M, ls);
+    return base;
 }
 
 // Pass 4: out[s, h] = merge(prefix partial, suffix partial) for every member
-// of a group with a shared prefix (one CTA per member slot, one warp per head).
-template <typename QT, int D>
+// of a group with a shared prefix; one warp per (member, q head).  The
+// prefix partial of the member's row is the prefix kernel's whole-unit row,
+// or, for a unit split between workers, its segments merged here (folded
+// four at a time with the suffix partial last, the (m, l) rule of zwxr.cn
+// section 3.3).
+template <typename QT, int D, int NT>
 __global__ void __launch_bounds__(256)
 pkv_cascade_combine_kernel(const DecodeParams p, const CascadeParams c) {
+    constexpr int R = 8 * NT;
+    constexpr int PER = D / 32;
     const int k = blockIdx.x;  // member slot
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int h = (int)blockIdx.y * 8 + warp;
     const int total = __ldg(c.grp_offsets + c.num_groups);
     const int4 info = c.member_info[k];  // (s, g, index in group, shared)
-    if (k >= total || !info.w) return;   // no sharing: the suffix pass wrote out
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (k >= total || !info.w || h >= p.num_heads) return;  // no sharing: the suffix pass wrote out
     const int s = info.x, g = info.y, mi = info.z;
-    constexpr int PER = D / 32;
-#pragma unroll 2
-    for (int h = warp; h < p.num_heads; h += blockDim.x >> 5) {
-        const int kh = h / p.g;
-        const int64_t pr = ((int64_t)g * p.num_kv_heads + kh) * c.rows + (int64_t)mi * p.g + h % p.g;
-        const int64_t sr = (int64_t)s * p.num_heads + h;
-        const float2 a = c.pre_ml[pr], b = c.suf_ml[sr];
-        const float M = fmaxf(a.x, b.x);
-        const float fa = (a.x == -INFINITY) ? 0.f : ex2(a.x - M);
-        const float fb = (b.x == -INFINITY) ? 0.f : ex2(b.x - M);
-        const float ls = a.y * fa + b.y * fb;
-        QT* out = reinterpret_cast<QT*>(p.out) + sr * D;
+    const int kh = h / p.g;
+    const int row = mi * p.g + h % p.g;                     // member row of the group
+    const int rc = row / R, rr = row % R;
+    const Lens<false> ln{c.prefix_eff, nullptr, c.num_groups, p.num_kv_heads * c.row_chunks, 0x7fffffff};
+    const int j = kh * c.row_chunks + rc;                   // unit of the group
+    const int nt = ntiles_of<16>(ln.eff(g));
+    const int64_t W = total_tiles<16>(ln);
+    const int64_t chunk = (W + c.prefix_workers - 1) / c.prefix_workers;
+    const int64_t T0 = group_tile_base(ln, g) + (int64_t)j * nt;
+    const int64_t bf = T0 / chunk, bl = (T0 + nt - 1) / chunk;
+    const int64_t unit = (int64_t)g * ln.units + j;
+
+    float M = -INFINITY, ls = 0.f, o[PER];
 #pragma unroll
-        for (int e = 0; e < PER; ++e) {
-            const int d = lane + 32 * e;
-            const float o = c.pre_o[pr * D + d] * fa + c.suf_o[sr * D + d] * fb;
-            out[d] = from_f32<QT>(ls > 0.f ? o / ls : 0.f);
+    for (int e = 0; e < PER; ++e) o[e] = 0.f;
+    auto fold = [&](const float2 (&ml)[4], const float (&v)[4][PER]) {
+        float Mb = M;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) Mb = fmaxf(Mb, ml[q].x);
+        if (Mb == -INFINITY) return;
+        const float fo = M == -INFINITY ? 0.f : ex2(M - Mb);
+        ls *= fo;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[e] *= fo;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float f = ml[q].x == -INFINITY ? 0.f : ex2(ml[q].x - Mb);
+            ls += ml[q].y * f;
+#pragma unroll
+            for (int e = 0; e < PER; ++e) o[e] += v[q][e] * f;
         }
+        M = Mb;
+    };
+    // the prefix partial: one whole-unit row, or segments bf..bl; then the
+    // suffix partial (index n of the sequence of partials)
+    const int n = bf == bl ? 1 : (int)(bl - bf + 1);
+    for (int i0 = 0; i0 <= n; i0 += 4) {
+        float2 ml[4];
+        float v[4][PER];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int i = i0 + q;
+            ml[q] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+            for (int e = 0; e < PER; ++e) v[q][e] = 0.f;
+            const float* src = nullptr;
+            if (i < n) {
+                if (bf == bl) {
+                    const int64_t pr = ((int64_t)g * p.num_kv_heads + kh) * c.rows + row;
+                    ml[q] = c.pre_ml[pr];
+                    src = c.pre_o + pr * D;
+                } else {
+                    const int64_t sg = (bf + i + unit) * R + rr;
+                    ml[q] = c.pre_seg_ml[sg];
+                    src = c.pre_seg_o + sg * D;
+                }
+            } else if (i == n) {
+                const int64_t sr = (int64_t)s * p.num_heads + h;
+                ml[q] = c.suf_ml[sr];
+                src = c.suf_o + sr * D;
+            }
+            if (src) {
+#pragma unroll
+                for (int e = 0; e < PER; ++e) v[q][e] = src[lane + 32 * e];
+            }
+        }
+        fold(ml, v);
     }
+    QT* out = reinterpret_cast<QT*>(p.out) + ((int64_t)s * p.num_heads + h) * D;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) out[lane + 32 * e] = from_f32<QT>(ls > 0.f ? o[e] / ls : 0.f);
 }
 
 }  // namespace pkv

@@ -263,7 +263,6 @@ struct Cfg {
     static_assert(kRowBytes % 128 == 0, "rows must be whole 128-byte columns");
     static_assert(kStageBytes % 1024 == 0 && kQSlot % 1024 == 0, "1024-byte stage alignment");
     static_assert(kWarps <= kMaxWarpsPerCta, "workspace sizing");
-    static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
 template <typename T> __device__ __forceinline__ T from_f32(float x);
