@@ -25,8 +25,7 @@ step by step for reading against them:
   tail so that the tail is evicted first, and evicted least-recently-used
   when space is needed; the hash is sha256.
 
-Readings where the pages are silent (each listed with its reason in the
-design notes):
+Readings where the pages are silent:
   * key of block i = sha256(key_{i-1} || token ids as little-endian int32 ||
     extras), with key_{-1} = 32 zero bytes;
   * allocation takes a never-cached free block first (in the free-list

@@ -32,10 +32,23 @@ pkv_status launch_decode_k(const DecodeLaunchArgs& a, cudaStream_t st) {
     pkv_decode_kernel<C, kSuffix><<<a.grid, C::kWarps * 32, C::kSmemBytes, st>>>(p, sx);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "decode launch: %s", cudaGetErrorString(e));
+    // the merge kernel is a programmatic dependent launch: its CTAs start
+    // while the decode grid drains, locate their unit from the lengths (which
+    // the decode kernel does not write) and wait for the decode grid's results
+    // only before reading the workspace
     const int64_t workers = (int64_t)a.grid * C::kWarps;
-    pkv_merge_kernel<typename C::q_t, C::D, C::kTT, kSuffix>
-        <<<(unsigned)workers, 32 * p.hpu, 0, st>>>(p, workers, sx);  // a warp per head row
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)workers);
+    cfg.blockDim = dim3(32 * p.hpu);  // a warp per head row
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, pkv_merge_kernel<typename C::q_t, C::D, C::kTT, kSuffix>, p, workers, sx);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "merge launch: %s", cudaGetErrorString(e));
     return PKV_OK;
 }

@@ -763,6 +763,10 @@ __device__ __forceinline__ void issue_tile(const DecodeParams& p, const Walk<C::
 template <class C, bool kSuffix>
 __global__ void __launch_bounds__(C::kWarps * 32, 1)
 pkv_decode_kernel(const DecodeParams p, const SuffixArg<kSuffix> sx) {
+    // let the merge grid (a programmatic dependent launch) be scheduled now:
+    // its CTAs locate their units while this grid runs and wait for its
+    // completion before reading any partial result
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -883,6 +887,9 @@ pkv_merge_kernel(const DecodeParams p, int64_t workers, const SuffixArg<kSuffix>
     const int nh = min(kHeadsPerUnit, p.g - kHeadsPerUnit * c);
     const int h = warp;
     if (h >= nh) return;
+    // launched as a programmatic dependent of the decode grid: its partials
+    // are complete and visible only after this point
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t u = ((int64_t)hit.s * p.num_kv_heads + kh) * p.nch + c;
     const int64_t row0 = (int64_t)hit.s * p.num_heads + (int64_t)kh * p.g + kHeadsPerUnit * c;
     constexpr int PER = D / 32;
