@@ -354,7 +354,8 @@ def run_ours(args):
                "sample": f"first {smp.k} of {wl.num_seqs} sequences of the same workload, "
                          f"fp64 C oracle, {smp.cores} OpenMP threads"}
 
-    launches_per_step = (1 if has_pairs else 0) + 1 + (6 if args.cascade else 2)
+    # copy_blocks, reshape_and_cache, then decode + merge (cascade: setup, prefix, suffix decode + merge, combine)
+    launches_per_step = (1 if has_pairs else 0) + 1 + (5 if args.cascade else 2)
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "seq-steps/s", "n_gpus": world,
