@@ -82,7 +82,8 @@ typedef enum {
 #define PKV_DEVERR_SLOT     0x2   /* slot_mapping entry >= num_blocks * block_size */
 #define PKV_DEVERR_SEQ_LEN  0x4   /* seq_len < 0 or > max_blocks_per_seq * block_size */
 #define PKV_DEVERR_COPY_ID  0x8   /* copy_blocks src/dst outside [0, num_blocks) */
-#define PKV_DEVERR_TIMEOUT  0x10  /* reserved: no kernel of this version waits on another */
+#define PKV_DEVERR_TIMEOUT  0x10  /* a bounded wait for tensor-core results ran out (pkv_paged_prefill);
+                                     the affected rows are not written */
 
 /*
  * pkv_reshape_and_cache -- store the K/V of new tokens in their cache slots.
@@ -281,7 +282,8 @@ pkv_status pkv_paged_attention_decode_cascade(void* out, const void* query, pkv_
  * (otherwise PKV_EUNSUPPORTED).  A seq_len shorter than its chunk or longer
  * than its table row, or a decreasing query_start, sets PKV_DEVERR_SEQ_LEN
  * (those rows are not written); an out-of-range block id reads zeros and
- * sets PKV_DEVERR_BLOCK_ID.  No workspace.
+ * sets PKV_DEVERR_BLOCK_ID.  No workspace.  The products run on the
+ * tensor core with accumulators in tensor memory (256 columns per CTA).
  */
 pkv_status pkv_paged_prefill(void* out, const void* query, pkv_dtype q_dtype, const void* key_cache,
                              const void* value_cache, pkv_dtype cache_dtype,

@@ -5,16 +5,22 @@
 // of sequence s sits at position p = seq_lens[s] - C_s + i and attends to the
 // cached tokens t <= p through the block table.
 //
-// Work unit: (sequence, kv head, tile of 64 query rows); a row is a (chunk
-// token, q head of the kv head's group) pair, so one K/V tile in shared
-// memory serves all g heads of every token in the unit.  A CTA of 4 warps
-// streams the unit's K/V tiles of 64 tokens (paged gather with 16-byte
-// cp.async, zero fill past the valid range, a 3-stage ring, XOR-swizzled
-// rows) and each warp runs the online softmax for its 16 rows with
-// mma.sync m16n8k16: S = Q K^T (q rows as A, K rows as B via ldmatrix),
-// O += P V (P re-packed from the S accumulators, V via ldmatrix.trans).  For
-// bf16, P is carried as hi + lo bf16 parts so P V keeps fp32-level accuracy.
-// Tiles past a warp's last position are skipped (causal).
+// Work unit: (sequence, kv head, 128 query rows); a row is a (chunk token,
+// q head of the kv head's group) pair, so one K/V tile in shared memory serves
+// all g heads of every token in the unit.  A CTA of 4 warps (thread = row):
+//   - gathers the unit's 64-token K/V tiles through the table with 16-byte
+//     cp.async (zero fill past the unit's last position, 2-stage ring) into
+//     the 128-byte-swizzled layout the tensor core reads;
+//   - one thread issues S = Q K^T on the 5th-generation tensor core
+//     (tcgen05.mma, M = 128 rows, N = 64 tokens, accumulator in tensor
+//     memory), every thread loads its row of S from tensor memory and runs
+//     the online softmax in registers;
+//   - P is written to shared memory (bf16: hi + lo parts, so P V keeps
+//     fp32-level accuracy) and O_t = P V_t is issued (N = head_dim, V read
+//     MN-major); each thread folds its row of O_t into its running output.
+// Completion of each group of tensor-core products is signalled on an
+// mbarrier (tcgen05.commit); every wait is bounded and a timeout sets
+// PKV_DEVERR_TIMEOUT.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -27,10 +33,10 @@
 namespace pkv {
 namespace {
 
-constexpr int kPfWarps = 4;
-constexpr int kPfRows = 16 * kPfWarps;  // query rows per unit
-constexpr int kPfTok = 64;              // KV tokens per tile
-constexpr int kPfStages = 3;            // K/V ring depth
+constexpr int kPfRows = 128;   // query rows per unit (tensor-core M)
+constexpr int kPfTok = 64;     // KV tokens per tile (N of S, K of P V)
+constexpr int kPfStages = 2;   // K/V ring depth
+constexpr int kPfThreads = 128;
 
 struct PrefillParams {
     void* out;
@@ -46,13 +52,74 @@ struct PrefillParams {
     float scale_log2;
 };
 
-// byte offset of 16-byte chunk c of row r in a [rows][D] 16-bit tile; the
-// chunk index is XOR-swizzled with the row inside each 128-byte group so the
-// eight row addresses of an ldmatrix hit eight different bank groups
-template <int D>
-__device__ __forceinline__ uint32_t pf_off(int r, int c) {
-    return (uint32_t)(r * (D * 2) + (((c & ~7) | ((c ^ r) & 7)) << 4));
+// Byte offset of 16-byte chunk c of row r in a [rows][cols] 16-bit tile kept
+// as column blocks of 64 elements: block c / 8 holds rows x 128 bytes, and
+// inside it 8-row groups of 1024 bytes with the 128-byte XOR swizzle.  This
+// is the canonical swizzled layout of the tensor core's shared-memory
+// operands (K-major rows for Q, K and P; MN-major for V).
+__device__ __forceinline__ uint32_t tc_off(int r, int c, int rows) {
+    return (uint32_t)((c >> 3) * rows * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
+
+// Shared-memory matrix descriptor: start address, leading / stride byte
+// offsets (16-byte units), descriptor version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr & 0x3FFFF) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor of kind::f16 with an fp32 accumulator.
+template <bool kBf16>
+__device__ __forceinline__ uint32_t tc_idesc(int M, int N, int b_mn_major) {
+    const uint32_t fmt = kBf16 ? 1u : 0u;
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    const uint32_t z = 0;
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}\n"
+                 ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(z));
+}
+__device__ __forceinline__ void tc_commit(uint32_t mbar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+                 : "memory");
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Wait for the mbarrier phase `parity`; false after 0.2 s of wall-clock time.
+__device__ __forceinline__ bool tc_wait(uint32_t mbar, uint32_t parity) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        uint32_t ok;
+        asm volatile("{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+                     "selp.b32 %0, 1, 0, P1;\n\t}\n"
+                     : "=r"(ok) : "r"(mbar), "r"(parity) : "memory");
+        if (ok) return true;
+        if ((it & 63) == 63) {
+            const uint64_t now = global_ns();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > 200000000ull) return false;
+        }
+    }
+}
+// 16 consecutive fp32 columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float* v) {
+    uint32_t r[16];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
 // 16-byte async copy; src_bytes = 0 writes zeros (no global read)
 __device__ __forceinline__ void cp16_zfill(uint32_t dst, const void* src, int src_bytes) {
@@ -63,30 +130,34 @@ __device__ __forceinline__ void pf_commit() { asm volatile("cp.async.commit_grou
 template <int N>
 __device__ __forceinline__ void pf_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// bf16 pair of (a, b) - hi, where hi is their bf16 rounding
-__device__ __forceinline__ uint32_t lo_part(float a, float b, uint32_t hi) {
-    const float2 h = unpack2<true>(hi);
-    return pack2<true>(a - h.x, b - h.y);
-}
+template <typename T, int D>
+struct PfSmem {
+    static constexpr int kQ = kPfRows * D * 2;
+    static constexpr int kTile = kPfTok * D * 2;   // one K or V tile
+    static constexpr int kP = kPfRows * kPfTok * 2;
+    static constexpr int kParts = std::is_same<T, __nv_bfloat16>::value ? 2 : 1;  // P hi (+ lo)
+    static constexpr int kBytes = kQ + 2 * kPfStages * kTile + kParts * kP + 1024;  // + alignment
+    static constexpr int kTmemCols = 256;            // S (64 columns) + O_t (D columns)
+};
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kPfWarps * 32, 2)
+__global__ void __launch_bounds__(kPfThreads, 1)
 pkv_prefill_kernel(const PrefillParams p) {
+    using SM = PfSmem<T, D>;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-    constexpr int CH = D / 8;            // 16-byte chunks per row
-    constexpr int KS = D / 16;           // k-steps of q.k
-    constexpr int NT = kPfTok / 8;       // n-tiles of S
-    constexpr int DT = D / 8;            // n-tiles of O
-    constexpr int TILE = kPfTok * D * 2; // bytes of one K or V tile
-    extern __shared__ __align__(128) uint8_t pf_smem[];
-    uint8_t* qsm = pf_smem;                       // kPfRows x D
-    uint8_t* ksm = pf_smem + kPfRows * D * 2;     // kPfStages stages
-    uint8_t* vsm = ksm + kPfStages * TILE;        // kPfStages stages
+    constexpr int CH = D / 8;  // 16-byte chunks per row
+    extern __shared__ uint8_t pf_raw[];
+    uint8_t* sm = pf_raw + ((1024 - (smem_u32(pf_raw) & 1023)) & 1023);  // 1024-byte aligned operands
+    uint8_t* qsm = sm;
+    uint8_t* ksm = qsm + SM::kQ;
+    uint8_t* vsm = ksm + kPfStages * SM::kTile;
+    uint8_t* psm = vsm + kPfStages * SM::kTile;  // P hi, then P lo (bf16)
+    __shared__ __align__(8) uint64_t bars[2];     // S done, O_t done
+    __shared__ uint32_t tmem_base;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int gid = lane >> 2, tig = lane & 3;
 
-    // ---- the unit: kv head from the block index, then the row tile u among
-    // all sequences' row tiles (warp-parallel scan; every warp finds it)
+    // ---- the unit: kv head from the block index, then row tile u among all
+    // sequences' row tiles (warp-parallel scan; every warp finds it)
     const int kh = (int)(blockIdx.x % p.num_kv_heads);
     const int64_t u = blockIdx.x / p.num_kv_heads;
     int s = -1, j = 0;
@@ -119,7 +190,6 @@ pkv_prefill_kernel(const PrefillParams p) {
         }
     }
     if (s < 0) return;  // past the last unit
-
     const int q0 = __ldg(p.qstart + s);
     const int C = __ldg(p.qstart + s + 1) - q0;
     const int L = __ldg(p.seq_lens + s);
@@ -135,8 +205,20 @@ pkv_prefill_kernel(const PrefillParams p) {
     const int nkv = (kv_end + kPfTok - 1) / kPfTok;
     const int32_t* trow = p.tables + (int64_t)s * p.mbps;
 
+    // ---- tensor memory and barriers
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base)),
+                     "r"(SM::kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+    }
+    if (tid == 0) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[i])));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+
     // ---- q rows (zero past the chunk), with the first K/V tile
-    for (int i = tid; i < kPfRows * CH; i += kPfWarps * 32) {
+    for (int i = tid; i < kPfRows * CH; i += kPfThreads) {
         const int r = i / CH, c = i % CH;
         const int tl = r / p.g;
         const uint8_t* src = static_cast<const uint8_t*>(p.q);
@@ -145,33 +227,34 @@ pkv_prefill_kernel(const PrefillParams p) {
             src += ((int64_t)(q0 + tok0 + tl) * p.num_heads + (int64_t)kh * p.g + r % p.g) * (D * 2) + c * 16;
             nb = 16;
         }
-        cp16_zfill(smem_u32(qsm + pf_off<D>(r, c)), src, nb);
+        cp16_zfill(smem_u32(qsm + tc_off(r, c, kPfRows)), src, nb);
     }
-    // each thread copies chunk cc of rows rr, rr + RSTEP, ... of a K/V tile.
-    // The tile's (at most 4) physical blocks are read from the table one tile
-    // ahead of their copies: the copies' asm is a compiler memory barrier,
-    // so table reads interleaved with them would each stall in turn.
-    constexpr int RSTEP = kPfWarps * 32 / CH;
+    // each thread copies chunk cc of rows rr, rr + RSTEP, ... of a K/V tile;
+    // the tile's physical blocks are read from the table one tile ahead of
+    // their copies (the copies' asm is a compiler memory barrier)
+    constexpr int RSTEP = kPfThreads / CH;
     constexpr int NIT = kPfTok / RSTEP;
-    constexpr int NBLK = kPfTok / 16;         // blocks per tile at block_size 16
+    constexpr int NBLK = kPfTok / 16;
     const int rr = tid / CH, cc = tid % CH;
     const int lg_bs = p.bs == 16 ? 4 : 5;
     auto load_phys = [&](int kt, int (&ph)[NBLK]) {
 #pragma unroll
-        for (int j = 0; j < NBLK; ++j) {
-            const int t = kt * kPfTok + (j << lg_bs);
-            ph[j] = (t < kv_end && (j << lg_bs) < kPfTok) ? __ldg(trow + (t >> lg_bs)) : -1;
+        for (int jb = 0; jb < NBLK; ++jb) {
+            const int t = kt * kPfTok + (jb << lg_bs);
+            ph[jb] = (t < kv_end && (jb << lg_bs) < kPfTok) ? __ldg(trow + (t >> lg_bs)) : -1;
         }
     };
     auto issue_kv = [&](int kt, int stage, const int (&ph)[NBLK]) {
-        uint8_t* kd = ksm + stage * TILE;
-        uint8_t* vd = vsm + stage * TILE;
+        uint8_t* kd = ksm + stage * SM::kTile;
+        uint8_t* vd = vsm + stage * SM::kTile;
 #pragma unroll
         for (int i = 0; i < NIT; ++i) {
             const int r = rr + RSTEP * i;
             const int t = kt * kPfTok + r;
-            const int j = r >> lg_bs;
-            const int phys = j == 0 ? ph[0] : j == 1 ? ph[1] : j == 2 ? ph[2] : ph[3];
+            const int jb = r >> lg_bs;
+            int phys = ph[0];
+#pragma unroll
+            for (int q = 1; q < NBLK; ++q) phys = jb == q ? ph[q] : phys;
             const uint8_t* ks = p.kc;
             const uint8_t* vs = p.vc;
             int nb = 0;
@@ -186,174 +269,152 @@ pkv_prefill_kernel(const PrefillParams p) {
                     raise_error(p.err, PKV_DEVERR_BLOCK_ID);
                 }
             }
-            const uint32_t so = pf_off<D>(r, cc);
+            const uint32_t so = tc_off(r, cc, kPfTok);
             cp16_zfill(smem_u32(kd + so), ks, nb);
             cp16_zfill(smem_u32(vd + so), vs, nb);
         }
     };
-    // async groups: {q, tile 0}, {tile 1}, then one group per iteration
-    // (possibly empty), so "all but the newest group done" means tile kt landed
     int phn[NBLK];
     load_phys(0, phn);
     issue_kv(0, 0, phn);
     pf_commit();
-    if (nkv > 1) {
-        load_phys(1, phn);
-        issue_kv(1, 1, phn);
-    }
-    pf_commit();
-    if (nkv > 2) load_phys(2, phn);
+    if (nkv > 1) load_phys(1, phn);
 
-    // ---- this thread's two rows (gid, gid + 8 of the warp's 16)
-    const int r0 = warp * 16 + gid, r1 = r0 + 8;
-    const int pos0 = (r0 / p.g < ntok) ? ctx + tok0 + r0 / p.g : -1;
-    const int pos1 = (r1 / p.g < ntok) ? ctx + tok0 + r1 / p.g : -1;
-    const int wlast = min(ntok - 1, (warp * 16 + 15) / p.g);
-    const int wmax = ((warp * 16) / p.g < ntok) ? ctx + tok0 + wlast : -1;  // last position of the warp
-
-    uint32_t qa[KS][4];
-    float o[DT][4];
+    // ---- this thread's row
+    const int row = tid;
+    const int pos = (row / p.g < ntok) ? ctx + tok0 + row / p.g : -1;
+    float o[D];
 #pragma unroll
-    for (int d = 0; d < DT; ++d) o[d][0] = o[d][1] = o[d][2] = o[d][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    for (int d = 0; d < D; ++d) o[d] = 0.f;
+    float m = -INFINITY, l = 0.f;
+
+    __syncthreads();  // barriers initialised, tensor memory allocated
+    tc_after_sync();
+    const uint32_t tmem = tmem_base;
+    const uint32_t tS = tmem, tO = tmem + kPfTok;                  // columns
+    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;        // this warp's 32 lanes
+    const uint32_t id_s = tc_idesc<kBf16>(kPfRows, kPfTok, 0);
+    const uint32_t id_o = tc_idesc<kBf16>(kPfRows, D, 1);
+    bool timed_out = false;
 
 #pragma unroll 1
     for (int kt = 0; kt < nkv; ++kt) {
-        pf_wait<1>();
-        __syncthreads();  // tile kt visible to all warps; all are done with tile kt - 1
-        if (kt + 2 < nkv) issue_kv(kt + 2, (kt + 2) % kPfStages, phn);  // refills tile kt - 1's stage
-        pf_commit();
-        if (kt + 3 < nkv) load_phys(kt + 3, phn);  // in flight during this tile's math
-        if (kt == 0) {
+        pf_wait<0>();
+        fence_async_smem();  // the copies, visible to the tensor core
+        __syncthreads();     // tile kt (and q) complete; every thread done with tile kt - 1
+        tc_after_sync();
+        const int st = kt % kPfStages;
+        if (tid == 0) {  // S = Q K^T
+            const uint32_t qa = smem_u32(qsm), kb = smem_u32(ksm + st * SM::kTile);
 #pragma unroll
-            for (int kk = 0; kk < KS; ++kk)
-                ldsm_x4(qa[kk], smem_u32(qsm + pf_off<D>(warp * 16 + (lane & 15), 2 * kk + (lane >> 4))));
+            for (int kk = 0; kk < D / 16; ++kk)
+                tc_mma(tS, tc_desc(qa + (kk >> 2) * kPfRows * 128 + (kk & 3) * 32, 16, 1024),
+                       tc_desc(kb + (kk >> 2) * kPfTok * 128 + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
+            tc_commit(smem_u32(&bars[0]));
         }
+        if (kt + 1 < nkv) {  // the next tile into the other stage (its last reader, tile kt - 1, is done)
+            issue_kv(kt + 1, (kt + 1) % kPfStages, phn);
+            if (kt + 2 < nkv) load_phys(kt + 2, phn);
+        }
+        pf_commit();
+        timed_out |= !tc_wait(smem_u32(&bars[0]), kt & 1);
+        tc_after_sync();
+        // ---- this row's scores: scale (log2 domain), causal mask, online softmax
+        float sc[kPfTok];
+#pragma unroll
+        for (int c0 = 0; c0 < kPfTok; c0 += 16) tc_ld16(tS + lane_addr + c0, sc + c0);
         const int t0 = kt * kPfTok;
-        if (t0 <= wmax) {
-            const uint8_t* kt_s = ksm + (kt % kPfStages) * TILE;
-            const uint8_t* vt_s = vsm + (kt % kPfStages) * TILE;
-            float sc[NT][4];
+        float mx = -INFINITY;
 #pragma unroll
-            for (int n = 0; n < NT; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
-            // k-steps outer: the NT accumulators are independent chains
+        for (int c = 0; c < kPfTok; ++c) {
+            sc[c] = t0 + c <= pos ? sc[c] * p.scale_log2 : -INFINITY;
+            mx = fmaxf(mx, sc[c]);
+        }
+        const float mn = fmaxf(m, mx);
+        const float ref = mn == -INFINITY ? 0.f : mn;  // a row with nothing attended yet
+        const float alpha = ex2(m - ref);
+        m = mn;
+        float ls = 0.f;
 #pragma unroll
-            for (int kk = 0; kk < KS; ++kk) {
+        for (int c = 0; c < kPfTok; ++c) {
+            sc[c] = ex2(sc[c] - ref);
+            ls += sc[c];
+        }
+        l = l * alpha + ls;
+        // ---- P to shared memory (K-major rows; bf16 as hi + lo parts)
 #pragma unroll
-                for (int np = 0; np < NT / 2; ++np) {
-                    uint32_t b[4];
-                    const int tr = np * 16 + (lane & 7) + ((lane >> 4) << 3);
-                    ldsm_x4(b, smem_u32(kt_s + pf_off<D>(tr, 2 * kk + ((lane >> 3) & 1))));
-                    mma16816<kBf16>(sc[2 * np], qa[kk], b[0], b[1]);
-                    mma16816<kBf16>(sc[2 * np + 1], qa[kk], b[2], b[3]);
-                }
-            }
-            // scale (log2 domain), causal mask, row maxima
-            float mx0 = -INFINITY, mx1 = -INFINITY;
+        for (int c8 = 0; c8 < kPfTok / 8; ++c8) {
+            uint32_t h[4], lo[4];
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                const int t = t0 + n * 8 + 2 * tig;
-                sc[n][0] = t <= pos0 ? sc[n][0] * p.scale_log2 : -INFINITY;
-                sc[n][1] = t + 1 <= pos0 ? sc[n][1] * p.scale_log2 : -INFINITY;
-                sc[n][2] = t <= pos1 ? sc[n][2] * p.scale_log2 : -INFINITY;
-                sc[n][3] = t + 1 <= pos1 ? sc[n][3] * p.scale_log2 : -INFINITY;
-                mx0 = fmaxf(mx0, fmaxf(sc[n][0], sc[n][1]));
-                mx1 = fmaxf(mx1, fmaxf(sc[n][2], sc[n][3]));
-            }
-#pragma unroll
-            for (int off = 1; off < 4; off <<= 1) {
-                mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
-            }
-            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-            const float ref0 = mn0 == -INFINITY ? 0.f : mn0;  // rows with nothing attended yet
-            const float ref1 = mn1 == -INFINITY ? 0.f : mn1;
-            const float a0 = ex2(m0 - ref0), a1 = ex2(m1 - ref1);
-            m0 = mn0;
-            m1 = mn1;
-            float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                sc[n][0] = ex2(sc[n][0] - ref0);
-                sc[n][1] = ex2(sc[n][1] - ref0);
-                sc[n][2] = ex2(sc[n][2] - ref1);
-                sc[n][3] = ex2(sc[n][3] - ref1);
-                ls0 += sc[n][0] + sc[n][1];
-                ls1 += sc[n][2] + sc[n][3];
-            }
-            l0 = l0 * a0 + ls0;
-            l1 = l1 * a1 + ls1;
-#pragma unroll
-            for (int d = 0; d < DT; ++d) {
-                o[d][0] *= a0; o[d][1] *= a0;
-                o[d][2] *= a1; o[d][3] *= a1;
-            }
-            // O += P V, 16 tokens per k-step
-#pragma unroll
-            for (int kk = 0; kk < NT / 2; ++kk) {
-                uint32_t pa[4], pl[4];
-                pa[0] = pack2<kBf16>(sc[2 * kk][0], sc[2 * kk][1]);
-                pa[1] = pack2<kBf16>(sc[2 * kk][2], sc[2 * kk][3]);
-                pa[2] = pack2<kBf16>(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
-                pa[3] = pack2<kBf16>(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
-                if constexpr (kBf16) {  // the residuals P - bf16(P)
-                    pl[0] = lo_part(sc[2 * kk][0], sc[2 * kk][1], pa[0]);
-                    pl[1] = lo_part(sc[2 * kk][2], sc[2 * kk][3], pa[1]);
-                    pl[2] = lo_part(sc[2 * kk + 1][0], sc[2 * kk + 1][1], pa[2]);
-                    pl[3] = lo_part(sc[2 * kk + 1][2], sc[2 * kk + 1][3], pa[3]);
-                }
-                // each V fragment is loaded once; the lo products of the
-                // previous fragment pair follow the hi products of the next
-                uint32_t bp[4];
-#pragma unroll
-                for (int dp = 0; dp < DT / 2; ++dp) {
-                    uint32_t b[4];
-                    const int tr = kk * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-                    ldsm_x4_trans(b, smem_u32(vt_s + pf_off<D>(tr, 2 * dp + (lane >> 4))));
-                    mma16816<kBf16>(o[2 * dp], pa, b[0], b[1]);
-                    mma16816<kBf16>(o[2 * dp + 1], pa, b[2], b[3]);
-                    if constexpr (kBf16) {
-                        if (dp > 0) {
-                            mma16816<kBf16>(o[2 * dp - 2], pl, bp[0], bp[1]);
-                            mma16816<kBf16>(o[2 * dp - 1], pl, bp[2], bp[3]);
-                        }
-                        bp[0] = b[0]; bp[1] = b[1]; bp[2] = b[2]; bp[3] = b[3];
-                    }
-                }
+            for (int e = 0; e < 4; ++e) {
+                const float a = sc[c8 * 8 + 2 * e], b = sc[c8 * 8 + 2 * e + 1];
+                h[e] = pack2<kBf16>(a, b);
                 if constexpr (kBf16) {
-                    mma16816<kBf16>(o[DT - 2], pl, bp[0], bp[1]);
-                    mma16816<kBf16>(o[DT - 1], pl, bp[2], bp[3]);
+                    const float2 hf = unpack2<true>(h[e]);
+                    lo[e] = pack2<true>(a - hf.x, b - hf.y);
                 }
             }
+            const uint32_t off = tc_off(row, c8, kPfRows);
+            *reinterpret_cast<uint4*>(psm + off) = make_uint4(h[0], h[1], h[2], h[3]);
+            if constexpr (kBf16) *reinterpret_cast<uint4*>(psm + SM::kP + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        fence_async_smem();
+        tc_before_sync();
+        __syncthreads();  // P complete; every thread has read its row of S
+        tc_after_sync();
+        if (tid == 0) {  // O_t = P V (hi, then lo)
+            const uint32_t vb = smem_u32(vsm + st * SM::kTile);
+#pragma unroll
+            for (int part = 0; part < SM::kParts; ++part) {
+                const uint32_t pa = smem_u32(psm + part * SM::kP);
+#pragma unroll
+                for (int kk = 0; kk < kPfTok / 16; ++kk)
+                    tc_mma(tO, tc_desc(pa + kk * 32, 16, 1024), tc_desc(vb + kk * 2048, kPfTok * 128, 1024), id_o,
+                           (part > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(smem_u32(&bars[1]));
+        }
+        timed_out |= !tc_wait(smem_u32(&bars[1]), kt & 1);
+        tc_after_sync();
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 16) {
+            float ov[16];
+            tc_ld16(tO + lane_addr + c0, ov);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[c0 + e] = o[c0 + e] * alpha + ov[e];
+        }
+        tc_before_sync();
+        if (__syncthreads_or(timed_out)) {
+            timed_out = true;
+            break;
         }
     }
     pf_wait<0>();
 
-    // ---- normalise and store the valid rows
+    // ---- normalise and store the row
+    if (timed_out) {
+        if (tid == 0) raise_error(p.err, PKV_DEVERR_TIMEOUT);
+    } else if (pos >= 0) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        T* out = static_cast<T*>(p.out) +
+                 ((int64_t)(q0 + tok0 + row / p.g) * p.num_heads + (int64_t)kh * p.g + row % p.g) * D;
 #pragma unroll
-    for (int off = 1; off < 4; off <<= 1) {
-        l0 += __shfl_xor_sync(kFull, l0, off);
-        l1 += __shfl_xor_sync(kFull, l1, off);
-    }
-    const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
-    T* out = static_cast<T*>(p.out);
-    if (pos0 >= 0) {
-        T* row = out + ((int64_t)(q0 + tok0 + r0 / p.g) * p.num_heads + (int64_t)kh * p.g + r0 % p.g) * D;
+        for (int c8 = 0; c8 < D / 8; ++c8) {
+            uint32_t w[4];
 #pragma unroll
-        for (int d = 0; d < DT; ++d)
-            *reinterpret_cast<uint32_t*>(row + d * 8 + 2 * tig) = pack2<kBf16>(o[d][0] * i0, o[d][1] * i0);
+            for (int e = 0; e < 4; ++e) w[e] = pack2<kBf16>(o[c8 * 8 + 2 * e] * inv, o[c8 * 8 + 2 * e + 1] * inv);
+            *reinterpret_cast<uint4*>(out + c8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
     }
-    if (pos1 >= 0) {
-        T* row = out + ((int64_t)(q0 + tok0 + r1 / p.g) * p.num_heads + (int64_t)kh * p.g + r1 % p.g) * D;
-#pragma unroll
-        for (int d = 0; d < DT; ++d)
-            *reinterpret_cast<uint32_t*>(row + d * 8 + 2 * tig) = pack2<kBf16>(o[d][2] * i1, o[d][3] * i1);
-    }
+    tc_before_sync();
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(SM::kTmemCols));
 }
 
 template <typename T, int D>
 pkv_status launch_prefill(const PrefillParams& p, int64_t grid, cudaStream_t st) {
-    constexpr int kSmem = kPfRows * D * 2 + 2 * kPfStages * kPfTok * D * 2;
+    constexpr int kSmem = PfSmem<T, D>::kBytes;
     static std::atomic<unsigned long long> configured{0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(PKV_ECUDA, "cudaGetDevice");
@@ -364,7 +425,7 @@ pkv_status launch_prefill(const PrefillParams& p, int64_t grid, cudaStream_t st)
         if (e != cudaSuccess) return fail(PKV_ECUDA, "prefill smem opt-in: %s", cudaGetErrorString(e));
         configured.fetch_or(bit);
     }
-    pkv_prefill_kernel<T, D><<<(unsigned)grid, kPfWarps * 32, kSmem, st>>>(p);
+    pkv_prefill_kernel<T, D><<<(unsigned)grid, kPfThreads, kSmem, st>>>(p);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "prefill launch: %s", cudaGetErrorString(e));
     return PKV_OK;

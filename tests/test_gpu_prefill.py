@@ -92,6 +92,27 @@ def test_prefill_full_step_sampled(budget):
     check(out, oracle_rows(wl, kc, vc, rows), wl.kv_dtype, rows)
 
 
+def test_growing_scores_exercise_the_rescale():
+    # keys of later positions scaled up so each 64-token tile's maximum score
+    # exceeds the running reference by far more than 2^8: the accumulator
+    # rescale path runs on every tile
+    wl = W.build_prefill("rescale", [0, 70], [200, 90], 8, 2, 128, 16, torch.bfloat16, seed=25)
+    bs = wl.block_size
+    for s_ in range(wl.num_seqs):
+        L = int(wl.seq_lens[s_])
+        C = int(wl.query_start[s_ + 1] - wl.query_start[s_])
+        for t in range(L - C):                      # cached context tokens
+            b = int(wl.block_tables[s_, t // bs])
+            wl.key_cache[b, t % bs] = (wl.key_cache[b, t % bs].float() * (1.0 + t / 8.0)).to(torch.bfloat16)
+    wl.new_key = (wl.new_key.float() * torch.linspace(1.0, 30.0, wl.num_tokens)[:, None, None]).to(torch.bfloat16)
+    wl.query = (wl.query.float() * 3.0).to(torch.bfloat16)
+    out, err, _, _ = gpu_prefill(wl)
+    assert err == 0
+    kc, vc = oracle_caches(wl)
+    ref = oracle.paged_prefill(wl.query, kc, vc, wl.block_tables, wl.seq_lens, wl.query_start, wl.scale)
+    check(out, ref, torch.bfloat16)
+
+
 def test_splitting_a_chunk_is_bit_identical():
     # the same 150 tokens as one chunk, or as chunks of 70 and 80 in two calls
     wl = W.build_prefill("whole", [40], [150], 8, 4, 128, 16, torch.bfloat16, seed=22)
