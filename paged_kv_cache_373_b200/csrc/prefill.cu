@@ -36,7 +36,7 @@ namespace {
 constexpr int kPfRows = 128;   // query rows per unit (tensor-core M)
 constexpr int kPfTok = 64;     // KV tokens per tile (N of S, K of P V)
 constexpr int kPfStages = 2;   // K/V ring depth
-constexpr int kPfThreads = 128;
+constexpr int kPfThreads = 256;  // two threads per row: warps w and w + 4 share TMEM lanes
 
 struct PrefillParams {
     void* out;
@@ -154,6 +154,7 @@ pkv_prefill_kernel(const PrefillParams p) {
     uint8_t* psm = vsm + kPfStages * SM::kTile;  // P hi, then P lo (bf16)
     __shared__ __align__(8) uint64_t bars[2];     // S done, O_t done
     __shared__ uint32_t tmem_base;
+    __shared__ float xmax[2][kPfRows];            // the two halves' row maxima (and, at the end, sums)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     // ---- the unit: kv head from the block index, then row tile u among all
@@ -280,19 +281,21 @@ pkv_prefill_kernel(const PrefillParams p) {
     pf_commit();
     if (nkv > 1) load_phys(1, phn);
 
-    // ---- this thread's row
-    const int row = tid;
+    // ---- this thread's row and half: S columns [32 half, 32 half + 32), O
+    // columns [half D / 2, (half + 1) D / 2)
+    const int row = tid & (kPfRows - 1), half = tid >> 7;
+    constexpr int SH = kPfTok / 2, DH = D / 2;
     const int pos = (row / p.g < ntok) ? ctx + tok0 + row / p.g : -1;
-    float o[D];
+    float o[DH];
 #pragma unroll
-    for (int d = 0; d < D; ++d) o[d] = 0.f;
+    for (int d = 0; d < DH; ++d) o[d] = 0.f;
     float m = -INFINITY, l = 0.f;
 
     __syncthreads();  // barriers initialised, tensor memory allocated
     tc_after_sync();
     const uint32_t tmem = tmem_base;
     const uint32_t tS = tmem, tO = tmem + kPfTok;                  // columns
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;        // this warp's 32 lanes
+    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;  // this warp's 32 lanes
     const uint32_t id_s = tc_idesc<kBf16>(kPfRows, kPfTok, 0);
     const uint32_t id_o = tc_idesc<kBf16>(kPfRows, D, 1);
     bool timed_out = false;
@@ -319,31 +322,35 @@ pkv_prefill_kernel(const PrefillParams p) {
         pf_commit();
         timed_out |= !tc_wait(smem_u32(&bars[0]), kt & 1);
         tc_after_sync();
-        // ---- this row's scores: scale (log2 domain), causal mask, online softmax
-        float sc[kPfTok];
+        // ---- this row's scores: scale (log2 domain), causal mask, online
+        // softmax; the row maximum is combined with the other half's
+        float sc[SH];
 #pragma unroll
-        for (int c0 = 0; c0 < kPfTok; c0 += 16) tc_ld16(tS + lane_addr + c0, sc + c0);
-        const int t0 = kt * kPfTok;
-        float mx = -INFINITY;
+        for (int c0 = 0; c0 < SH; c0 += 16) tc_ld16(tS + lane_addr + half * SH + c0, sc + c0);
+        const int t0 = kt * kPfTok + half * SH;
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < kPfTok; ++c) {
+        for (int c = 0; c < SH; ++c) {
             sc[c] = t0 + c <= pos ? sc[c] * p.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, sc[c]);
+            mx4[c & 3] = fmaxf(mx4[c & 3], sc[c]);
         }
+        xmax[half][row] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        __syncthreads();
+        const float mx = fmaxf(xmax[0][row], xmax[1][row]);
         const float mn = fmaxf(m, mx);
         const float ref = mn == -INFINITY ? 0.f : mn;  // a row with nothing attended yet
         const float alpha = ex2(m - ref);
         m = mn;
-        float ls = 0.f;
+        float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < kPfTok; ++c) {
+        for (int c = 0; c < SH; ++c) {
             sc[c] = ex2(sc[c] - ref);
-            ls += sc[c];
+            ls4[c & 3] += sc[c];
         }
-        l = l * alpha + ls;
-        // ---- P to shared memory (K-major rows; bf16 as hi + lo parts)
+        l = l * alpha + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));  // this half's share of the sum
+        // ---- this half of P to shared memory (K-major rows; bf16 as hi + lo parts)
 #pragma unroll
-        for (int c8 = 0; c8 < kPfTok / 8; ++c8) {
+        for (int c8 = 0; c8 < SH / 8; ++c8) {
             uint32_t h[4], lo[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -354,7 +361,7 @@ pkv_prefill_kernel(const PrefillParams p) {
                     lo[e] = pack2<true>(a - hf.x, b - hf.y);
                 }
             }
-            const uint32_t off = tc_off(row, c8, kPfRows);
+            const uint32_t off = tc_off(row, half * (SH / 8) + c8, kPfRows);
             *reinterpret_cast<uint4*>(psm + off) = make_uint4(h[0], h[1], h[2], h[3]);
             if constexpr (kBf16) *reinterpret_cast<uint4*>(psm + SM::kP + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
@@ -377,9 +384,9 @@ pkv_prefill_kernel(const PrefillParams p) {
         timed_out |= !tc_wait(smem_u32(&bars[1]), kt & 1);
         tc_after_sync();
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 16) {
+        for (int c0 = 0; c0 < DH; c0 += 16) {
             float ov[16];
-            tc_ld16(tO + lane_addr + c0, ov);
+            tc_ld16(tO + lane_addr + half * DH + c0, ov);
 #pragma unroll
             for (int e = 0; e < 16; ++e) o[c0 + e] = o[c0 + e] * alpha + ov[e];
         }
@@ -391,15 +398,18 @@ pkv_prefill_kernel(const PrefillParams p) {
     }
     pf_wait<0>();
 
-    // ---- normalise and store the row
+    // ---- normalise (the two halves' sums combined) and store this half of the row
+    xmax[half][row] = l;
+    __syncthreads();
+    const float lt = xmax[0][row] + xmax[1][row];
     if (timed_out) {
         if (tid == 0) raise_error(p.err, PKV_DEVERR_TIMEOUT);
     } else if (pos >= 0) {
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
         T* out = static_cast<T*>(p.out) +
-                 ((int64_t)(q0 + tok0 + row / p.g) * p.num_heads + (int64_t)kh * p.g + row % p.g) * D;
+                 ((int64_t)(q0 + tok0 + row / p.g) * p.num_heads + (int64_t)kh * p.g + row % p.g) * D + half * DH;
 #pragma unroll
-        for (int c8 = 0; c8 < D / 8; ++c8) {
+        for (int c8 = 0; c8 < DH / 8; ++c8) {
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) w[e] = pack2<kBf16>(o[c8 * 8 + 2 * e] * inv, o[c8 * 8 + 2 * e + 1] * inv);
