@@ -5,22 +5,29 @@
 // of sequence s sits at position p = seq_lens[s] - C_s + i and attends to the
 // cached tokens t <= p through the block table.
 //
-// Work unit: (sequence, kv head, 128 query rows); a row is a (chunk token,
-// q head of the kv head's group) pair, so one K/V tile in shared memory serves
-// all g heads of every token in the unit.  A CTA of 4 warps (thread = row):
-//   - gathers the unit's 64-token K/V tiles through the table with 16-byte
-//     cp.async (zero fill past the unit's last position, 2-stage ring) into
-//     the 128-byte-swizzled layout the tensor core reads;
-//   - one thread issues S = Q K^T on the 5th-generation tensor core
-//     (tcgen05.mma, M = 128 rows, N = 64 tokens, accumulator in tensor
-//     memory), every thread loads its row of S from tensor memory and runs
-//     the online softmax in registers;
-//   - P is written to shared memory (bf16: hi + lo parts, so P V keeps
-//     fp32-level accuracy) and O_t = P V_t is issued (N = head_dim, V read
-//     MN-major); each thread folds its row of O_t into its running output.
-// Completion of each group of tensor-core products is signalled on an
-// mbarrier (tcgen05.commit); every wait is bounded and a timeout sets
-// PKV_DEVERR_TIMEOUT.
+// Unit: (sequence, kv head, 128 query rows); a row is a (chunk token, q head
+// of the kv head's group) pair, so one K/V tile serves all g heads of every
+// token in the unit.  A CTA takes two adjacent units of one (sequence, kv
+// head) -- they read the same K/V tiles -- and keeps the tensor core busy on
+// one unit while the other runs its softmax:
+//   - warp 17 (one lane) copies the units' q rows and then, through the
+//     block table, each 64-token K and V tile with TMA into the 128-byte
+//     swizzled layout the tensor core reads (2-stage K and V rings);
+//   - warp 16 (one lane) owns tensor memory and issues, per tile,
+//     O_0 += P_0 V, S_0' = Q_0 K'^T, O_1 += P_1 V, S_1' = Q_1 K'^T
+//     (tcgen05.mma, M = 128 rows, fp32 accumulators in tensor memory);
+//   - warps 0-7 and 8-15 are the two units' softmax groups, two threads per
+//     row (one per half of the 64 scores and of the head_dim outputs): load
+//     S from tensor memory, mask, exponentiate against a reference maximum,
+//     write P to shared memory (bf16 as hi + lo parts, so P V keeps
+//     fp32-level accuracy).  O stays in tensor memory across tiles; it is
+//     rescaled only when a row's maximum passes its reference by 2^8.
+// Every hand-off is an mbarrier; every wait is bounded (0.2 s of
+// %globaltimer): a timeout sets PKV_DEVERR_TIMEOUT, every role leaves its
+// loop, the copies and products already issued are drained, and the CTA
+// frees its tensor memory and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -33,16 +40,32 @@
 namespace pkv {
 namespace {
 
-constexpr int kPfRows = 128;   // query rows per unit (tensor-core M)
-constexpr int kPfTok = 64;     // KV tokens per tile (N of S, K of P V)
-constexpr int kPfStages = 2;   // K/V ring depth
-constexpr int kPfThreads = 256;  // two threads per row: warps w and w + 4 share TMEM lanes
+constexpr int kPfRows = 128;        // query rows per unit (tensor-core M)
+constexpr int kPfTok = 64;          // KV tokens per tile (N of S, K of P V)
+constexpr int kPfGroup = 256;       // softmax threads per unit: two per row
+constexpr int kPfMmaWarp = 16;      // issues the tensor-core products, owns tensor memory
+constexpr int kPfLoadWarp = 17;     // issues the TMA copies
+constexpr int kPfThreads = 18 * 32;
+constexpr int kPfTmemCols = 512;    // unit u: S in columns [256 u, 256 u + 64), O from 256 u + 64
+constexpr uint64_t kPfWaitNs = 200000000ull;
+
+// mbarriers
+enum : int {
+    kBarQ = 0,        // q rows landed (TMA transaction count)
+    kBarKFull = 1,    // [2] K tile landed
+    kBarVFull = 3,    // [2] V tile landed
+    kBarKEmpty = 5,   // [2] every S product of the K stage finished
+    kBarVEmpty = 7,   // [2] every P V product of the V stage finished
+    kBarVFix = 9,     // the last V tile's rows past the unit's end are zeroed
+    kBarS = 10,       // [2] S of unit u ready
+    kBarP = 12,       // [2] P of unit u written (and S read): kPfGroup arrivals
+    kBarO = 14,       // [2] P V of unit u finished
+    kBarDrain = 16,   // products drained (abort path)
+    kNumBars = 17
+};
 
 struct PrefillParams {
     void* out;
-    const void* q;
-    const uint8_t* kc;
-    const uint8_t* vc;
     const int32_t* tables;
     const int32_t* seq_lens;
     const int32_t* qstart;
@@ -56,7 +79,8 @@ struct PrefillParams {
 // as column blocks of 64 elements: block c / 8 holds rows x 128 bytes, and
 // inside it 8-row groups of 1024 bytes with the 128-byte XOR swizzle.  This
 // is the canonical swizzled layout of the tensor core's shared-memory
-// operands (K-major rows for Q, K and P; MN-major for V).
+// operands (K-major rows for Q, K and P; MN-major for V), and the layout a
+// TMA copy with 128-byte swizzle writes for a box 64 elements wide.
 __device__ __forceinline__ uint32_t tc_off(int r, int c, int rows) {
     return (uint32_t)((c >> 3) * rows * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
@@ -89,8 +113,18 @@ __device__ __forceinline__ uint64_t global_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-// Wait for the mbarrier phase `parity`; false after 0.2 s of wall-clock time.
-__device__ __forceinline__ bool tc_wait(uint32_t mbar, uint32_t parity) {
+__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
+}
+// Wait for the mbarrier phase `parity`.  False after 0.2 s of wall-clock time
+// (the abort flag is then raised) or as soon as another role raised it.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, volatile int* abort) {
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
         uint32_t ok;
@@ -99,69 +133,123 @@ __device__ __forceinline__ bool tc_wait(uint32_t mbar, uint32_t parity) {
                      : "=r"(ok) : "r"(mbar), "r"(parity) : "memory");
         if (ok) return true;
         if ((it & 63) == 63) {
+            if (abort && *abort) return false;
             const uint64_t now = global_ns();
-            if (t0 == 0) t0 = now;
-            else if (now - t0 > 200000000ull) return false;
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > kPfWaitNs) {
+                if (abort) *abort = 1;
+                return false;
+            }
         }
     }
 }
-// 16 consecutive fp32 columns of this thread's tensor-memory lane.
+// Named barrier over one softmax group (kPfGroup threads, whole warps) that
+// also ORs a flag across it.
+__device__ __forceinline__ bool group_sync_or(int id, bool flag) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}\n"
+                 : "=r"(r) : "r"((uint32_t)flag), "r"(id), "n"(kPfGroup) : "memory");
+    return r != 0;
+}
+// 3-D TMA tile load into shared memory, completing on an mbarrier.
+__device__ __forceinline__ void tma_load3(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                          uint32_t mbar) {
+    asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+                 "[%0], [%1, {%2, %3, %4}], [%5];"
+                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(mbar)
+                 : "memory");
+}
+// 16 / 32 consecutive fp32 columns of this thread's tensor-memory lane; the
+// wait is in the same statement, so no use of the values can move above it.
 __device__ __forceinline__ void tc_ld16(uint32_t taddr, float* v) {
     uint32_t r[16];
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
                    "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
                    "=r"(r[14]), "=r"(r[15])
-                 : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                 : "r"(taddr)
+                 : "memory");
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+                   "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+                   "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 16 fp32 columns into this thread's lane, waited for before returning.
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const float* v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+                 "tcgen05.wait::st.sync.aligned;"
+                 ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+                   "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+                   "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+                   "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+                   "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+                   "r"(__float_as_uint(v[15]))
+                 : "memory");
 }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 16-byte async copy; src_bytes = 0 writes zeros (no global read)
-__device__ __forceinline__ void cp16_zfill(uint32_t dst, const void* src, int src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void pf_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void pf_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
 template <typename T, int D>
 struct PfSmem {
-    static constexpr int kQ = kPfRows * D * 2;
+    static constexpr int kQ = kPfRows * D * 2;     // one unit's q rows
     static constexpr int kTile = kPfTok * D * 2;   // one K or V tile
     static constexpr int kP = kPfRows * kPfTok * 2;
     static constexpr int kParts = std::is_same<T, __nv_bfloat16>::value ? 2 : 1;  // P hi (+ lo)
-    static constexpr int kBytes = kQ + 2 * kPfStages * kTile + kParts * kP + 1024;  // + alignment
-    static constexpr int kTmemCols = 256;            // S (64 columns) + O_t (D columns)
+    static constexpr int kData = 2 * kQ + 4 * kTile + 2 * kParts * kP + 1024;     // + alignment
+    // at least 120 KB, so one CTA (and its 512 tensor-memory columns) per SM
+    static constexpr int kBytes = kData > 120 * 1024 ? kData : 120 * 1024;
+};
+
+// The geometry of one 128-row unit.
+struct PfUnit {
+    int tok0, ntok, pos0, kv_end, nkv;
 };
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kPfThreads, 1)
-pkv_prefill_kernel(const PrefillParams p) {
+pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
+                   const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v) {
     using SM = PfSmem<T, D>;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr int CH = D / 8;  // 16-byte chunks per row
     extern __shared__ uint8_t pf_raw[];
     uint8_t* sm = pf_raw + ((1024 - (smem_u32(pf_raw) & 1023)) & 1023);  // 1024-byte aligned operands
-    uint8_t* qsm = sm;
-    uint8_t* ksm = qsm + SM::kQ;
-    uint8_t* vsm = ksm + kPfStages * SM::kTile;
-    uint8_t* psm = vsm + kPfStages * SM::kTile;  // P hi, then P lo (bf16)
-    __shared__ __align__(8) uint64_t bars[2];     // S done, O_t done
+    uint8_t* qsm = sm;                          // [2 units]
+    uint8_t* ksm = qsm + 2 * SM::kQ;            // [2 stages]
+    uint8_t* vsm = ksm + 2 * SM::kTile;         // [2 stages]
+    uint8_t* psm = vsm + 2 * SM::kTile;         // [2 units][hi, lo]
+    __shared__ __align__(8) uint64_t bars[kNumBars];
     __shared__ uint32_t tmem_base;
-    __shared__ float xmax[2][kPfRows];            // the two halves' row maxima (and, at the end, sums)
+    __shared__ int abort_flag;
+    __shared__ float xmax[2][2][2][kPfRows];    // [unit][tile parity][half][row] partial row maxima
+    __shared__ float xsum[2][2][kPfRows];       // [unit][half][row] partial row sums
+    volatile int* abort = &abort_flag;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
-    // ---- the unit: kv head from the block index, then row tile u among all
-    // sequences' row tiles (warp-parallel scan; every warp finds it)
+    // ---- the unit pair: kv head from the block index, then pair u among all
+    // sequences' pairs (warp-parallel scan; every warp finds it).  A
+    // sequence's row tiles pair from the last: (n-1, n-2), (n-3, n-4), ...
     const int kh = (int)(blockIdx.x % p.num_kv_heads);
     const int64_t u = blockIdx.x / p.num_kv_heads;
-    int s = -1, j = 0;
+    int s = -1, jp = 0, nrt_s = 0;
     {
         int64_t base = 0;
         for (int s0 = 0; s0 < p.num_seqs && s < 0; s0 += 32) {
@@ -172,25 +260,26 @@ pkv_prefill_kernel(const PrefillParams p) {
                 if (C < 0 && blockIdx.x == 0 && warp == 0) raise_error(p.err, PKV_DEVERR_SEQ_LEN);
                 nrt = C > 0 ? (int)(((int64_t)C * p.g + kPfRows - 1) / kPfRows) : 0;
             }
-            int incl = nrt;
+            const int npr = (nrt + 1) >> 1;
+            int incl = npr;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int y = __shfl_up_sync(kFull, incl, o);
                 if (lane >= o) incl += y;
             }
-            const int64_t lo = base + incl - nrt;
-            const unsigned hit = __ballot_sync(kFull, nrt > 0 && u >= lo && u < lo + nrt);
+            const int64_t lo = base + incl - npr;
+            const unsigned hit = __ballot_sync(kFull, npr > 0 && u >= lo && u < lo + npr);
             if (hit) {
                 const int src = __ffs(hit) - 1;
                 s = s0 + src;
                 const int64_t l0 = __shfl_sync(kFull, lo, src);
-                const int nr = __shfl_sync(kFull, nrt, src);
-                j = nr - 1 - (int)(u - l0);  // a sequence's last (heaviest) row tile first
+                nrt_s = __shfl_sync(kFull, nrt, src);
+                jp = (int)(u - l0);  // a sequence's heaviest pair first
             }
             base += __shfl_sync(kFull, incl, 31);
         }
     }
-    if (s < 0) return;  // past the last unit
+    if (s < 0) return;  // past the last pair
     const int q0 = __ldg(p.qstart + s);
     const int C = __ldg(p.qstart + s + 1) - q0;
     const int L = __ldg(p.seq_lens + s);
@@ -199,232 +288,365 @@ pkv_prefill_kernel(const PrefillParams p) {
         return;
     }
     const int ctx = L - C;
-    const int tpu = kPfRows / p.g;           // chunk tokens per unit (g divides 16)
-    const int tok0 = j * tpu;
-    const int ntok = min(tpu, C - tok0);
-    const int kv_end = ctx + tok0 + ntok;    // the unit reads KV tokens [0, kv_end)
-    const int nkv = (kv_end + kPfTok - 1) / kPfTok;
-    const int32_t* trow = p.tables + (int64_t)s * p.mbps;
+    const int tpu = kPfRows / p.g;  // chunk tokens per unit (g divides 16)
+    const int j0 = nrt_s - 1 - 2 * jp, j1 = j0 - 1;
+    const int nunits = j1 >= 0 ? 2 : 1;
+    auto make_unit = [&](int j) {
+        PfUnit w;
+        w.tok0 = j * tpu;
+        w.ntok = min(tpu, C - w.tok0);
+        w.pos0 = ctx + w.tok0;
+        w.kv_end = w.pos0 + w.ntok;
+        w.nkv = (w.kv_end + kPfTok - 1) / kPfTok;
+        return w;
+    };
+    const PfUnit U0 = make_unit(j0);                 // the later rows: the longer K/V range
+    const PfUnit U1 = make_unit(j1 >= 0 ? j1 : j0);  // (unused when nunits == 1)
+    const int nkv = U0.nkv;
+    const bool need_fix = (U0.kv_end % kPfTok) != 0;  // V rows past the end must read as zeros
 
-    // ---- tensor memory and barriers
-    if (warp == 0) {
+    // ---- tensor memory, barriers
+    if (warp == kPfMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base)),
-                     "r"(SM::kTmemCols));
+                     "r"(kPfTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
     }
     if (tid == 0) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[i])));
+        for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), (i == kBarP || i == kBarP + 1) ? kPfGroup : 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        abort_flag = 0;
     }
-
-    // ---- q rows (zero past the chunk), with the first K/V tile
-    for (int i = tid; i < kPfRows * CH; i += kPfThreads) {
-        const int r = i / CH, c = i % CH;
-        const int tl = r / p.g;
-        const uint8_t* src = static_cast<const uint8_t*>(p.q);
-        int nb = 0;
-        if (tl < ntok) {
-            src += ((int64_t)(q0 + tok0 + tl) * p.num_heads + (int64_t)kh * p.g + r % p.g) * (D * 2) + c * 16;
-            nb = 16;
-        }
-        cp16_zfill(smem_u32(qsm + tc_off(r, c, kPfRows)), src, nb);
-    }
-    // each thread copies chunk cc of rows rr, rr + RSTEP, ... of a K/V tile;
-    // the tile's physical blocks are read from the table one tile ahead of
-    // their copies (the copies' asm is a compiler memory barrier)
-    constexpr int RSTEP = kPfThreads / CH;
-    constexpr int NIT = kPfTok / RSTEP;
-    constexpr int NBLK = kPfTok / 16;
-    const int rr = tid / CH, cc = tid % CH;
-    const int lg_bs = p.bs == 16 ? 4 : 5;
-    auto load_phys = [&](int kt, int (&ph)[NBLK]) {
-#pragma unroll
-        for (int jb = 0; jb < NBLK; ++jb) {
-            const int t = kt * kPfTok + (jb << lg_bs);
-            ph[jb] = (t < kv_end && (jb << lg_bs) < kPfTok) ? __ldg(trow + (t >> lg_bs)) : -1;
-        }
-    };
-    auto issue_kv = [&](int kt, int stage, const int (&ph)[NBLK]) {
-        uint8_t* kd = ksm + stage * SM::kTile;
-        uint8_t* vd = vsm + stage * SM::kTile;
-#pragma unroll
-        for (int i = 0; i < NIT; ++i) {
-            const int r = rr + RSTEP * i;
-            const int t = kt * kPfTok + r;
-            const int jb = r >> lg_bs;
-            int phys = ph[0];
-#pragma unroll
-            for (int q = 1; q < NBLK; ++q) phys = jb == q ? ph[q] : phys;
-            const uint8_t* ks = p.kc;
-            const uint8_t* vs = p.vc;
-            int nb = 0;
-            if (t < kv_end) {
-                if (phys >= 0 && phys < p.num_blocks) {
-                    const int64_t off =
-                        (((int64_t)phys * p.bs + (t & (p.bs - 1))) * p.num_kv_heads + kh) * (D * 2) + cc * 16;
-                    ks += off;
-                    vs += off;
-                    nb = 16;
-                } else if (cc == 0) {
-                    raise_error(p.err, PKV_DEVERR_BLOCK_ID);
-                }
-            }
-            const uint32_t so = tc_off(r, cc, kPfTok);
-            cp16_zfill(smem_u32(kd + so), ks, nb);
-            cp16_zfill(smem_u32(vd + so), vs, nb);
-        }
-    };
-    int phn[NBLK];
-    load_phys(0, phn);
-    issue_kv(0, 0, phn);
-    pf_commit();
-    if (nkv > 1) load_phys(1, phn);
-
-    // ---- this thread's row and half: S columns [32 half, 32 half + 32), O
-    // columns [half D / 2, (half + 1) D / 2)
-    const int row = tid & (kPfRows - 1), half = tid >> 7;
-    constexpr int SH = kPfTok / 2, DH = D / 2;
-    const int pos = (row / p.g < ntok) ? ctx + tok0 + row / p.g : -1;
-    float o[DH];
-#pragma unroll
-    for (int d = 0; d < DH; ++d) o[d] = 0.f;
-    float m = -INFINITY, l = 0.f;
-
-    __syncthreads();  // barriers initialised, tensor memory allocated
+    __syncthreads();
     tc_after_sync();
     const uint32_t tmem = tmem_base;
-    const uint32_t tS = tmem, tO = tmem + kPfTok;                  // columns
-    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;  // this warp's 32 lanes
-    const uint32_t id_s = tc_idesc<kBf16>(kPfRows, kPfTok, 0);
-    const uint32_t id_o = tc_idesc<kBf16>(kPfRows, D, 1);
-    bool timed_out = false;
 
+    if (warp < 2 * (kPfGroup / 32)) {
+        // ================= softmax groups: unit X, two threads per row
+        const int X = warp >> 3;
+        if (X < nunits) {
+            const PfUnit U = X ? U1 : U0;
+            const int wq = warp & 3, half = (warp >> 2) & 1;
+            const int row = wq * 32 + lane;
+            const int pos = (row / p.g < U.ntok) ? U.pos0 + row / p.g : -1;
+            const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
+            const uint32_t tS = tmem + lane_addr + X * 256 + half * (kPfTok / 2);
+            const uint32_t tO = tmem + lane_addr + X * 256 + kPfTok + half * (D / 2);
+            uint8_t* pu = psm + X * SM::kParts * SM::kP;
+            const float sl2 = p.scale_log2;
+            float mref = -INFINITY, l = 0.f;  // reference maximum (log2 domain) and this half's sum
+            bool failed = false;
 #pragma unroll 1
-    for (int kt = 0; kt < nkv; ++kt) {
-        pf_wait<0>();
-        fence_async_smem();  // the copies, visible to the tensor core
-        __syncthreads();     // tile kt (and q) complete; every thread done with tile kt - 1
-        tc_after_sync();
-        const int st = kt % kPfStages;
-        if (tid == 0) {  // S = Q K^T
-            const uint32_t qa = smem_u32(qsm), kb = smem_u32(ksm + st * SM::kTile);
+            for (int kt = 0; kt < U.nkv; ++kt) {
+                bool ok = !failed && mbar_wait(bar(kBarS + X), kt & 1, abort);
+                ok = __all_sync(kFull, ok);
+                float sc[kPfTok / 2];
+                float pm = -INFINITY;
+                if (ok) {
+                    tc_after_sync();
+                    tc_ld32(tS, sc);
+                    if (kt * kPfTok + kPfTok - 1 > U.pos0) {  // a tile on the causal diagonal
+                        const int t0 = kt * kPfTok + half * (kPfTok / 2);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-                tc_mma(tS, tc_desc(qa + (kk >> 2) * kPfRows * 128 + (kk & 3) * 32, 16, 1024),
-                       tc_desc(kb + (kk >> 2) * kPfTok * 128 + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
-            tc_commit(smem_u32(&bars[0]));
-        }
-        if (kt + 1 < nkv) {  // the next tile into the other stage (its last reader, tile kt - 1, is done)
-            issue_kv(kt + 1, (kt + 1) % kPfStages, phn);
-            if (kt + 2 < nkv) load_phys(kt + 2, phn);
-        }
-        pf_commit();
-        timed_out |= !tc_wait(smem_u32(&bars[0]), kt & 1);
-        tc_after_sync();
-        // ---- this row's scores: scale (log2 domain), causal mask, online
-        // softmax; the row maximum is combined with the other half's
-        float sc[SH];
+                        for (int c = 0; c < kPfTok / 2; ++c) sc[c] = t0 + c <= pos ? sc[c] : -INFINITY;
+                    }
+                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c0 = 0; c0 < SH; c0 += 16) tc_ld16(tS + lane_addr + half * SH + c0, sc + c0);
-        const int t0 = kt * kPfTok + half * SH;
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    for (int c = 0; c < kPfTok / 2; ++c) m4[c & 3] = fmaxf(m4[c & 3], sc[c]);
+                    pm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                }
+                xmax[X][kt & 1][half][row] = pm;
+                if (group_sync_or(1 + X, !ok)) {
+                    failed = true;
+                    break;
+                }
+                // the row maximum of this tile (both halves), in the log2 domain
+                const float mx = fmaxf(xmax[X][kt & 1][0][row], xmax[X][kt & 1][1][row]) * sl2;
+                const bool grow = mx > mref + 8.f;  // also the first finite maximum
+                float alpha = 1.f;
+                if (grow) {
+                    alpha = ex2(mref - mx);  // 0 while nothing was attended
+                    l *= alpha;
+                    mref = mx;
+                }
+                const float ref = mref == -INFINITY ? 0.f : mref;
+                float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < SH; ++c) {
-            sc[c] = t0 + c <= pos ? sc[c] * p.scale_log2 : -INFINITY;
-            mx4[c & 3] = fmaxf(mx4[c & 3], sc[c]);
-        }
-        xmax[half][row] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        __syncthreads();
-        const float mx = fmaxf(xmax[0][row], xmax[1][row]);
-        const float mn = fmaxf(m, mx);
-        const float ref = mn == -INFINITY ? 0.f : mn;  // a row with nothing attended yet
-        const float alpha = ex2(m - ref);
-        m = mn;
-        float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int c = 0; c < kPfTok / 2; ++c) {
+                    sc[c] = ex2(fmaf(sc[c], sl2, -ref));
+                    ls4[c & 3] += sc[c];
+                }
+                l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+                if (kt > 0) {  // P V of the previous tile done: its P buffer is free, O is settled
+                    ok = mbar_wait(bar(kBarO + X), (kt - 1) & 1, abort);
+                    ok = __all_sync(kFull, ok);
+                    if (ok) {
+                        tc_after_sync();
+                        if (__any_sync(kFull, grow)) {  // rescale this half row of O
+#pragma unroll 1
+                            for (int c0 = 0; c0 < D / 2; c0 += 16) {
+                                float v[16];
+                                tc_ld16(tO + c0, v);
 #pragma unroll
-        for (int c = 0; c < SH; ++c) {
-            sc[c] = ex2(sc[c] - ref);
-            ls4[c & 3] += sc[c];
-        }
-        l = l * alpha + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));  // this half's share of the sum
-        // ---- this half of P to shared memory (K-major rows; bf16 as hi + lo parts)
+                                for (int e = 0; e < 16; ++e) v[e] *= alpha;
+                                tc_st16(tO + c0, v);
+                            }
+                        }
+                    }
+                }
+                if (!ok) {
+                    failed = true;
+                    continue;  // the next tile's group barrier ends the loop for the whole group
+                }
+                // ---- this half of P (K-major rows; bf16 as hi + lo parts)
 #pragma unroll
-        for (int c8 = 0; c8 < SH / 8; ++c8) {
-            uint32_t h[4], lo[4];
+                for (int c8 = 0; c8 < kPfTok / 16; ++c8) {
+                    uint32_t h[4], lo[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float a = sc[c8 * 8 + 2 * e], b = sc[c8 * 8 + 2 * e + 1];
-                h[e] = pack2<kBf16>(a, b);
-                if constexpr (kBf16) {
-                    const float2 hf = unpack2<true>(h[e]);
-                    lo[e] = pack2<true>(a - hf.x, b - hf.y);
+                    for (int e = 0; e < 4; ++e) {
+                        const float a = sc[c8 * 8 + 2 * e], b = sc[c8 * 8 + 2 * e + 1];
+                        h[e] = pack2<kBf16>(a, b);
+                        if constexpr (kBf16) {
+                            const float2 hf = unpack2<true>(h[e]);
+                            lo[e] = pack2<true>(a - hf.x, b - hf.y);
+                        }
+                    }
+                    const uint32_t off = tc_off(row, half * (kPfTok / 16) + c8, kPfRows);
+                    *reinterpret_cast<uint4*>(pu + off) = make_uint4(h[0], h[1], h[2], h[3]);
+                    if constexpr (kBf16)
+                        *reinterpret_cast<uint4*>(pu + SM::kP + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                }
+                fence_async_smem();
+                tc_before_sync();
+                mbar_arrive(bar(kBarP + X));
+            }
+            // ---- the last P V, then normalise (the halves' sums combined) and store
+            bool ok = !failed && mbar_wait(bar(kBarO + X), (U.nkv - 1) & 1, abort);
+            ok = __all_sync(kFull, ok);
+            xsum[X][half][row] = l;
+            if (!group_sync_or(1 + X, !ok)) {
+                tc_after_sync();
+                const float lt = xsum[X][0][row] + xsum[X][1][row];
+                const float inv = lt > 0.f ? 1.f / lt : 0.f;
+                T* out = static_cast<T*>(p.out) +
+                         ((int64_t)(q0 + U.tok0 + row / p.g) * p.num_heads + (int64_t)kh * p.g + row % p.g) * D +
+                         half * (D / 2);
+#pragma unroll 1
+                for (int c0 = 0; c0 < D / 2; c0 += 16) {
+                    float v[16];
+                    tc_ld16(tO + c0, v);  // every lane loads (warp-collective); only real rows store
+                    uint32_t w[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) w[e] = pack2<kBf16>(v[2 * e] * inv, v[2 * e + 1] * inv);
+                    if (pos >= 0) {
+                        *reinterpret_cast<uint4*>(out + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+                        *reinterpret_cast<uint4*>(out + c0 + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+                    }
                 }
             }
-            const uint32_t off = tc_off(row, half * (SH / 8) + c8, kPfRows);
-            *reinterpret_cast<uint4*>(psm + off) = make_uint4(h[0], h[1], h[2], h[3]);
-            if constexpr (kBf16) *reinterpret_cast<uint4*>(psm + SM::kP + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
-        fence_async_smem();
-        tc_before_sync();
-        __syncthreads();  // P complete; every thread has read its row of S
-        tc_after_sync();
-        if (tid == 0) {  // O_t = P V (hi, then lo)
-            const uint32_t vb = smem_u32(vsm + st * SM::kTile);
+    } else if (warp == kPfMmaWarp) {
+        // ================= tensor-core issue (one lane)
+        if (lane == 0) {
+            const uint32_t id_s = tc_idesc<kBf16>(kPfRows, kPfTok, 0);
+            const uint32_t id_o = tc_idesc<kBf16>(kPfRows, D, 1);
+            auto issue_s = [&](int X, int st) {  // S_X = Q_X K^T
+                const uint32_t qa = smem_u32(qsm + X * SM::kQ), kb = smem_u32(ksm + st * SM::kTile);
 #pragma unroll
-            for (int part = 0; part < SM::kParts; ++part) {
-                const uint32_t pa = smem_u32(psm + part * SM::kP);
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc_mma(tmem + X * 256, tc_desc(qa + (kk >> 2) * kPfRows * 128 + (kk & 3) * 32, 16, 1024),
+                           tc_desc(kb + (kk >> 2) * kPfTok * 128 + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
+                tc_commit(bar(kBarS + X));
+            };
+            auto issue_pv = [&](int X, int st, bool acc) {  // O_X (+)= P_X V (hi, then lo)
+                const uint32_t vb = smem_u32(vsm + st * SM::kTile);
 #pragma unroll
-                for (int kk = 0; kk < kPfTok / 16; ++kk)
-                    tc_mma(tO, tc_desc(pa + kk * 32, 16, 1024), tc_desc(vb + kk * 2048, kPfTok * 128, 1024), id_o,
-                           (part > 0 || kk > 0) ? 1u : 0u);
+                for (int part = 0; part < SM::kParts; ++part) {
+                    const uint32_t pa = smem_u32(psm + (X * SM::kParts + part) * SM::kP);
+#pragma unroll
+                    for (int kk = 0; kk < kPfTok / 16; ++kk)
+                        tc_mma(tmem + X * 256 + kPfTok, tc_desc(pa + kk * 32, 16, 1024),
+                               tc_desc(vb + kk * 2048, kPfTok * 128, 1024), id_o, (acc || part > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(bar(kBarO + X));
+            };
+            bool ok = mbar_wait(bar(kBarQ), 0, abort) && mbar_wait(bar(kBarKFull), 0, abort);
+            if (ok) {
+                tc_after_sync();
+                issue_s(0, 0);
+                if (nunits > 1) issue_s(1, 0);
+                tc_commit(bar(kBarKEmpty));
             }
-            tc_commit(smem_u32(&bars[1]));
+#pragma unroll 1
+            for (int kt = 0; ok && kt < nkv; ++kt) {
+                const int st = kt & 1;
+                const bool a1 = nunits > 1 && kt < U1.nkv, a1n = nunits > 1 && kt + 1 < U1.nkv;
+                ok = mbar_wait(bar(kBarVFull + st), (kt >> 1) & 1, abort) &&
+                     (kt != nkv - 1 || !need_fix || mbar_wait(bar(kBarVFix), 0, abort)) &&
+                     mbar_wait(bar(kBarP), kt & 1, abort);
+                if (!ok) break;
+                tc_after_sync();
+                issue_pv(0, st, kt > 0);
+                if (!a1) tc_commit(bar(kBarVEmpty + st));
+                if (kt + 1 < nkv) {
+                    ok = mbar_wait(bar(kBarKFull + (st ^ 1)), ((kt + 1) >> 1) & 1, abort);
+                    if (!ok) break;
+                    tc_after_sync();
+                    issue_s(0, st ^ 1);
+                    if (!a1n) tc_commit(bar(kBarKEmpty + (st ^ 1)));
+                }
+                if (a1) {
+                    ok = mbar_wait(bar(kBarP + 1), kt & 1, abort);
+                    if (!ok) break;
+                    tc_after_sync();
+                    issue_pv(1, st, kt > 0);
+                    tc_commit(bar(kBarVEmpty + st));
+                    if (a1n) {
+                        issue_s(1, st ^ 1);
+                        tc_commit(bar(kBarKEmpty + (st ^ 1)));
+                    }
+                }
+            }
+            tc_commit(bar(kBarDrain));  // every product issued has finished before tensor memory is freed
+            mbar_wait(bar(kBarDrain), 0, nullptr);
         }
-        timed_out |= !tc_wait(smem_u32(&bars[1]), kt & 1);
-        tc_after_sync();
+        __syncwarp();
+    } else if (warp == kPfLoadWarp) {
+        // ================= TMA copies (one lane), then the V tail fix (the warp)
+        bool ok = true;
+        if (lane == 0) {
+            int nk[2] = {0, 0}, nv[2] = {0, 0};
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
+            mbar_expect_tx(bar(kBarQ), (uint32_t)(nunits * SM::kQ));
+#pragma unroll 1
+            for (int X = 0; X < nunits; ++X) {
+                const PfUnit& W = X ? U1 : U0;
 #pragma unroll
-        for (int c0 = 0; c0 < DH; c0 += 16) {
-            float ov[16];
-            tc_ld16(tO + lane_addr + half * DH + c0, ov);
+                for (int cb = 0; cb < D / 64; ++cb)
+                    tma_load3(smem_u32(qsm + X * SM::kQ + cb * kPfRows * 128), &tmap_q, cb * 64, kh * p.g,
+                              q0 + W.tok0, bar(kBarQ));
+            }
+            const int32_t* trow = p.tables + (int64_t)s * p.mbps;
+            const int lg_bs = p.bs == 16 ? 4 : 5;
+            const int nblk = kPfTok >> lg_bs;
+#pragma unroll 1
+            for (int kt = 0; kt < nkv; ++kt) {
+                const int st = kt & 1;
+                int phys[kPfTok / 16];
+                int nb = 0;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) o[c0 + e] = o[c0 + e] * alpha + ov[e];
+                for (int jb = 0; jb < kPfTok / 16; ++jb) {
+                    const int t = kt * kPfTok + (jb << lg_bs);
+                    phys[jb] = 0;
+                    if (jb < nblk && t < U0.kv_end) {
+                        int ph = __ldg(trow + (t >> lg_bs));
+                        if (ph < 0 || ph >= p.num_blocks) {
+                            raise_error(p.err, PKV_DEVERR_BLOCK_ID);
+                            ph = 0;
+                        }
+                        phys[jb] = ph;
+                        ++nb;
+                    }
+                }
+                const uint32_t bytes = (uint32_t)(nb * p.bs * D * 2);
+                if (kt >= 2 && !(ok = mbar_wait(bar(kBarKEmpty + st), ((kt - 2) >> 1) & 1, abort))) break;
+                mbar_expect_tx(bar(kBarKFull + st), bytes);
+#pragma unroll 1
+                for (int jb = 0; jb < nb; ++jb)
+#pragma unroll
+                    for (int cb = 0; cb < D / 64; ++cb)
+                        tma_load3(smem_u32(ksm + st * SM::kTile + cb * kPfTok * 128 + jb * p.bs * 128), &tmap_k,
+                                  cb * 64, kh, phys[jb] * p.bs, bar(kBarKFull + st));
+                ++nk[st];
+                if (kt >= 2 && !(ok = mbar_wait(bar(kBarVEmpty + st), ((kt - 2) >> 1) & 1, abort))) break;
+                mbar_expect_tx(bar(kBarVFull + st), bytes);
+#pragma unroll 1
+                for (int jb = 0; jb < nb; ++jb)
+#pragma unroll
+                    for (int cb = 0; cb < D / 64; ++cb)
+                        tma_load3(smem_u32(vsm + st * SM::kTile + cb * kPfTok * 128 + jb * p.bs * 128), &tmap_v,
+                                  cb * 64, kh, phys[jb] * p.bs, bar(kBarVFull + st));
+                ++nv[st];
+            }
+            if (!ok) {  // let the copies in flight land before the CTA ends
+                mbar_wait(bar(kBarQ), 0, nullptr);
+                for (int st = 0; st < 2; ++st) {
+                    if (nk[st]) mbar_wait(bar(kBarKFull + st), (nk[st] - 1) & 1, nullptr);
+                    if (nv[st]) mbar_wait(bar(kBarVFull + st), (nv[st] - 1) & 1, nullptr);
+                }
+            }
         }
-        tc_before_sync();
-        if (__syncthreads_or(timed_out)) {
-            timed_out = true;
-            break;
+        __syncwarp();
+        ok = __shfl_sync(kFull, ok, 0);
+        if (need_fix) {  // zero the last V tile's rows at and past the unit's end
+            const int kl = nkv - 1, st = kl & 1;
+            bool fine = ok && mbar_wait(bar(kBarVFull + st), (kl >> 1) & 1, abort);
+            fine = __all_sync(kFull, fine);
+            if (fine) {
+                const int r0 = U0.kv_end - kl * kPfTok;
+                uint8_t* vt = vsm + st * SM::kTile;
+                for (int i = lane; i < (kPfTok - r0) * CH; i += 32)
+                    *reinterpret_cast<uint4*>(vt + tc_off(r0 + i / CH, i % CH, kPfTok)) = make_uint4(0, 0, 0, 0);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarVFix));
+            }
         }
     }
-    pf_wait<0>();
 
-    // ---- normalise (the two halves' sums combined) and store this half of the row
-    xmax[half][row] = l;
-    __syncthreads();
-    const float lt = xmax[0][row] + xmax[1][row];
-    if (timed_out) {
-        if (tid == 0) raise_error(p.err, PKV_DEVERR_TIMEOUT);
-    } else if (pos >= 0) {
-        const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        T* out = static_cast<T*>(p.out) +
-                 ((int64_t)(q0 + tok0 + row / p.g) * p.num_heads + (int64_t)kh * p.g + row % p.g) * D + half * DH;
-#pragma unroll
-        for (int c8 = 0; c8 < DH / 8; ++c8) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) w[e] = pack2<kBf16>(o[c8 * 8 + 2 * e] * inv, o[c8 * 8 + 2 * e + 1] * inv);
-            *reinterpret_cast<uint4*>(out + c8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-    }
     tc_before_sync();
     __syncthreads();
-    if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(SM::kTmemCols));
+    if (warp == kPfMmaWarp) {
+        tc_after_sync();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPfTmemCols));
+    }
+    if (tid == 0 && abort_flag) raise_error(p.err, PKV_DEVERR_TIMEOUT);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on the driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }();
+    return fn;
+}
+
+// A 3-D map over a 16-bit [d2][d1][d0] array (d0 contiguous), boxes of
+// {64, b1, b2} elements written with the 128-byte swizzle.
+pkv_status encode_map(CUtensorMap* m, bool bf16, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                      uint32_t b1, uint32_t b2) {
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return fail(PKV_ECUDA, "cuTensorMapEncodeTiled unavailable");
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    const cuuint32_t box[3] = {64, b1, b2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                           const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PKV_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return PKV_OK;
 }
 
 template <typename T, int D>
-pkv_status launch_prefill(const PrefillParams& p, int64_t grid, cudaStream_t st) {
+pkv_status launch_prefill(const PrefillParams& p, const void* query, const void* kc, const void* vc,
+                          int64_t num_tokens, int64_t num_blocks, int64_t grid, cudaStream_t st) {
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr int kSmem = PfSmem<T, D>::kBytes;
+    static_assert(kSmem <= 227 * 1024 - 8 * 1024, "prefill shared memory");
+    CUtensorMap tq, tk, tv;
+    pkv_status r = encode_map(&tq, kBf16, query, D, p.num_heads, num_tokens, p.g, kPfRows / p.g);
+    if (r == PKV_OK) r = encode_map(&tk, kBf16, kc, D, p.num_kv_heads, num_blocks * p.bs, 1, p.bs);
+    if (r == PKV_OK) r = encode_map(&tv, kBf16, vc, D, p.num_kv_heads, num_blocks * p.bs, 1, p.bs);
+    if (r != PKV_OK) return r;
     static std::atomic<unsigned long long> configured{0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(PKV_ECUDA, "cudaGetDevice");
@@ -435,7 +657,7 @@ pkv_status launch_prefill(const PrefillParams& p, int64_t grid, cudaStream_t st)
         if (e != cudaSuccess) return fail(PKV_ECUDA, "prefill smem opt-in: %s", cudaGetErrorString(e));
         configured.fetch_or(bit);
     }
-    pkv_prefill_kernel<T, D><<<(unsigned)grid, kPfThreads, kSmem, st>>>(p);
+    pkv_prefill_kernel<T, D><<<(unsigned)grid, kPfThreads, kSmem, st>>>(p, tq, tk, tv);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "prefill launch: %s", cudaGetErrorString(e));
     return PKV_OK;
@@ -474,9 +696,6 @@ extern "C" pkv_status pkv_paged_prefill(void* out, const void* query, pkv_dtype 
     if (!err) return fail(PKV_ECUDA, "device error word unavailable");
     PrefillParams p{};
     p.out = out;
-    p.q = query;
-    p.kc = static_cast<const uint8_t*>(key_cache);
-    p.vc = static_cast<const uint8_t*>(value_cache);
     p.tables = block_tables;
     p.seq_lens = seq_lens;
     p.qstart = query_start;
@@ -489,13 +708,20 @@ extern "C" pkv_status pkv_paged_prefill(void* out, const void* query, pkv_dtype 
     p.mbps = max_blocks_per_seq;
     p.bs = block_size;
     p.scale_log2 = scale * 1.4426950408889634f;
-    // row tiles: sum_s ceil(C_s g / 64) <= ceil(T g / 64) + S
-    const int64_t units = (num_query_tokens * g + kPfRows - 1) / kPfRows + num_seqs;
-    const int64_t grid = units * num_kv_heads;
+    // unit pairs: sum_s ceil(ceil(C_s g / 128) / 2) <= ceil(T g / 256) + S
+    const int64_t pairs = (num_query_tokens * g + 2 * kPfRows - 1) / (2 * kPfRows) + num_seqs;
+    const int64_t grid = pairs * num_kv_heads;
     if (grid > 0x7fffffffLL) return fail(PKV_EUNSUPPORTED, "too many query rows");
+    // TMA coordinates are 32-bit: token rows of the query and of the pool
+    if (num_query_tokens > 0x7fffffffLL || num_blocks * block_size > 0x7fffffffLL)
+        return fail(PKV_EUNSUPPORTED, "query or pool too large for 32-bit copy coordinates");
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t T = num_query_tokens;
     if (cache_dtype == PKV_F16)
-        return head_dim == 64 ? launch_prefill<__half, 64>(p, grid, cs) : launch_prefill<__half, 128>(p, grid, cs);
-    return head_dim == 64 ? launch_prefill<__nv_bfloat16, 64>(p, grid, cs)
-                          : launch_prefill<__nv_bfloat16, 128>(p, grid, cs);
+        return head_dim == 64
+                   ? launch_prefill<__half, 64>(p, query, key_cache, value_cache, T, num_blocks, grid, cs)
+                   : launch_prefill<__half, 128>(p, query, key_cache, value_cache, T, num_blocks, grid, cs);
+    return head_dim == 64
+               ? launch_prefill<__nv_bfloat16, 64>(p, query, key_cache, value_cache, T, num_blocks, grid, cs)
+               : launch_prefill<__nv_bfloat16, 128>(p, query, key_cache, value_cache, T, num_blocks, grid, cs);
 }
