@@ -22,6 +22,10 @@
 //     write P to shared memory (bf16 as hi + lo parts, so P V keeps
 //     fp32-level accuracy).  O stays in tensor memory across tiles; it is
 //     rescaled only when a row's maximum passes its reference by 2^8.
+// A unit without a partner (a decode row, the first row tile of a sequence
+// with an odd count) splits its tiles instead: group 0 takes the even tiles,
+// group 1 the odd ones, and group 0 merges the two partial (max, sum, O)
+// results at the end.
 // Every hand-off is an mbarrier; every wait is bounded (0.2 s of
 // %globaltimer): a timeout sets PKV_DEVERR_TIMEOUT, every role leaves its
 // loop, the copies and products already issued are drained, and the CTA
@@ -153,6 +157,14 @@ __device__ __forceinline__ bool group_sync_or(int id, bool flag) {
                  : "=r"(r) : "r"((uint32_t)flag), "r"(id), "n"(kPfGroup) : "memory");
     return r != 0;
 }
+// The same over both softmax groups (barrier 3, 2 kPfGroup threads).
+__device__ __forceinline__ bool pair_sync_or(bool flag) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 3, %2, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}\n"
+                 : "=r"(r) : "r"((uint32_t)flag), "n"(2 * kPfGroup) : "memory");
+    return r != 0;
+}
 // 3-D TMA tile load into shared memory, completing on an mbarrier.
 __device__ __forceinline__ void tma_load3(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
                                           uint32_t mbar) {
@@ -239,7 +251,8 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     __shared__ float xmax[2][2][2][kPfRows];    // [unit][tile parity][half][row] partial row maxima
-    __shared__ float xsum[2][2][kPfRows];       // [unit][half][row] partial row sums
+    __shared__ float xsum[2][2][kPfRows];       // [group][half][row] partial row sums
+    __shared__ float xref[kPfRows];             // group 1's reference maxima (split unit)
     volatile int* abort = &abort_flag;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -303,6 +316,9 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     const PfUnit U0 = make_unit(j0);                 // the later rows: the longer K/V range
     const PfUnit U1 = make_unit(j1 >= 0 ? j1 : j0);  // (unused when nunits == 1)
     const int nkv = U0.nkv;
+    // a unit alone splits its K/V tiles between the two groups (even / odd
+    // tiles), whose partial results are merged at the end
+    const bool split = nunits == 1;
     const bool need_fix = (U0.kv_end % kPfTok) != 0;  // V rows past the end must read as zeros
 
     // ---- tensor memory, barriers
@@ -321,10 +337,13 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     const uint32_t tmem = tmem_base;
 
     if (warp < 2 * (kPfGroup / 32)) {
-        // ================= softmax groups: unit X, two threads per row
+        // ================= softmax group X: unit X (or, for a unit alone,
+        // its tiles of stage X), two threads per row
         const int X = warp >> 3;
-        if (X < nunits) {
-            const PfUnit U = X ? U1 : U0;
+        {
+            const PfUnit U = X && !split ? U1 : U0;
+            const int kt0 = split ? X : 0, kstep = split ? 2 : 1;  // this group's tiles
+            const int ntiles = split ? (nkv - X + 1) / 2 : U.nkv;
             const int wq = warp & 3, half = (warp >> 2) & 1;
             const int row = wq * 32 + lane;
             const int pos = (row / p.g < U.ntok) ? U.pos0 + row / p.g : -1;
@@ -336,8 +355,9 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
             float mref = -INFINITY, l = 0.f;  // reference maximum (log2 domain) and this half's sum
             bool failed = false;
 #pragma unroll 1
-            for (int kt = 0; kt < U.nkv; ++kt) {
-                bool ok = !failed && mbar_wait(bar(kBarS + X), kt & 1, abort);
+            for (int i = 0; i < ntiles; ++i) {
+                const int kt = kt0 + i * kstep;
+                bool ok = !failed && mbar_wait(bar(kBarS + X), i & 1, abort);
                 ok = __all_sync(kFull, ok);
                 float sc[kPfTok / 2];
                 float pm = -INFINITY;
@@ -354,13 +374,13 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                     for (int c = 0; c < kPfTok / 2; ++c) m4[c & 3] = fmaxf(m4[c & 3], sc[c]);
                     pm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
                 }
-                xmax[X][kt & 1][half][row] = pm;
+                xmax[X][i & 1][half][row] = pm;
                 if (group_sync_or(1 + X, !ok)) {
                     failed = true;
                     break;
                 }
                 // the row maximum of this tile (both halves), in the log2 domain
-                const float mx = fmaxf(xmax[X][kt & 1][0][row], xmax[X][kt & 1][1][row]) * sl2;
+                const float mx = fmaxf(xmax[X][i & 1][0][row], xmax[X][i & 1][1][row]) * sl2;
                 const bool grow = mx > mref + 8.f;  // also the first finite maximum
                 float alpha = 1.f;
                 if (grow) {
@@ -376,8 +396,8 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                     ls4[c & 3] += sc[c];
                 }
                 l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
-                if (kt > 0) {  // P V of the previous tile done: its P buffer is free, O is settled
-                    ok = mbar_wait(bar(kBarO + X), (kt - 1) & 1, abort);
+                if (i > 0) {  // P V of the previous tile done: its P buffer is free, O is settled
+                    ok = mbar_wait(bar(kBarO + X), (i - 1) & 1, abort);
                     ok = __all_sync(kFull, ok);
                     if (ok) {
                         tc_after_sync();
@@ -419,14 +439,30 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                 tc_before_sync();
                 mbar_arrive(bar(kBarP + X));
             }
-            // ---- the last P V, then normalise (the halves' sums combined) and store
-            bool ok = !failed && mbar_wait(bar(kBarO + X), (U.nkv - 1) & 1, abort);
+            // ---- the last P V, then normalise (the halves' sums combined; a
+            // split unit also merges group 1's partial result) and store
+            bool ok = !failed && (ntiles == 0 || mbar_wait(bar(kBarO + X), (ntiles - 1) & 1, abort));
+            // (group 1's last P V, read in the merge: after group 0's own last
+            // one, at most that phase of group 1 is outstanding)
+            if (split && X == 0 && nkv > 1) ok = ok && mbar_wait(bar(kBarO + 1), ((nkv >> 1) - 1) & 1, abort);
             ok = __all_sync(kFull, ok);
             xsum[X][half][row] = l;
-            if (!group_sync_or(1 + X, !ok)) {
+            if (split && X == 1 && half == 0) xref[row] = mref;
+            const bool bad = split ? pair_sync_or(!ok) : group_sync_or(1 + X, !ok);
+            if (!bad && !(split && X == 1)) {
                 tc_after_sync();
-                const float lt = xsum[X][0][row] + xsum[X][1][row];
+                float lt = xsum[X][0][row] + xsum[X][1][row];
+                float a0 = 1.f, a1 = 0.f;
+                const bool merge = split && nkv > 1;
+                if (merge) {
+                    const float m1 = xref[row], m = fmaxf(mref, m1);
+                    a0 = mref == -INFINITY ? 0.f : ex2(mref - m);
+                    a1 = m1 == -INFINITY ? 0.f : ex2(m1 - m);
+                    lt = a0 * lt + a1 * (xsum[1][0][row] + xsum[1][1][row]);
+                }
                 const float inv = lt > 0.f ? 1.f / lt : 0.f;
+                a0 *= inv;
+                a1 *= inv;
                 T* out = static_cast<T*>(p.out) +
                          ((int64_t)(q0 + U.tok0 + row / p.g) * p.num_heads + (int64_t)kh * p.g + row % p.g) * D +
                          half * (D / 2);
@@ -434,9 +470,18 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                 for (int c0 = 0; c0 < D / 2; c0 += 16) {
                     float v[16];
                     tc_ld16(tO + c0, v);  // every lane loads (warp-collective); only real rows store
+                    if (merge) {
+                        float v1[16];
+                        tc_ld16(tO + 256 + c0, v1);  // group 1's O: same lanes, the next 256 columns
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] = a0 * v[e] + a1 * v1[e];
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] *= a0;
+                    }
                     uint32_t w[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) w[e] = pack2<kBf16>(v[2 * e] * inv, v[2 * e + 1] * inv);
+                    for (int e = 0; e < 8; ++e) w[e] = pack2<kBf16>(v[2 * e], v[2 * e + 1]);
                     if (pos >= 0) {
                         *reinterpret_cast<uint4*>(out + c0) = make_uint4(w[0], w[1], w[2], w[3]);
                         *reinterpret_cast<uint4*>(out + c0 + 8) = make_uint4(w[4], w[5], w[6], w[7]);
@@ -449,8 +494,8 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         if (lane == 0) {
             const uint32_t id_s = tc_idesc<kBf16>(kPfRows, kPfTok, 0);
             const uint32_t id_o = tc_idesc<kBf16>(kPfRows, D, 1);
-            auto issue_s = [&](int X, int st) {  // S_X = Q_X K^T
-                const uint32_t qa = smem_u32(qsm + X * SM::kQ), kb = smem_u32(ksm + st * SM::kTile);
+            auto issue_s = [&](int X, int st) {  // S_X = Q_X K^T (a split unit: both groups read q slot 0)
+                const uint32_t qa = smem_u32(qsm + (split ? 0 : X) * SM::kQ), kb = smem_u32(ksm + st * SM::kTile);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     tc_mma(tmem + X * 256, tc_desc(qa + (kk >> 2) * kPfRows * 128 + (kk & 3) * 32, 16, 1024),
@@ -469,40 +514,79 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                 }
                 tc_commit(bar(kBarO + X));
             };
-            bool ok = mbar_wait(bar(kBarQ), 0, abort) && mbar_wait(bar(kBarKFull), 0, abort);
-            if (ok) {
-                tc_after_sync();
-                issue_s(0, 0);
-                if (nunits > 1) issue_s(1, 0);
-                tc_commit(bar(kBarKEmpty));
-            }
-#pragma unroll 1
-            for (int kt = 0; ok && kt < nkv; ++kt) {
-                const int st = kt & 1;
-                const bool a1 = nunits > 1 && kt < U1.nkv, a1n = nunits > 1 && kt + 1 < U1.nkv;
-                ok = mbar_wait(bar(kBarVFull + st), (kt >> 1) & 1, abort) &&
-                     (kt != nkv - 1 || !need_fix || mbar_wait(bar(kBarVFix), 0, abort)) &&
-                     mbar_wait(bar(kBarP), kt & 1, abort);
-                if (!ok) break;
-                tc_after_sync();
-                issue_pv(0, st, kt > 0);
-                if (!a1) tc_commit(bar(kBarVEmpty + st));
-                if (kt + 1 < nkv) {
-                    ok = mbar_wait(bar(kBarKFull + (st ^ 1)), ((kt + 1) >> 1) & 1, abort);
-                    if (!ok) break;
+            bool ok = mbar_wait(bar(kBarQ), 0, abort);
+            if (!split) {
+                // paired units: every tile serves both; per tile
+                // O_0 += P_0 V, S_0' = Q_0 K'^T, O_1 += P_1 V, S_1' = Q_1 K'^T
+                ok = ok && mbar_wait(bar(kBarKFull), 0, abort);
+                if (ok) {
                     tc_after_sync();
-                    issue_s(0, st ^ 1);
-                    if (!a1n) tc_commit(bar(kBarKEmpty + (st ^ 1)));
+                    issue_s(0, 0);
+                    issue_s(1, 0);
+                    tc_commit(bar(kBarKEmpty));
                 }
-                if (a1) {
-                    ok = mbar_wait(bar(kBarP + 1), kt & 1, abort);
+#pragma unroll 1
+                for (int kt = 0; ok && kt < nkv; ++kt) {
+                    const int st = kt & 1;
+                    const bool a1 = kt < U1.nkv, a1n = kt + 1 < U1.nkv;
+                    ok = mbar_wait(bar(kBarVFull + st), (kt >> 1) & 1, abort) &&
+                         (kt != nkv - 1 || !need_fix || mbar_wait(bar(kBarVFix), 0, abort)) &&
+                         mbar_wait(bar(kBarP), kt & 1, abort);
                     if (!ok) break;
                     tc_after_sync();
-                    issue_pv(1, st, kt > 0);
-                    tc_commit(bar(kBarVEmpty + st));
-                    if (a1n) {
-                        issue_s(1, st ^ 1);
-                        tc_commit(bar(kBarKEmpty + (st ^ 1)));
+                    issue_pv(0, st, kt > 0);
+                    if (!a1) tc_commit(bar(kBarVEmpty + st));
+                    if (kt + 1 < nkv) {
+                        ok = mbar_wait(bar(kBarKFull + (st ^ 1)), ((kt + 1) >> 1) & 1, abort);
+                        if (!ok) break;
+                        tc_after_sync();
+                        issue_s(0, st ^ 1);
+                        if (!a1n) tc_commit(bar(kBarKEmpty + (st ^ 1)));
+                    }
+                    if (a1) {
+                        ok = mbar_wait(bar(kBarP + 1), kt & 1, abort);
+                        if (!ok) break;
+                        tc_after_sync();
+                        issue_pv(1, st, kt > 0);
+                        tc_commit(bar(kBarVEmpty + st));
+                        if (a1n) {
+                            issue_s(1, st ^ 1);
+                            tc_commit(bar(kBarKEmpty + (st ^ 1)));
+                        }
+                    }
+                }
+            } else {
+                // a split unit: group X takes the tiles of stage X (tile
+                // 2 i + X); per step i: O_0 += P_0 V_2i, S_0 = Q K_2i+2^T,
+                // O_1 += P_1 V_2i+1, S_1 = Q K_2i+3^T
+#pragma unroll 1
+                for (int X = 0; ok && X < 2 && X < nkv; ++X) {
+                    ok = mbar_wait(bar(kBarKFull + X), 0, abort);
+                    if (!ok) break;
+                    tc_after_sync();
+                    issue_s(X, X);
+                    tc_commit(bar(kBarKEmpty + X));
+                }
+#pragma unroll 1
+                for (int i = 0; ok && 2 * i < nkv; ++i) {
+#pragma unroll 1
+                    for (int X = 0; X < 2; ++X) {
+                        const int kt = 2 * i + X;
+                        if (kt >= nkv) break;
+                        ok = mbar_wait(bar(kBarVFull + X), i & 1, abort) &&
+                             (kt != nkv - 1 || !need_fix || mbar_wait(bar(kBarVFix), 0, abort)) &&
+                             mbar_wait(bar(kBarP + X), i & 1, abort);
+                        if (!ok) break;
+                        tc_after_sync();
+                        issue_pv(X, X, i > 0);
+                        tc_commit(bar(kBarVEmpty + X));
+                        if (kt + 2 < nkv) {
+                            ok = mbar_wait(bar(kBarKFull + X), (i + 1) & 1, abort);
+                            if (!ok) break;
+                            tc_after_sync();
+                            issue_s(X, X);
+                            tc_commit(bar(kBarKEmpty + X));
+                        }
                     }
                 }
             }
