@@ -12,15 +12,15 @@
 // one unit while the other runs its softmax:
 //   - warp 17 (one lane) copies the units' q rows and then, through the
 //     block table, each 64-token K and V tile with TMA into the 128-byte
-//     swizzled layout the tensor core reads (2-stage K and V rings);
+//     swizzled layout the tensor core reads (3-stage K and V rings);
 //   - warp 16 (one lane) owns tensor memory and issues, per tile,
 //     O_0 += P_0 V, S_0' = Q_0 K'^T, O_1 += P_1 V, S_1' = Q_1 K'^T
 //     (tcgen05.mma, M = 128 rows, fp32 accumulators in tensor memory);
 //   - warps 0-7 and 8-15 are the two units' softmax groups, two threads per
 //     row (one per half of the 64 scores and of the head_dim outputs): load
 //     S from tensor memory, mask, exponentiate against a reference maximum,
-//     write P to shared memory (bf16 as hi + lo parts, so P V keeps
-//     fp32-level accuracy).  O stays in tensor memory across tiles; it is
+//     write P back to tensor memory, where the P V product reads it as its
+//     A operand (bf16 as hi + lo parts, so P V keeps fp32-level accuracy).  O stays in tensor memory across tiles; it is
 //     rescaled only when a row's maximum passes its reference by 2^8.
 // A unit without a partner (a decode row, the first row tile of a sequence
 // with an odd count) splits its tiles instead: group 0 takes the even tiles,
@@ -50,22 +50,24 @@ constexpr int kPfGroup = 256;       // softmax threads per unit: two per row
 constexpr int kPfMmaWarp = 16;      // issues the tensor-core products, owns tensor memory
 constexpr int kPfLoadWarp = 17;     // issues the TMA copies
 constexpr int kPfThreads = 18 * 32;
-constexpr int kPfTmemCols = 512;    // unit u: S in columns [256 u, 256 u + 64), O from 256 u + 64
+constexpr int kPfStages = 3;        // K and V ring depth
+constexpr int kPfTmemCols = 512;    // unit u: S in columns 256 u + [0, 64), O from 256 u + 64,
+constexpr int kPfTmemP = 192;       //   P (hi, lo: 32 columns each) from 256 u + 192
 constexpr uint64_t kPfWaitNs = 200000000ull;
 
 // mbarriers
 enum : int {
-    kBarQ = 0,        // q rows landed (TMA transaction count)
-    kBarKFull = 1,    // [2] K tile landed
-    kBarVFull = 3,    // [2] V tile landed
-    kBarKEmpty = 5,   // [2] every S product of the K stage finished
-    kBarVEmpty = 7,   // [2] every P V product of the V stage finished
-    kBarVFix = 9,     // the last V tile's rows past the unit's end are zeroed
-    kBarS = 10,       // [2] S of unit u ready
-    kBarP = 12,       // [2] P of unit u written (and S read): kPfGroup arrivals
-    kBarO = 14,       // [2] P V of unit u finished
-    kBarDrain = 16,   // products drained (abort path)
-    kNumBars = 17
+    kBarQ = 0,                             // q rows landed (TMA transaction count)
+    kBarKFull = 1,                         // [stage] K tile landed
+    kBarVFull = kBarKFull + kPfStages,     // [stage] V tile landed
+    kBarKEmpty = kBarVFull + kPfStages,    // [stage] every S product of the K stage finished
+    kBarVEmpty = kBarKEmpty + kPfStages,   // [stage] every P V product of the V stage finished
+    kBarVFix = kBarVEmpty + kPfStages,     // the last V tile's rows past the unit's end are zeroed
+    kBarS = kBarVFix + 1,                  // [unit] S ready
+    kBarP = kBarS + 2,                     // [unit] P written (and S read): kPfGroup arrivals
+    kBarO = kBarP + 2,                     // [unit] P V finished
+    kBarDrain = kBarO + 2,                 // products drained (abort path)
+    kNumBars = kBarDrain + 1
 };
 
 struct PrefillParams {
@@ -95,6 +97,12 @@ __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, uint32_t lbo, uint32
     return (uint64_t)((saddr & 0x3FFFF) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
+// A descriptor whose start address is `c` 16-byte units further on (the
+// start field is the low 14 bits and shared-memory addresses stay below
+// 256 KB, so the add never carries out of it).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t c) {
+    return (d & 0xFFFFFFFF00000000ull) | (uint64_t)((uint32_t)d + c);
+}
 // Instruction descriptor of kind::f16 with an fp32 accumulator.
 template <bool kBf16>
 __device__ __forceinline__ uint32_t tc_idesc(int M, int N, int b_mn_major) {
@@ -107,6 +115,14 @@ __device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t a, uint64_t b, 
     asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
                  "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}\n"
                  ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(z));
+}
+// The same with A (P) read from tensor memory.
+__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc,
+                                          uint32_t acc) {
+    const uint32_t z = 0;
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}\n"
+                 ::"r"(tmem_d), "r"(tmem_a), "l"(b), "r"(idesc), "r"(acc), "r"(z));
 }
 __device__ __forceinline__ void tc_commit(uint32_t mbar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
@@ -214,6 +230,15 @@ __device__ __forceinline__ void tc_st16(uint32_t taddr, const float* v) {
                    "r"(__float_as_uint(v[15]))
                  : "memory");
 }
+// 16 32-bit columns into this thread's lane (asynchronous: tc_wait_st).
+__device__ __forceinline__ void tc_st16u(uint32_t taddr, const uint32_t* w) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+                 ::"r"(taddr), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]),
+                   "r"(w[7]), "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]),
+                   "r"(w[15])
+                 : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -222,9 +247,8 @@ template <typename T, int D>
 struct PfSmem {
     static constexpr int kQ = kPfRows * D * 2;     // one unit's q rows
     static constexpr int kTile = kPfTok * D * 2;   // one K or V tile
-    static constexpr int kP = kPfRows * kPfTok * 2;
     static constexpr int kParts = std::is_same<T, __nv_bfloat16>::value ? 2 : 1;  // P hi (+ lo)
-    static constexpr int kData = 2 * kQ + 4 * kTile + 2 * kParts * kP + 1024;     // + alignment
+    static constexpr int kData = 2 * kQ + 2 * kPfStages * kTile + 1024;           // + alignment
     // at least 120 KB, so one CTA (and its 512 tensor-memory columns) per SM
     static constexpr int kBytes = kData > 120 * 1024 ? kData : 120 * 1024;
 };
@@ -244,9 +268,8 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     extern __shared__ uint8_t pf_raw[];
     uint8_t* sm = pf_raw + ((1024 - (smem_u32(pf_raw) & 1023)) & 1023);  // 1024-byte aligned operands
     uint8_t* qsm = sm;                          // [2 units]
-    uint8_t* ksm = qsm + 2 * SM::kQ;            // [2 stages]
-    uint8_t* vsm = ksm + 2 * SM::kTile;         // [2 stages]
-    uint8_t* psm = vsm + 2 * SM::kTile;         // [2 units][hi, lo]
+    uint8_t* ksm = qsm + 2 * SM::kQ;            // [stage]
+    uint8_t* vsm = ksm + kPfStages * SM::kTile; // [stage]
     __shared__ __align__(8) uint64_t bars[kNumBars];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
@@ -256,6 +279,10 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     volatile int* abort = &abort_flag;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
+    // K/V tile kt sits in ring stage kt % kPfStages; its full / empty
+    // barriers complete once per pass of the ring
+    auto stg = [](int kt) { return kt % kPfStages; };
+    auto pass = [](int kt) { return (uint32_t)((kt / kPfStages) & 1); };
 
     // ---- the unit pair: kv head from the block index, then pair u among all
     // sequences' pairs (warp-parallel scan; every warp finds it).  A
@@ -350,7 +377,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
             const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
             const uint32_t tS = tmem + lane_addr + X * 256 + half * (kPfTok / 2);
             const uint32_t tO = tmem + lane_addr + X * 256 + kPfTok + half * (D / 2);
-            uint8_t* pu = psm + X * SM::kParts * SM::kP;
+            const uint32_t tP = tmem + lane_addr + X * 256 + kPfTmemP + half * (kPfTok / 4);
             const float sl2 = p.scale_log2;
             float mref = -INFINITY, l = 0.f;  // reference maximum (log2 domain) and this half's sum
             bool failed = false;
@@ -417,25 +444,23 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                     failed = true;
                     continue;  // the next tile's group barrier ends the loop for the whole group
                 }
-                // ---- this half of P (K-major rows; bf16 as hi + lo parts)
+                // ---- this half of P into tensor memory: row = lane, two
+                // tokens per 32-bit column (bf16 as hi + lo parts, 32 columns apart)
+                {
+                    uint32_t h[kPfTok / 4], lo[kPfTok / 4];
 #pragma unroll
-                for (int c8 = 0; c8 < kPfTok / 16; ++c8) {
-                    uint32_t h[4], lo[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float a = sc[c8 * 8 + 2 * e], b = sc[c8 * 8 + 2 * e + 1];
+                    for (int e = 0; e < kPfTok / 4; ++e) {
+                        const float a = sc[2 * e], b = sc[2 * e + 1];
                         h[e] = pack2<kBf16>(a, b);
                         if constexpr (kBf16) {
                             const float2 hf = unpack2<true>(h[e]);
                             lo[e] = pack2<true>(a - hf.x, b - hf.y);
                         }
                     }
-                    const uint32_t off = tc_off(row, half * (kPfTok / 16) + c8, kPfRows);
-                    *reinterpret_cast<uint4*>(pu + off) = make_uint4(h[0], h[1], h[2], h[3]);
-                    if constexpr (kBf16)
-                        *reinterpret_cast<uint4*>(pu + SM::kP + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    tc_st16u(tP, h);
+                    if constexpr (kBf16) tc_st16u(tP + kPfTok / 2, lo);
+                    tc_wait_st();
                 }
-                fence_async_smem();
                 tc_before_sync();
                 mbar_arrive(bar(kBarP + X));
             }
@@ -494,24 +519,32 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         if (lane == 0) {
             const uint32_t id_s = tc_idesc<kBf16>(kPfRows, kPfTok, 0);
             const uint32_t id_o = tc_idesc<kBf16>(kPfRows, D, 1);
+            // operand descriptors built once; per product only a constant
+            // offset is added (the issue rate of this one thread bounds the
+            // tensor core otherwise)
+            const uint64_t dq0 = tc_desc(smem_u32(qsm), 16, 1024);
+            const uint64_t dq1 = tc_desc(smem_u32(qsm + (split ? 0 : SM::kQ)), 16, 1024);
+            const uint64_t dk0 = tc_desc(smem_u32(ksm), 16, 1024);
+            const uint64_t dv0 = tc_desc(smem_u32(vsm), kPfTok * 128, 1024);
             auto issue_s = [&](int X, int st) {  // S_X = Q_X K^T (a split unit: both groups read q slot 0)
-                const uint32_t qa = smem_u32(qsm + (split ? 0 : X) * SM::kQ), kb = smem_u32(ksm + st * SM::kTile);
+                const uint64_t qd = X ? dq1 : dq0;
+                const uint64_t kd = desc_add(dk0, (uint32_t)(st * (SM::kTile >> 4)));
+                const uint32_t d = tmem + X * 256;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc_mma(tmem + X * 256, tc_desc(qa + (kk >> 2) * kPfRows * 128 + (kk & 3) * 32, 16, 1024),
-                           tc_desc(kb + (kk >> 2) * kPfTok * 128 + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
+                    tc_mma(d, desc_add(qd, ((kk >> 2) * kPfRows * 128 + (kk & 3) * 32) >> 4),
+                           desc_add(kd, ((kk >> 2) * kPfTok * 128 + (kk & 3) * 32) >> 4), id_s, kk > 0);
                 tc_commit(bar(kBarS + X));
             };
-            auto issue_pv = [&](int X, int st, bool acc) {  // O_X (+)= P_X V (hi, then lo)
-                const uint32_t vb = smem_u32(vsm + st * SM::kTile);
+            auto issue_pv = [&](int X, int st, bool acc) {  // O_X (+)= P_X V (hi, then lo; P in tensor memory)
+                const uint64_t vd = desc_add(dv0, (uint32_t)(st * (SM::kTile >> 4)));
+                const uint32_t d = tmem + X * 256 + kPfTok, a = tmem + X * 256 + kPfTmemP;
 #pragma unroll
-                for (int part = 0; part < SM::kParts; ++part) {
-                    const uint32_t pa = smem_u32(psm + (X * SM::kParts + part) * SM::kP);
+                for (int part = 0; part < SM::kParts; ++part)
 #pragma unroll
                     for (int kk = 0; kk < kPfTok / 16; ++kk)
-                        tc_mma(tmem + X * 256 + kPfTok, tc_desc(pa + kk * 32, 16, 1024),
-                               tc_desc(vb + kk * 2048, kPfTok * 128, 1024), id_o, (acc || part > 0 || kk > 0) ? 1u : 0u);
-                }
+                        tc_mma_ts(d, a + part * (kPfTok / 2) + kk * 8, desc_add(vd, (kk * 2048) >> 4), id_o,
+                                  (acc || part > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(bar(kBarO + X));
             };
             bool ok = mbar_wait(bar(kBarQ), 0, abort);
@@ -527,9 +560,9 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                 }
 #pragma unroll 1
                 for (int kt = 0; ok && kt < nkv; ++kt) {
-                    const int st = kt & 1;
+                    const int st = stg(kt), sn = stg(kt + 1);
                     const bool a1 = kt < U1.nkv, a1n = kt + 1 < U1.nkv;
-                    ok = mbar_wait(bar(kBarVFull + st), (kt >> 1) & 1, abort) &&
+                    ok = mbar_wait(bar(kBarVFull + st), pass(kt), abort) &&
                          (kt != nkv - 1 || !need_fix || mbar_wait(bar(kBarVFix), 0, abort)) &&
                          mbar_wait(bar(kBarP), kt & 1, abort);
                     if (!ok) break;
@@ -537,11 +570,11 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                     issue_pv(0, st, kt > 0);
                     if (!a1) tc_commit(bar(kBarVEmpty + st));
                     if (kt + 1 < nkv) {
-                        ok = mbar_wait(bar(kBarKFull + (st ^ 1)), ((kt + 1) >> 1) & 1, abort);
+                        ok = mbar_wait(bar(kBarKFull + sn), pass(kt + 1), abort);
                         if (!ok) break;
                         tc_after_sync();
-                        issue_s(0, st ^ 1);
-                        if (!a1n) tc_commit(bar(kBarKEmpty + (st ^ 1)));
+                        issue_s(0, sn);
+                        if (!a1n) tc_commit(bar(kBarKEmpty + sn));
                     }
                     if (a1) {
                         ok = mbar_wait(bar(kBarP + 1), kt & 1, abort);
@@ -550,22 +583,21 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                         issue_pv(1, st, kt > 0);
                         tc_commit(bar(kBarVEmpty + st));
                         if (a1n) {
-                            issue_s(1, st ^ 1);
-                            tc_commit(bar(kBarKEmpty + (st ^ 1)));
+                            issue_s(1, sn);
+                            tc_commit(bar(kBarKEmpty + sn));
                         }
                     }
                 }
             } else {
-                // a split unit: group X takes the tiles of stage X (tile
-                // 2 i + X); per step i: O_0 += P_0 V_2i, S_0 = Q K_2i+2^T,
-                // O_1 += P_1 V_2i+1, S_1 = Q K_2i+3^T
+                // a split unit: group X takes tiles 2 i + X; per step i:
+                // O_0 += P_0 V_2i, S_0 = Q K_2i+2^T, O_1 += P_1 V_2i+1, S_1 = Q K_2i+3^T
 #pragma unroll 1
                 for (int X = 0; ok && X < 2 && X < nkv; ++X) {
-                    ok = mbar_wait(bar(kBarKFull + X), 0, abort);
+                    ok = mbar_wait(bar(kBarKFull + stg(X)), pass(X), abort);
                     if (!ok) break;
                     tc_after_sync();
-                    issue_s(X, X);
-                    tc_commit(bar(kBarKEmpty + X));
+                    issue_s(X, stg(X));
+                    tc_commit(bar(kBarKEmpty + stg(X)));
                 }
 #pragma unroll 1
                 for (int i = 0; ok && 2 * i < nkv; ++i) {
@@ -573,19 +605,19 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                     for (int X = 0; X < 2; ++X) {
                         const int kt = 2 * i + X;
                         if (kt >= nkv) break;
-                        ok = mbar_wait(bar(kBarVFull + X), i & 1, abort) &&
+                        ok = mbar_wait(bar(kBarVFull + stg(kt)), pass(kt), abort) &&
                              (kt != nkv - 1 || !need_fix || mbar_wait(bar(kBarVFix), 0, abort)) &&
                              mbar_wait(bar(kBarP + X), i & 1, abort);
                         if (!ok) break;
                         tc_after_sync();
-                        issue_pv(X, X, i > 0);
-                        tc_commit(bar(kBarVEmpty + X));
+                        issue_pv(X, stg(kt), i > 0);
+                        tc_commit(bar(kBarVEmpty + stg(kt)));
                         if (kt + 2 < nkv) {
-                            ok = mbar_wait(bar(kBarKFull + X), (i + 1) & 1, abort);
+                            ok = mbar_wait(bar(kBarKFull + stg(kt + 2)), pass(kt + 2), abort);
                             if (!ok) break;
                             tc_after_sync();
-                            issue_s(X, X);
-                            tc_commit(bar(kBarKEmpty + X));
+                            issue_s(X, stg(kt + 2));
+                            tc_commit(bar(kBarKEmpty + stg(kt + 2)));
                         }
                     }
                 }
@@ -598,7 +630,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         // ================= TMA copies (one lane), then the V tail fix (the warp)
         bool ok = true;
         if (lane == 0) {
-            int nk[2] = {0, 0}, nv[2] = {0, 0};
+            int nk[kPfStages] = {}, nv[kPfStages] = {};
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
             mbar_expect_tx(bar(kBarQ), (uint32_t)(nunits * SM::kQ));
@@ -615,7 +647,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
             const int nblk = kPfTok >> lg_bs;
 #pragma unroll 1
             for (int kt = 0; kt < nkv; ++kt) {
-                const int st = kt & 1;
+                const int st = stg(kt);
                 int phys[kPfTok / 16];
                 int nb = 0;
 #pragma unroll
@@ -633,7 +665,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                     }
                 }
                 const uint32_t bytes = (uint32_t)(nb * p.bs * D * 2);
-                if (kt >= 2 && !(ok = mbar_wait(bar(kBarKEmpty + st), ((kt - 2) >> 1) & 1, abort))) break;
+                if (kt >= kPfStages && !(ok = mbar_wait(bar(kBarKEmpty + st), pass(kt - kPfStages), abort))) break;
                 mbar_expect_tx(bar(kBarKFull + st), bytes);
 #pragma unroll 1
                 for (int jb = 0; jb < nb; ++jb)
@@ -642,7 +674,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                         tma_load3(smem_u32(ksm + st * SM::kTile + cb * kPfTok * 128 + jb * p.bs * 128), &tmap_k,
                                   cb * 64, kh, phys[jb] * p.bs, bar(kBarKFull + st));
                 ++nk[st];
-                if (kt >= 2 && !(ok = mbar_wait(bar(kBarVEmpty + st), ((kt - 2) >> 1) & 1, abort))) break;
+                if (kt >= kPfStages && !(ok = mbar_wait(bar(kBarVEmpty + st), pass(kt - kPfStages), abort))) break;
                 mbar_expect_tx(bar(kBarVFull + st), bytes);
 #pragma unroll 1
                 for (int jb = 0; jb < nb; ++jb)
@@ -654,7 +686,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
             }
             if (!ok) {  // let the copies in flight land before the CTA ends
                 mbar_wait(bar(kBarQ), 0, nullptr);
-                for (int st = 0; st < 2; ++st) {
+                for (int st = 0; st < kPfStages; ++st) {
                     if (nk[st]) mbar_wait(bar(kBarKFull + st), (nk[st] - 1) & 1, nullptr);
                     if (nv[st]) mbar_wait(bar(kBarVFull + st), (nv[st] - 1) & 1, nullptr);
                 }
@@ -663,8 +695,8 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         __syncwarp();
         ok = __shfl_sync(kFull, ok, 0);
         if (need_fix) {  // zero the last V tile's rows at and past the unit's end
-            const int kl = nkv - 1, st = kl & 1;
-            bool fine = ok && mbar_wait(bar(kBarVFull + st), (kl >> 1) & 1, abort);
+            const int kl = nkv - 1, st = stg(kl);
+            bool fine = ok && mbar_wait(bar(kBarVFull + st), pass(kl), abort);
             fine = __all_sync(kFull, fine);
             if (fine) {
                 const int r0 = U0.kv_end - kl * kPfTok;
