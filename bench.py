@@ -582,7 +582,7 @@ def run_prefill(args):
                    "flops": flops, "l2": "flushed between steps"},
         "prefill_ms": attn_ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "peak_kind": kind, "traffic": None},
+                     "frac": achieved / peak, "peak_kind": kind, "traffic": recorded_traffic(wl.name)},
         "clocks": clk.summary(), "gpu_launches": 2 * K, "e2e": None, "cpu_baseline": cpu,
     }
     print(json.dumps(line))
