@@ -281,9 +281,12 @@ pkv_status pkv_paged_attention_decode_cascade(void* out, const void* query, pkv_
  * head_dim in {64, 128}, block_size in {16, 32}, g in {1, 2, 4, 8, 16}
  * (otherwise PKV_EUNSUPPORTED).  A seq_len shorter than its chunk or longer
  * than its table row, or a decreasing query_start, sets PKV_DEVERR_SEQ_LEN
- * (those rows are not written); an out-of-range block id reads zeros and
- * sets PKV_DEVERR_BLOCK_ID.  No workspace.  The products run on the
- * tensor core with accumulators in tensor memory (256 columns per CTA).
+ * (those rows are not written); an out-of-range block id is read as block 0
+ * (the affected rows are unspecified) and sets PKV_DEVERR_BLOCK_ID.
+ * num_query_tokens and num_blocks * block_size must stay below 2^31 (32-bit
+ * copy coordinates; otherwise PKV_EUNSUPPORTED).  No workspace.  The
+ * products run on the tensor core with accumulators in tensor memory: one
+ * CTA per SM holding all 512 columns; q and K/V tiles are copied by TMA.
  */
 pkv_status pkv_paged_prefill(void* out, const void* query, pkv_dtype q_dtype, const void* key_cache,
                              const void* value_cache, pkv_dtype cache_dtype,
