@@ -52,7 +52,8 @@ constexpr int kPfLoadWarp = 17;     // issues the TMA copies
 constexpr int kPfThreads = 18 * 32;
 constexpr int kPfStages = 3;        // K and V ring depth
 constexpr int kPfTmemCols = 512;    // unit u: S in columns 256 u + [0, 64), O from 256 u + 64,
-constexpr int kPfTmemP = 192;       //   P (hi, lo: 32 columns each) from 256 u + 192
+constexpr int kPfTmemP = 192;       //   P (hi, lo: 32 columns each) from 256 (1 - u) + 192: the
+                                    //   other half from its O (measured 1 % faster than beside it)
 constexpr uint64_t kPfWaitNs = 200000000ull;
 
 // mbarriers
@@ -375,7 +376,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
             const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
             const uint32_t tS = tmem + lane_addr + X * 256 + half * (kPfTok / 2);
             const uint32_t tO = tmem + lane_addr + X * 256 + kPfTok + half * (D / 2);
-            const uint32_t tP = tmem + lane_addr + X * 256 + kPfTmemP + half * (kPfTok / 4);
+            const uint32_t tP = tmem + lane_addr + (X ^ 1) * 256 + kPfTmemP + half * (kPfTok / 4);
             const float sl2 = p.scale_log2;
             float mref = -INFINITY, l = 0.f;  // reference maximum (log2 domain) and this half's sum
             bool failed = false;
@@ -536,7 +537,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
             };
             auto issue_pv = [&](int X, int st, bool acc) {  // O_X (+)= P_X V (hi, then lo; P in tensor memory)
                 const uint64_t vd = desc_add(dv0, (uint32_t)(st * (SM::kTile >> 4)));
-                const uint32_t d = tmem + X * 256 + kPfTok, a = tmem + X * 256 + kPfTmemP;
+                const uint32_t d = tmem + X * 256 + kPfTok, a = tmem + (X ^ 1) * 256 + kPfTmemP;
 #pragma unroll
                 for (int part = 0; part < SM::kParts; ++part)
 #pragma unroll
