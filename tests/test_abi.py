@@ -97,3 +97,44 @@ def test_decode_step_struct_layout():
     assert pkv.DecodeStepArgs.num_blocks.offset == 24
     assert pkv.DecodeStepArgs.h_query.offset == 48
     assert pkv.DecodeStepArgs.workspace_bytes.offset == 224
+
+
+def _prefill(L, **kw):
+    a = dict(out=None, query=None, q_dtype=pkv.PKV_BF16, key_cache=None, value_cache=None,
+             cache_dtype=pkv.PKV_BF16, block_tables=None, max_blocks_per_seq=4, seq_lens=None,
+             query_start=None, num_seqs=2, num_query_tokens=10, num_heads=8, num_kv_heads=4, head_dim=128,
+             block_size=16, num_blocks=64, scale=0.1, stream=None)
+    a.update(kw)
+    return L.pkv_paged_prefill(*a.values())
+
+
+def test_prefill_host_validation_without_gpu(L):
+    assert _prefill(L, head_dim=96) == pkv.PKV_EUNSUPPORTED
+    assert _prefill(L, block_size=8) == pkv.PKV_EUNSUPPORTED
+    assert _prefill(L, num_heads=12, num_kv_heads=4) == pkv.PKV_EUNSUPPORTED   # g = 3
+    assert _prefill(L, num_heads=6, num_kv_heads=4) == pkv.PKV_EINVAL
+    assert _prefill(L, cache_dtype=pkv.PKV_FP8_E4M3) == pkv.PKV_EUNSUPPORTED
+    assert _prefill(L, q_dtype=pkv.PKV_F16) == pkv.PKV_EUNSUPPORTED            # q dtype != cache dtype
+    assert _prefill(L, q_dtype=pkv.PKV_F32, cache_dtype=pkv.PKV_F32) == pkv.PKV_EUNSUPPORTED
+    assert _prefill(L, scale=0.0) == pkv.PKV_EINVAL
+    assert _prefill(L, num_query_tokens=-1) == pkv.PKV_EINVAL
+    assert _prefill(L, num_blocks=0) == pkv.PKV_EINVAL
+    assert _prefill(L, num_seqs=0) == pkv.PKV_OK                               # nothing to do
+    assert _prefill(L, num_query_tokens=0) == pkv.PKV_OK
+    assert _prefill(L) == pkv.PKV_EINVAL                                        # null pointers
+    assert b"null" in L.pkv_last_error_message()
+
+
+def test_swap_host_validation_without_gpu(L):
+    def swap(**kw):
+        a = dict(dk=None, dv=None, dnb=64, sk=None, sv=None, snb=64, layers=2, mapping=None, pairs=3,
+                 block_bytes=4096, stream=None)
+        a.update(kw)
+        return L.pkv_swap_blocks(*a.values())
+    assert swap(pairs=-1) == pkv.PKV_EINVAL
+    assert swap(layers=0) == pkv.PKV_EINVAL
+    assert swap(dnb=0) == pkv.PKV_EINVAL
+    assert swap(block_bytes=4095) == pkv.PKV_EINVAL
+    assert swap(block_bytes=0) == pkv.PKV_EINVAL
+    assert swap(pairs=0) == pkv.PKV_OK                                     # nothing to do
+    assert swap() == pkv.PKV_EINVAL                                        # null pointers
