@@ -210,6 +210,23 @@ class OracleSample:
         return self.k / self.time(self.k)
 
 
+def pool_bytes(wl) -> int:
+    return wl.num_blocks * wl.block_size * wl.num_kv_heads * wl.head_dim * wl.kv_elem_bytes() * 2
+
+
+def decode_config(wl, cascade: bool, world: int) -> dict:
+    """The decode line's config, shared by both arms."""
+    flush = pool_bytes(wl) < 2 * L2_BYTES
+    return {"workload": wl.name + ("_cascade" if cascade else ""),
+            "num_seqs": wl.num_seqs, "num_heads": wl.num_heads,
+            "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+            "block_size": wl.block_size, "num_blocks": wl.num_blocks,
+            "max_seq_len": wl.max_seq_len, "cow_pairs": int(wl.cow_pairs.shape[0]),
+            "kv_bytes_alg": wl.algorithmic_bytes(),
+            "l2": "flushed between steps" if flush else "inputs larger than L2 (126 MB)",
+            "parallelism": f"replicas x{world} (independent batches)"}
+
+
 def run_reference(args):
     rank, world, local = dist_env()
     if rank != 0:
@@ -225,7 +242,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * wl.num_seqs / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "num_seqs": wl.num_seqs},
+        "config": decode_config(wl, args.cascade, args.gpus),
         "cpu_baseline": {"value": value, "unit": "seq-steps/s", "cores": cores, "kind": "oracle",
                          "sample": f"first {k_used} of {wl.num_seqs} sequences per step, fp64 C oracle"},
         "e2e": {"value": value, "unit": "seq-steps/s", "h2d_bytes_per_step": 0,
@@ -262,9 +279,7 @@ def run_ours(args):
                              args.num_ctas, device=dev)
     has_pairs = g["pairs"].numel() > 0
     stream = torch.cuda.current_stream()
-    kv_bytes = (wl.num_blocks * wl.block_size * wl.num_kv_heads * wl.head_dim *
-                wl.kv_elem_bytes() * 2)
-    flush = kv_bytes < 2 * L2_BYTES
+    flush = pool_bytes(wl) < 2 * L2_BYTES
     scratch = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if flush else None
 
     if args.cascade:
@@ -365,14 +380,7 @@ def run_ours(args):
             "dtype": {True: "fp8_e4m3 kv / fp32 accum", False: str(wl.kv_dtype).replace("torch.", "")
                       + " kv / fp32 accum"}[wl.is_fp8],
             "data": "synthetic",
-            "config": {"workload": wl.name + ("_cascade" if args.cascade else ""),
-                       "num_seqs": wl.num_seqs, "num_heads": wl.num_heads,
-                       "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
-                       "block_size": wl.block_size, "num_blocks": wl.num_blocks,
-                       "max_seq_len": wl.max_seq_len, "cow_pairs": int(wl.cow_pairs.shape[0]),
-                       "kv_bytes_alg": b_alg,
-                       "l2": "flushed between steps" if flush else "inputs larger than L2 (126 MB)",
-                       "parallelism": f"replicas x{world} (independent batches)"},
+            "config": decode_config(wl, args.cascade, world),
             "attention_ms": attn_avg_ms,
             "kv_read_gbs": achieved,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
