@@ -20,8 +20,9 @@
 //     row (one per half of the 64 scores and of the head_dim outputs): load
 //     S from tensor memory, mask, exponentiate against a reference maximum,
 //     write P back to tensor memory, where the P V product reads it as its
-//     A operand (bf16 as hi + lo parts, so P V keeps fp32-level accuracy).  O stays in tensor memory across tiles; it is
-//     rescaled only when a row's maximum passes its reference by 2^8.
+//     A operand (bf16 as hi + lo parts, so P V keeps fp32-level accuracy).
+//     O stays in tensor memory across tiles; it is rescaled only when a
+//     row's maximum passes its reference by 2^8.
 // A unit without a partner (a decode row, the first row tile of a sequence
 // with an odd count) splits its tiles instead: group 0 takes the even tiles,
 // group 1 the odd ones, and group 0 merges the two partial (max, sum, O)
