@@ -32,7 +32,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention seq-steps/s and KV-read HBM GB/s (% of B200 peak)"
 L2_BYTES = 126 * 1024 * 1024
-WORKLOADS = {"cfg1": 1, "cfg2": 2, "cfg3": 3, "cfg4": 4, "cfg5": 5}
+WORKLOADS = {"cfg1": 1, "cfg2": 2, "cfg3": 3, "cfg4": 4, "cfg5": 5,
+             "short": 7}    # 2048 sequences of U[1, 64] tokens (not one of the five configurations)
 
 
 # ---------------------------------------------------------------- distributed
@@ -67,7 +68,7 @@ def make_workload(name: str, rank: int, num_seqs: int = 0):
     from paged_kv_cache_373_b200 import workloads as W
     cfg = WORKLOADS[name]
     kw = {}
-    if num_seqs and cfg in (2, 3, 4):
+    if num_seqs and cfg in (2, 3, 4, 7):
         kw["num_seqs"] = num_seqs
     elif num_seqs and cfg == 5:
         kw["num_prompts"] = max(1, num_seqs // 8)
@@ -145,10 +146,11 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
             self.f.close()
+        self.rows = self._read()
 
-    def summary(self):
+    def _read(self):
         if not self.path or not os.path.exists(self.path):
-            return None
+            return []
         import datetime
         rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -164,9 +166,15 @@ class ClockSampler:
                 except ValueError:
                     continue
         os.unlink(self.path)
+        return rows
+
+    def summary(self, window=None):
+        """Median SM clock, max clock and throttle reasons of the samples taken
+        inside `window` (wall-clock (t0, t1); default: the timed region)."""
+        rows = getattr(self, "rows", None) or []
         if not rows:
             return None
-        t0, t1 = self.window or (rows[0][0], rows[-1][0])
+        t0, t1 = window or self.window or (rows[0][0], rows[-1][0])
         inside = [r for r in rows if t0 - 0.02 <= r[0] <= t1 + 0.02]
         scope = "timed region"
         if not inside:  # region shorter than the sampling period: nearest samples
@@ -189,25 +197,55 @@ class OracleSample:
         self.oracle, self.wl = oracle, wl
         self.cores = threads or oracle.num_threads_available()
         kmax = wl.num_seqs if not wl.is_fp8 else min(wl.num_seqs, 64)
+        self.kmax = kmax
         self.kc, self.vc = oracle_caches(wl, None if not wl.is_fp8 else list(range(kmax)))
+        self.k = self._calibrate(budget_s, self.cores)
+
+    def _calibrate(self, budget_s: float, threads: int) -> int:
         k = 1
         while True:
-            dt = self.time(k)
-            if dt >= budget_s / 2 or k >= kmax:
-                break
-            k = min(kmax, max(k + 1, int(k * min(8.0, budget_s / max(dt, 1e-4)))))
-        self.k = k
+            dt = self.time(k, threads)
+            if dt >= budget_s / 2 or k >= self.kmax:
+                return k
+            k = min(self.kmax, max(k + 1, int(k * min(8.0, budget_s / max(dt, 1e-4)))))
 
-    def time(self, k: int) -> float:
+    def time(self, k: int, threads: int = 0) -> float:
         wl = self.wl
         t0 = time.perf_counter()
         self.oracle.paged_attention_decode(wl.query, self.kc, self.vc, wl.block_tables, wl.seq_lens,
                                            wl.scale, wl.k_scale, wl.v_scale,
-                                           seq_subset=list(range(k)), num_threads=self.cores)
+                                           seq_subset=list(range(k)), num_threads=threads or self.cores)
         return time.perf_counter() - t0
 
     def rate(self) -> float:
         return self.k / self.time(self.k)
+
+    def single_thread(self, budget_s: float):
+        """(seq-steps/s, sequences timed) with one thread."""
+        k1 = self._calibrate(budget_s, 1)
+        return k1 / self.time(k1, 1), k1
+
+
+def host_cores() -> dict:
+    """os.cpu_count() and nproc (the cores this process may use)."""
+    try:
+        nproc = int(subprocess.run(["nproc"], capture_output=True, text=True).stdout.strip())
+    except Exception:
+        nproc = None
+    return {"os_cpu_count": os.cpu_count(), "nproc": nproc}
+
+
+def cpu_baseline_line(wl, budget_s: float) -> dict:
+    """The oracle on the host cores: all threads (the reported value) and one thread."""
+    smp = OracleSample(wl, budget_s=budget_s)
+    r = smp.rate()
+    r1, k1 = smp.single_thread(budget_s / 3)
+    return {"value": r, "unit": "seq-steps/s", "cores": smp.cores, "kind": "oracle",
+            "sample": f"first {smp.k} of {wl.num_seqs} sequences of the same workload, "
+                      f"fp64 C oracle, {smp.cores} OpenMP threads",
+            "single_thread": {"value": r1, "unit": "seq-steps/s", "cores": 1,
+                              "sample": f"first {k1} of {wl.num_seqs} sequences, 1 thread"},
+            **host_cores()}
 
 
 def pool_bytes(wl) -> int:
@@ -232,8 +270,12 @@ def run_reference(args):
     if rank != 0:
         return 0
     wl = make_workload(args.workload, 0, args.num_seqs)
-    # each step is a bounded sample so the whole run stays within a few minutes
-    smp = OracleSample(wl, budget_s=max(0.5, min(args.ref_budget, 120.0 / max(1, args.steps))))
+    # each step is a bounded sample so the whole run (warm-up included) stays
+    # within a few minutes
+    budget = max(0.5, min(args.ref_budget, 120.0 / max(1, args.steps + args.warmup)))
+    smp = OracleSample(wl, budget_s=budget)
+    for _ in range(args.warmup):
+        smp.rate()
     rates = [smp.rate() for _ in range(args.steps)]
     k_used, cores = smp.k, smp.cores
     value = statistics.median(rates)
@@ -244,7 +286,9 @@ def run_reference(args):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": decode_config(wl, args.cascade, args.gpus),
         "cpu_baseline": {"value": value, "unit": "seq-steps/s", "cores": cores, "kind": "oracle",
-                         "sample": f"first {k_used} of {wl.num_seqs} sequences per step, fp64 C oracle"},
+                         "sample": f"first {k_used} of {wl.num_seqs} sequences per step, fp64 C oracle, "
+                                   f"median of {args.steps} steps",
+                         **host_cores()},
         "e2e": {"value": value, "unit": "seq-steps/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -270,10 +314,8 @@ def run_ours(args):
     wl = make_workload(args.workload, rank, args.num_seqs)
 
     # ---- resident device state
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from pkv_testutil import gpu_inputs
-    g = gpu_inputs(wl, dev)
-    pristine = None
+    from paged_kv_cache_373_b200.device_inputs import decode_inputs
+    g = decode_inputs(wl, dev)
     out = torch.empty_like(g["q"])
     ws = pkv.alloc_workspace(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim,
                              args.num_ctas, device=dev)
@@ -308,6 +350,17 @@ def run_ours(args):
         if ev_a1 is not None:
             ev_a1.record(stream)
 
+    def timed_steps(n):
+        """n steps, each bracketed by events (step, and attention inside it)."""
+        ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(n)]
+        for i in range(n):
+            if flush:
+                scratch.fill_(i & 0xff)     # evict the small workload from L2 (outside the step events)
+            ev[i][0].record(stream)
+            step(ev[i][1], ev[i][2])
+            ev[i][3].record(stream)
+        return ev
+
     # warm-up: at least W steps and at least --spinup-ms of GPU work, so the SM
     # clock has left its idle state before the timed region
     clk = ClockSampler(dev.index).start()
@@ -322,26 +375,18 @@ def run_ours(args):
     if pkv.get_device_error() != 0:
         raise RuntimeError("device error during warm-up")
 
+    # ---- the timed region: exactly K steps
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize()
     wall0 = time.time()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for i in range(K):
-        if flush:
-            scratch.fill_(i & 0xff)     # evict the small workload from L2 (outside the step events)
-        ev[i][0].record(stream)
-        step(ev[i][1], ev[i][2])
-        ev[i][3].record(stream)
+    ev = timed_steps(K)
     t_end.record(stream)
     torch.cuda.synchronize()
     clk.window = (wall0, time.time())
-    clk.stop()
     barrier(world)
     step_ms = [a.elapsed_time(d) for a, _, _, d in ev]
     attn_ms = [b.elapsed_time(c) for _, b, c, _ in ev]
@@ -350,24 +395,49 @@ def run_ours(args):
     if pkv.get_device_error() != 0:
         raise RuntimeError("device error during the timed steps")
 
+    # ---- the measurement protocol of the scope table, after the timed
+    # region: the median of >= 50 individually timed steps spanning >= 0.5 s,
+    # with the SM clock sampled over that window
+    proto = None
+    if not args.no_protocol:
+        n_proto, proto_ms, proto_attn = 0, [], []
+        wallp = time.time()
+        while n_proto < 50 or time.time() - wallp < 0.5:
+            evp = timed_steps(50)
+            torch.cuda.synchronize()
+            proto_ms += [a.elapsed_time(d) for a, _, _, d in evp]
+            proto_attn += [b.elapsed_time(c) for _, b, c, _ in evp]
+            n_proto += 50
+        window = (wallp, time.time())
+        med_attn = statistics.median(proto_attn)
+        proto = {"runs": n_proto, "median_step_ms": statistics.median(proto_ms),
+                 "median_attention_ms": med_attn,
+                 "p10_p90_attention_ms": [sorted(proto_attn)[n_proto // 10],
+                                          sorted(proto_attn)[(9 * n_proto) // 10]],
+                 "kv_read_gbs_at_median": wl.algorithmic_bytes() / (med_attn / 1000.0) / 1e9,
+                 "window_s": window[1] - window[0], "clocks": None}
+        proto["_window"] = window
+        if pkv.get_device_error() != 0:
+            raise RuntimeError("device error during the protocol steps")
+    clk.stop()
+    if proto is not None:
+        proto["clocks"] = clk.summary(proto.pop("_window"))
+
     ms_per_step = total_ms / K
     value = world * wl.num_seqs / (ms_per_step / 1000.0)
     attn_avg_ms = statistics.mean(attn_ms)
     b_alg = wl.algorithmic_bytes()
     peak, peak_kind = measured_peaks()
     achieved = b_alg / (attn_avg_ms / 1000.0) / 1e9
+    traffic = recorded_traffic(wl.name + ("_cascade" if args.cascade else ""))
 
     # ---- end-to-end through the C ABI with host buffers
-    e2e = e2e_leg(pkv, wl, g, ws, args, dev) if not args.no_e2e else None
+    e2e = e2e_leg(pkv, wl, g, ws, args, dev, out_ref=None if args.cascade else out) if not args.no_e2e else None
     e2e_value = reduce_max(e2e["ms"], world, dev) if e2e else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        smp = OracleSample(wl, budget_s=args.ref_budget)
-        r = smp.rate()
-        cpu = {"value": r, "unit": "seq-steps/s", "cores": smp.cores, "kind": "oracle",
-               "sample": f"first {smp.k} of {wl.num_seqs} sequences of the same workload, "
-                         f"fp64 C oracle, {smp.cores} OpenMP threads"}
+        cpu = cpu_baseline_line(wl, args.ref_budget)
 
     # copy_blocks, reshape_and_cache, then decode + merge (cascade: setup, prefix, suffix decode + merge, combine)
     launches_per_step = (1 if has_pairs else 0) + 1 + (5 if args.cascade else 2)
@@ -375,22 +445,33 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": value, "unit": "seq-steps/s", "n_gpus": world,
             "steps": K, "warmup": warm, "warmup_requested": args.warmup,
+            "warmup_note": f"at least the requested steps and at least {args.spinup_ms:.0f} ms of GPU "
+                           "work, so the SM clock has left its idle state before the timed region",
             "ms_per_step": ms_per_step,
+            "timing": f"sum of {K} per-step event intervals (L2 flushed between steps)" if flush else
+                      f"one event interval over {K} back-to-back steps (mean)",
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": {True: "fp8_e4m3 kv / fp32 accum", False: str(wl.kv_dtype).replace("torch.", "")
                       + " kv / fp32 accum"}[wl.is_fp8],
             "data": "synthetic",
             "config": decode_config(wl, args.cascade, world),
             "attention_ms": attn_avg_ms,
+            "attention_ms_median": statistics.median(attn_ms),
             "kv_read_gbs": achieved,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
-                         "traffic": recorded_traffic(wl.name)},
+                         "traffic": traffic,
+                         "traffic_source": None if traffic is None else
+                         "profiles/traffic.json: ncu dram__bytes_read.sum + dram__bytes_write.sum of one "
+                         "attention call (decode + merge kernels) on this workload, not measured in this run"},
             "clocks": clk.summary(),
+            "protocol": proto,
             "gpu_launches": launches_per_step * K,
             "e2e": None if e2e is None else {
                 "value": world * wl.num_seqs / (e2e_value / 1000.0), "unit": "seq-steps/s",
-                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                "copies_per_step": e2e["copies"], "output_matches_device_path": e2e["matches_device_path"],
+                "api": "pkv_decode_step_host, packed inputs (one H2D, one D2H, one stream sync per step)"},
             "cpu_baseline": cpu,
         }
         print(json.dumps(line))
@@ -685,32 +766,42 @@ class _OracleAdapter:
         self.ob.free_sequence(sid)
 
 
-def e2e_leg(pkv, wl, g, ws, args, dev):
-    """decode_step_host: pinned host inputs -> H2D -> step -> D2H -> sync."""
-    pin = lambda t: t.contiguous().pin_memory()
-    h = dict(q=pin(wl.query), nk=pin(wl.new_key.to(wl.q_dtype)), nv=pin(wl.new_value.to(wl.q_dtype)),
-             slots=pin(wl.slot_mapping), tables=pin(wl.block_tables), lens=pin(wl.seq_lens),
-             pairs=pin(wl.cow_pairs), out=torch.empty_like(wl.query).pin_memory())
-    d = dict(q=torch.empty_like(g["q"]), nk=torch.empty_like(g["nk"]), nv=torch.empty_like(g["nv"]),
-             slots=torch.empty_like(g["slots"]), tables=torch.empty_like(g["tables"]),
-             lens=torch.empty_like(g["lens"]), pairs=torch.empty_like(g["pairs"]),
-             out=torch.empty_like(g["q"]))
+def e2e_leg(pkv, wl, g, ws, args, dev, out_ref=None):
+    """decode_step_host with packed inputs: the step's inputs sit in one pinned
+    host buffer (laid out by pkv_decode_step_layout) -> one H2D copy ->
+    copy_blocks / reshape_and_cache / decode -> one D2H copy of the output ->
+    stream sync, every step."""
+    qd = pkv.dtype_code(wl.query)
+    npairs = int(wl.cow_pairs.shape[0])
+    lay = pkv.decode_step_layout(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, qd,
+                                 wl.max_blocks_per_seq, npairs)
+    hbuf = torch.zeros(lay.total, dtype=torch.uint8).pin_memory()
+
+    def put(off, t):
+        b = t.contiguous().view(-1).view(torch.uint8)
+        hbuf[off:off + b.numel()] = b
+
+    put(lay.query, wl.query)
+    put(lay.new_key, wl.new_key.to(wl.q_dtype))
+    put(lay.new_value, wl.new_value.to(wl.q_dtype))
+    put(lay.slot_mapping, wl.slot_mapping)
+    put(lay.block_tables, wl.block_tables)
+    put(lay.seq_lens, wl.seq_lens)
+    if npairs:
+        put(lay.cow_pairs, wl.cow_pairs)
+    dbuf = torch.empty(max(lay.total, 16), dtype=torch.uint8, device=dev)
+    h_out = torch.empty_like(wl.query).pin_memory()
+    d_out = torch.empty_like(g["q"])
     a = pkv.DecodeStepArgs()
     a.num_seqs, a.num_heads, a.num_kv_heads = wl.num_seqs, wl.num_heads, wl.num_kv_heads
     a.head_dim, a.block_size, a.max_blocks_per_seq = wl.head_dim, wl.block_size, wl.max_blocks_per_seq
     a.num_blocks = wl.num_blocks
-    a.q_dtype = pkv.dtype_code(wl.query)
-    a.cache_dtype = pkv.PKV_FP8_E4M3 if wl.is_fp8 else pkv.dtype_code(wl.query)
+    a.q_dtype = qd
+    a.cache_dtype = pkv.PKV_FP8_E4M3 if wl.is_fp8 else qd
     a.scale, a.num_ctas = wl.scale, args.num_ctas
-    a.h_query, a.h_new_key, a.h_new_value = h["q"].data_ptr(), h["nk"].data_ptr(), h["nv"].data_ptr()
-    a.h_slot_mapping, a.h_block_tables = h["slots"].data_ptr(), h["tables"].data_ptr()
-    a.h_seq_lens, a.h_out = h["lens"].data_ptr(), h["out"].data_ptr()
-    a.num_cow_pairs = int(wl.cow_pairs.shape[0])
-    a.h_cow_pairs = h["pairs"].data_ptr() if a.num_cow_pairs else None
-    a.d_query, a.d_new_key, a.d_new_value = d["q"].data_ptr(), d["nk"].data_ptr(), d["nv"].data_ptr()
-    a.d_slot_mapping, a.d_block_tables = d["slots"].data_ptr(), d["tables"].data_ptr()
-    a.d_seq_lens, a.d_out = d["lens"].data_ptr(), d["out"].data_ptr()
-    a.d_cow_pairs = d["pairs"].data_ptr() if a.num_cow_pairs else None
+    a.num_cow_pairs = npairs
+    a.h_packed, a.d_packed = hbuf.data_ptr(), dbuf.data_ptr()
+    a.h_out, a.d_out = h_out.data_ptr(), d_out.data_ptr()
     a.key_cache, a.value_cache = g["kc"].data_ptr(), g["vc"].data_ptr()
     a.k_scale = g["ks"].data_ptr() if g["ks"] is not None else None
     a.v_scale = g["vs"].data_ptr() if g["vs"] is not None else None
@@ -726,10 +817,10 @@ def e2e_leg(pkv, wl, g, ws, args, dev):
         pkv.decode_step_host(a, stream)
     e1.record(stream)
     torch.cuda.synchronize()
-    h2d = sum(h[k].numel() * h[k].element_size() for k in ("q", "nk", "nv", "slots", "tables", "lens"))
-    h2d += h["pairs"].numel() * 8
-    d2h = h["out"].numel() * h["out"].element_size()
-    return {"ms": e0.elapsed_time(e1) / K, "h2d": h2d, "d2h": d2h}
+    same = None if out_ref is None else bool(torch.equal(h_out.view(-1).view(torch.uint8),
+                                                         out_ref.cpu().view(-1).view(torch.uint8)))
+    return {"ms": e0.elapsed_time(e1) / K, "h2d": int(lay.total),
+            "d2h": h_out.numel() * h_out.element_size(), "copies": 2, "matches_device_path": same}
 
 
 def main():
@@ -738,7 +829,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="cfg2", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="cfg3", choices=sorted(WORKLOADS),
+                    help="cfg3 (the largest single-GPU configuration) by default")
     ap.add_argument("--num-ctas", type=int, default=0)
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="override the workload's batch (profiling a smaller case)")
@@ -746,6 +838,8 @@ def main():
                     help="minimum untimed warm-up time (clock ramp-up)")
     ap.add_argument("--ref-budget", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-protocol", action="store_true",
+                    help="skip the median-of->=50-steps measurement after the timed region")
     ap.add_argument("--cascade", action="store_true",
                     help="prefix-sharing workloads: read each shared prefix once per group")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -164,7 +164,8 @@ pkv_status pkv_swap_blocks(void* const* dst_key_caches, void* const* dst_value_c
  * split units, (12 * num_ctas + units) x heads_per_unit x (head_dim + 2)
  * floats, where units = num_seqs * num_kv_heads * ceil(g / 8),
  * g = num_heads / num_kv_heads and heads_per_unit = min(g, 8).  num_ctas = 0 means the default grid of the
- * current device (pkv_default_num_ctas).  Returns 0 for invalid shapes.
+ * current device (pkv_default_num_ctas).  Returns 0 for invalid shapes
+ * (num_ctas outside [0, 2^20] included).
  * The workspace needs no initialisation.
  */
 size_t pkv_paged_attention_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
@@ -201,7 +202,8 @@ int pkv_default_num_ctas(void);
  * physical block ids and independent of block sharing, for a fixed num_ctas.
  * workspace: device, >= pkv_paged_attention_workspace_bytes(...) bytes,
  *   16-byte aligned, contents need no initialisation.
- * num_ctas: 0 = default; otherwise the persistent grid size (sets the split).
+ * num_ctas: 0 = default; otherwise the persistent grid size (sets the split),
+ *   at most 2^20 (PKV_EINVAL above).
  * out, query, caches: 16-byte aligned device pointers.
  */
 pkv_status pkv_paged_attention_decode(void* out, const void* query, pkv_dtype q_dtype,
@@ -309,15 +311,23 @@ pkv_status pkv_paged_prefill(void* out, const void* query, pkv_dtype q_dtype, co
  *
  * Same arguments, semantics and results as pkv_paged_attention_decode; the
  * split-merge scratch is one file-scope device array of
- * PKV_STATIC_WORKSPACE_BYTES (16 MiB) that every GPU loading this library holds
- * until the process exits.  The call allocates nothing (no cudaMalloc,
- * cudaFree or allocating library routine).
+ * PKV_STATIC_WORKSPACE_BYTES (16 MiB), held on a device until the process
+ * exits.  The call itself runs no cudaMalloc, cudaFree or allocating library
+ * routine.
  *   - Limit: if pkv_paged_attention_workspace_bytes(num_seqs, num_heads,
  *     num_kv_heads, head_dim, num_ctas) exceeds PKV_STATIC_WORKSPACE_BYTES the
  *     call returns PKV_EINVAL and launches nothing.
- *   - Set-up: the first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress with that device current); make that first call
- *     before any stream capture.
+ *   - Set-up: every call looks up the array's device address on the current
+ *     device (cudaGetSymbolAddress).  Under lazy module loading (the CUDA
+ *     default) the first lookup on a device is what commits the 16 MiB there,
+ *     so the FIRST call on each device may allocate and synchronise.  Make one
+ *     warm-up call per device, with that device current, before the KV pool
+ *     takes the device memory and before any stream capture: a call with
+ *     num_seqs = 0 (dtypes, head_dim, block_size, num_blocks and
+ *     max_blocks_per_seq valid; pointers may be NULL) does only that set-up
+ *     and returns PKV_OK.  Later calls allocate nothing.  Because the address
+ *     is looked up each time, a call after cudaDeviceReset uses the new
+ *     context's array (and is again a first call).
  *   - Sharing: every call on a device uses the same array, which keeps the
  *     last call's contents.  Nothing in it has to start at zero (every value
  *     read is written earlier by the same call), but calls that overlap on the
@@ -342,6 +352,13 @@ pkv_status pkv_paged_attention_decode_noalloc(void* out, const void* query, pkv_
  * the stream.  Host buffers should be pinned for asynchronous copies.
  * The caches stay resident on the device.  Device staging buffers are
  * caller-owned and sized like their host counterparts.
+ *
+ * Packed inputs (h_packed != NULL): the caller writes all the step's inputs
+ * into ONE pinned host buffer at the offsets pkv_decode_step_layout gives,
+ * and the step moves them with one host -> device copy into d_packed (device,
+ * layout.total bytes, 16-byte aligned) instead of one copy per input; the
+ * h_query ... h_cow_pairs and d_query ... d_cow_pairs fields are then
+ * ignored.  The output still goes d_out -> h_out in one copy.
  */
 typedef struct pkv_decode_step_args {
     /* shapes */
@@ -377,9 +394,28 @@ typedef struct pkv_decode_step_args {
     const float* v_scale;
     void* workspace;
     size_t workspace_bytes;
+    /* packed inputs (optional; see above) */
+    const void* h_packed;             /* pinned host, layout.total bytes, or NULL */
+    void* d_packed;                   /* device, layout.total bytes */
 } pkv_decode_step_args;
 
 pkv_status pkv_decode_step_host(const pkv_decode_step_args* args, pkv_stream_t stream);
+
+/* Byte offsets of a decode step's inputs inside one packed buffer: each
+ * array starts on a 256-byte boundary, in the order query [S, Hq, D],
+ * new_key and new_value [S, Hkv, D] (q dtype), slot_mapping int64 [S],
+ * block_tables int32 [S, max_blocks_per_seq], seq_lens int32 [S],
+ * cow_pairs int64 [num_cow_pairs, 2]; total = the packed size in bytes. */
+typedef struct pkv_step_layout {
+    size_t query, new_key, new_value, slot_mapping, block_tables, seq_lens, cow_pairs;
+    size_t total;
+} pkv_step_layout;
+
+/* Fill *layout for these shapes.  PKV_EINVAL for negative sizes, a bad dtype
+ * or a null layout. */
+pkv_status pkv_decode_step_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                  pkv_dtype q_dtype, int max_blocks_per_seq,
+                                  int64_t num_cow_pairs, pkv_step_layout* layout);
 
 /* Synchronise `stream`, return the device error word of the current device
  * in *code_out and clear it.  Returns PKV_EDEVICE if it was non-zero. */

@@ -8,7 +8,7 @@ are not on a CUDA device, the call raises.
 Names follow the C entry points without their ``pkv_`` prefix:
   reshape_and_cache, copy_blocks, swap_blocks, paged_attention_decode, paged_prefill,
   paged_attention_decode_noalloc, paged_attention_decode_cascade,
-  paged_attention_workspace_bytes, default_num_ctas, decode_step_host,
+  paged_attention_workspace_bytes, default_num_ctas, decode_step_host, decode_step_layout,
   get_device_error, status_string
 """
 from __future__ import annotations
@@ -33,6 +33,7 @@ EXPORTED = ("pkv_reshape_and_cache", "pkv_copy_blocks", "pkv_swap_blocks", "pkv_
             "pkv_default_num_ctas", "pkv_paged_attention_decode",
             "pkv_paged_attention_decode_noalloc", "pkv_paged_attention_cascade_workspace_bytes",
             "pkv_paged_attention_decode_cascade", "pkv_paged_prefill", "pkv_decode_step_host",
+            "pkv_decode_step_layout", "pkv_testing_prefill_timeout",
             "pkv_get_device_error", "pkv_status_string", "pkv_last_error_message")
 
 
@@ -62,7 +63,14 @@ class DecodeStepArgs(ctypes.Structure):
         ("key_cache", ctypes.c_void_p), ("value_cache", ctypes.c_void_p),
         ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("h_packed", ctypes.c_void_p), ("d_packed", ctypes.c_void_p),
     ]
+
+
+class StepLayout(ctypes.Structure):
+    """Mirror of ``pkv_step_layout`` (byte offsets inside one packed input buffer)."""
+    _fields_ = [(n, ctypes.c_size_t) for n in ("query", "new_key", "new_value", "slot_mapping",
+                                               "block_tables", "seq_lens", "cow_pairs", "total")]
 
 
 _lib_handle = None
@@ -109,6 +117,11 @@ def lib() -> ctypes.CDLL:
                                     c_int, c_int, c_int, i64, ctypes.c_float, vp]
     L.pkv_decode_step_host.restype = c_int
     L.pkv_decode_step_host.argtypes = [ctypes.POINTER(DecodeStepArgs), vp]
+    L.pkv_decode_step_layout.restype = c_int
+    L.pkv_decode_step_layout.argtypes = [c_int, c_int, c_int, c_int, c_int, c_int, i64,
+                                         ctypes.POINTER(StepLayout)]
+    L.pkv_testing_prefill_timeout.restype = c_int
+    L.pkv_testing_prefill_timeout.argtypes = [c_int, ctypes.c_uint64]
     L.pkv_get_device_error.restype = c_int
     L.pkv_get_device_error.argtypes = [ctypes.POINTER(i32), vp]
     L.pkv_status_string.restype = ctypes.c_char_p
@@ -300,6 +313,15 @@ def paged_attention_decode_cascade(out, query, key_cache, value_cache, block_tab
 def decode_step_host(args: DecodeStepArgs, stream=None) -> None:
     """One host-driven decode step (see pkv_decode_step_host); synchronises."""
     _check(lib().pkv_decode_step_host(ctypes.byref(args), _stream(stream)))
+
+
+def decode_step_layout(num_seqs: int, num_heads: int, num_kv_heads: int, head_dim: int,
+                       q_dtype: int, max_blocks_per_seq: int, num_cow_pairs: int = 0) -> StepLayout:
+    """Offsets of a decode step's inputs in one packed buffer (pkv_decode_step_layout)."""
+    lay = StepLayout()
+    _check(lib().pkv_decode_step_layout(num_seqs, num_heads, num_kv_heads, head_dim, q_dtype,
+                                        max_blocks_per_seq, num_cow_pairs, ctypes.byref(lay)))
+    return lay
 
 
 def get_device_error(stream=None) -> int:

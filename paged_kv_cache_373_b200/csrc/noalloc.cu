@@ -2,46 +2,36 @@
 // entry point for callers that cannot hand the library a workspace.
 //
 // The split-merge scratch lives in one file-scope device array of a fixed
-// size (kStaticWorkspaceBytes).  Every GPU that loads this library holds it
-// until the process exits.  Host code cannot pass the array's name to a
-// kernel (on the host it is only a stand-in symbol), so its device address is
-// looked up once per device with cudaGetSymbolAddress while that device is
-// current, and that address is what the existing decode path receives.
-#include <mutex>
-
+// size (kStaticWorkspaceBytes).  Host code cannot pass the array's name to a
+// kernel (on the host it is only a stand-in symbol), so every call looks up
+// its device address with cudaGetSymbolAddress on the current device and
+// hands that address to the existing decode path.  The lookup is repeated on
+// every call (after the first it is a table lookup that allocates nothing),
+// so an address never outlives the context it belongs to, e.g. across a
+// cudaDeviceReset.
+//
+// With lazy module loading (the CUDA default, CUDA_MODULE_LOADING=LAZY) the
+// array is committed on a device by the first lookup there, i.e. by the first
+// call on that device; with eager loading it is committed when the context is
+// created.  Either way it stays until the process exits.
 #include "pkv_internal.h"
 
 namespace pkv {
 namespace {
 
 constexpr size_t kStaticWorkspaceBytes = (size_t)PKV_STATIC_WORKSPACE_BYTES;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
 
-void* g_ws_ptr[kMaxDevices] = {nullptr};
-std::mutex g_ws_mu;
-
-// Device address of the static scratch on the current device (first call on a
-// device does the lookup); null on failure.
+// Device address of the static scratch on the current device; null on failure.
 void* static_workspace(pkv_status* st) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-        *st = fail(PKV_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess || !p) {
+        *st = fail(PKV_ECUDA, "cudaGetSymbolAddress(static workspace): %s", cudaGetErrorString(e));
         return nullptr;
     }
-    std::lock_guard<std::mutex> lk(g_ws_mu);
-    if (!g_ws_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_static_workspace);
-        if (e != cudaSuccess || !p) {
-            *st = fail(PKV_ECUDA, "cudaGetSymbolAddress(static workspace): %s", cudaGetErrorString(e));
-            return nullptr;
-        }
-        g_ws_ptr[dev] = p;
-    }
-    return g_ws_ptr[dev];
+    return p;
 }
 
 }  // namespace

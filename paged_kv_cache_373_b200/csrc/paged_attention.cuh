@@ -41,6 +41,7 @@ namespace pkv {
 constexpr int kTileTokens = 16;    // tokens per pipeline tile (32 for FP8 caches with 32-token blocks)
 constexpr int kHeadsPerUnit = 8;   // q heads served by one KV read (one mma N tile)
 constexpr int kMaxWarpsPerCta = 12; // workspace is sized for this many workers per CTA
+constexpr int kMaxCtas = 1 << 20;   // bound on num_ctas: every worker count (CTAs x warps) fits a grid dimension
 
 struct DecodeParams {
     void* out;

@@ -5,7 +5,6 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
-#include <mutex>
 
 #include "paged_attention.cuh"
 #include "pkv_internal.h"
@@ -17,10 +16,6 @@ __device__ int g_pkv_error;
 
 namespace {
 thread_local char g_msg[512] = "";
-constexpr int kMaxDevices = 64;
-int* g_err_ptr[kMaxDevices] = {nullptr};
-std::mutex g_err_mu;
-
 }  // namespace
 
 pkv_status fail(pkv_status st, const char* fmt, ...) {
@@ -41,15 +36,11 @@ int dtype_bytes(pkv_dtype d) {
 }
 
 int* device_error_word() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::lock_guard<std::mutex> lk(g_err_mu);
-    if (!g_err_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_pkv_error) != cudaSuccess) return nullptr;
-        g_err_ptr[dev] = static_cast<int*>(p);
-    }
-    return g_err_ptr[dev];
+    // looked up on every call (a table lookup once the module is loaded), so
+    // the address always belongs to the current device's current context
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_pkv_error) != cudaSuccess) return nullptr;
+    return static_cast<int*>(p);
 }
 
 static int default_ctas() {
@@ -67,7 +58,7 @@ struct WsLayout {
 static bool ws_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int num_ctas,
                       WsLayout* w) {
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return false;
-    if (head_dim <= 0 || num_ctas < 0) return false;
+    if (head_dim <= 0 || num_ctas < 0 || num_ctas > kMaxCtas) return false;
     const int g = num_heads / num_kv_heads;
     w->grid = num_ctas > 0 ? num_ctas : default_ctas();
     if (w->grid <= 0) return false;
@@ -113,7 +104,7 @@ pkv_status decode_prepare(DecodeParams* pp, DecodeLauncher* launch_out, int* gri
     if (max_blocks_per_seq <= 0 || (int64_t)max_blocks_per_seq * block_size > 0x7fffffffLL)
         return fail(PKV_EINVAL, "max_blocks_per_seq out of range");
     if (!std::isfinite(scale)) return fail(PKV_EINVAL, "scale must be finite");
-    if (num_ctas < 0) return fail(PKV_EINVAL, "num_ctas < 0");
+    if (num_ctas < 0 || num_ctas > kMaxCtas) return fail(PKV_EINVAL, "num_ctas %d outside [0, %d]", num_ctas, kMaxCtas);
     // dtype combination -> launcher
     DecodeLauncher launch = nullptr;
     if (cache_dtype == PKV_F32 && q_dtype == PKV_F32)
@@ -199,6 +190,33 @@ extern "C" pkv_status pkv_paged_attention_decode(void* out, const void* query, p
     return launch(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+extern "C" pkv_status pkv_decode_step_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                             pkv_dtype q_dtype, int max_blocks_per_seq,
+                                             int64_t num_cow_pairs, pkv_step_layout* l) {
+    if (!l) return fail(PKV_EINVAL, "null layout");
+    const int qb = dtype_bytes(q_dtype);
+    if (qb == 0) return fail(PKV_EINVAL, "q dtype");
+    if (num_seqs < 0 || num_heads < 0 || num_kv_heads < 0 || head_dim < 0 || max_blocks_per_seq < 0 ||
+        num_cow_pairs < 0)
+        return fail(PKV_EINVAL, "negative size");
+    const size_t S = (size_t)num_seqs;
+    size_t at = 0;
+    auto take = [&](size_t n) {
+        const size_t off = at;
+        at = (at + n + 255) & ~(size_t)255;
+        return off;
+    };
+    l->query = take(S * num_heads * head_dim * qb);
+    l->new_key = take(S * num_kv_heads * head_dim * qb);
+    l->new_value = take(S * num_kv_heads * head_dim * qb);
+    l->slot_mapping = take(S * sizeof(int64_t));
+    l->block_tables = take(S * max_blocks_per_seq * sizeof(int32_t));
+    l->seq_lens = take(S * sizeof(int32_t));
+    l->cow_pairs = take((size_t)num_cow_pairs * 2 * sizeof(int64_t));
+    l->total = at;
+    return PKV_OK;
+}
+
 extern "C" pkv_status pkv_decode_step_host(const pkv_decode_step_args* a, pkv_stream_t stream) {
     if (!a) return fail(PKV_EINVAL, "null args");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -208,42 +226,70 @@ extern "C" pkv_status pkv_decode_step_host(const pkv_decode_step_args* a, pkv_st
     if (qb == 0) return fail(PKV_EINVAL, "q dtype");
     const size_t q_bytes = (size_t)S * a->num_heads * a->head_dim * qb;
     const size_t kv_bytes = (size_t)S * a->num_kv_heads * a->head_dim * qb;
-    struct Cp { void* dst; const void* src; size_t n; };
-    const Cp h2d[] = {
-        {a->d_query, a->h_query, q_bytes},
-        {a->d_new_key, a->h_new_key, kv_bytes},
-        {a->d_new_value, a->h_new_value, kv_bytes},
-        {a->d_slot_mapping, a->h_slot_mapping, (size_t)S * sizeof(int64_t)},
-        {a->d_block_tables, a->h_block_tables, (size_t)S * a->max_blocks_per_seq * sizeof(int32_t)},
-        {a->d_seq_lens, a->h_seq_lens, (size_t)S * sizeof(int32_t)},
-        {a->d_cow_pairs, a->h_cow_pairs, (size_t)(a->num_cow_pairs > 0 ? a->num_cow_pairs : 0) * 2 * sizeof(int64_t)},
-    };
-    for (const Cp& c : h2d) {
-        if (c.n == 0) continue;
-        if (!c.dst || !c.src) return fail(PKV_EINVAL, "null staging or host buffer");
-        const cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, st);
-        if (e != cudaSuccess) return fail(PKV_ECUDA, "H2D copy: %s", cudaGetErrorString(e));
+    const int64_t npairs = a->num_cow_pairs > 0 ? a->num_cow_pairs : 0;
+    // device addresses of the step's inputs
+    const void* d_query = a->d_query;
+    const void* d_new_key = a->d_new_key;
+    const void* d_new_value = a->d_new_value;
+    const int64_t* d_slots = a->d_slot_mapping;
+    const int32_t* d_tables = a->d_block_tables;
+    const int32_t* d_lens = a->d_seq_lens;
+    const int64_t* d_pairs = a->d_cow_pairs;
+    if (a->h_packed) {
+        // one copy of the whole packed input buffer
+        pkv_step_layout l;
+        pkv_status s = pkv_decode_step_layout(S, a->num_heads, a->num_kv_heads, a->head_dim, a->q_dtype,
+                                              a->max_blocks_per_seq, npairs, &l);
+        if (s != PKV_OK) return s;
+        if (!a->d_packed || !aligned16(a->d_packed)) return fail(PKV_EINVAL, "d_packed null or not 16-byte aligned");
+        uint8_t* d = static_cast<uint8_t*>(a->d_packed);
+        if (l.total) {
+            const cudaError_t e = cudaMemcpyAsync(d, a->h_packed, l.total, cudaMemcpyHostToDevice, st);
+            if (e != cudaSuccess) return fail(PKV_ECUDA, "H2D copy: %s", cudaGetErrorString(e));
+        }
+        d_query = d + l.query;
+        d_new_key = d + l.new_key;
+        d_new_value = d + l.new_value;
+        d_slots = reinterpret_cast<const int64_t*>(d + l.slot_mapping);
+        d_tables = reinterpret_cast<const int32_t*>(d + l.block_tables);
+        d_lens = reinterpret_cast<const int32_t*>(d + l.seq_lens);
+        d_pairs = reinterpret_cast<const int64_t*>(d + l.cow_pairs);
+    } else {
+        struct Cp { const void* dst; const void* src; size_t n; };
+        const Cp h2d[] = {
+            {a->d_query, a->h_query, q_bytes},
+            {a->d_new_key, a->h_new_key, kv_bytes},
+            {a->d_new_value, a->h_new_value, kv_bytes},
+            {a->d_slot_mapping, a->h_slot_mapping, (size_t)S * sizeof(int64_t)},
+            {a->d_block_tables, a->h_block_tables, (size_t)S * a->max_blocks_per_seq * sizeof(int32_t)},
+            {a->d_seq_lens, a->h_seq_lens, (size_t)S * sizeof(int32_t)},
+            {a->d_cow_pairs, a->h_cow_pairs, (size_t)npairs * 2 * sizeof(int64_t)},
+        };
+        for (const Cp& c : h2d) {
+            if (c.n == 0) continue;
+            if (!c.dst || !c.src) return fail(PKV_EINVAL, "null staging or host buffer");
+            const cudaError_t e = cudaMemcpyAsync(const_cast<void*>(c.dst), c.src, c.n, cudaMemcpyHostToDevice, st);
+            if (e != cudaSuccess) return fail(PKV_ECUDA, "H2D copy: %s", cudaGetErrorString(e));
+        }
     }
     pkv_status s;
-    if (a->num_cow_pairs > 0) {
+    if (npairs > 0) {
         void* kcs[1] = {a->key_cache};
         void* vcs[1] = {a->value_cache};
         const size_t block_bytes = (size_t)a->block_size * a->num_kv_heads * a->head_dim *
                                    dtype_bytes(a->cache_dtype);
-        if ((s = pkv_copy_blocks(kcs, vcs, 1, a->d_cow_pairs, a->num_cow_pairs, a->num_blocks,
-                                 block_bytes, stream)) != PKV_OK)
+        if ((s = pkv_copy_blocks(kcs, vcs, 1, d_pairs, npairs, a->num_blocks, block_bytes, stream)) != PKV_OK)
             return s;
     }
-    if ((s = pkv_reshape_and_cache(a->d_new_key, a->d_new_value, a->q_dtype, a->key_cache,
-                                   a->value_cache, a->cache_dtype, a->d_slot_mapping, S,
-                                   a->num_blocks, a->block_size, a->num_kv_heads, a->head_dim,
-                                   a->k_scale, a->v_scale, stream)) != PKV_OK)
+    if ((s = pkv_reshape_and_cache(d_new_key, d_new_value, a->q_dtype, a->key_cache, a->value_cache,
+                                   a->cache_dtype, d_slots, S, a->num_blocks, a->block_size,
+                                   a->num_kv_heads, a->head_dim, a->k_scale, a->v_scale, stream)) != PKV_OK)
         return s;
-    if ((s = pkv_paged_attention_decode(a->d_out, a->d_query, a->q_dtype, a->key_cache, a->value_cache,
-                                        a->cache_dtype, a->d_block_tables, a->max_blocks_per_seq,
-                                        a->d_seq_lens, S, a->num_heads, a->num_kv_heads, a->head_dim,
-                                        a->block_size, a->num_blocks, a->scale, a->k_scale, a->v_scale,
-                                        a->workspace, a->workspace_bytes, a->num_ctas, stream)) != PKV_OK)
+    if ((s = pkv_paged_attention_decode(a->d_out, d_query, a->q_dtype, a->key_cache, a->value_cache,
+                                        a->cache_dtype, d_tables, a->max_blocks_per_seq, d_lens, S,
+                                        a->num_heads, a->num_kv_heads, a->head_dim, a->block_size,
+                                        a->num_blocks, a->scale, a->k_scale, a->v_scale, a->workspace,
+                                        a->workspace_bytes, a->num_ctas, stream)) != PKV_OK)
         return s;
     if (q_bytes) {
         if (!a->h_out || !a->d_out) return fail(PKV_EINVAL, "null output buffer");

@@ -81,6 +81,8 @@ struct PrefillParams {
     int64_t num_blocks;
     int num_seqs, num_heads, num_kv_heads, g, mbps, bs;
     float scale_log2;
+    uint64_t wait_ns;  // limit of every wait (kPfWaitNs)
+    int stop_tile;     // < 0; a test of the timeout path sets k >= 0: K/V tiles k, k+1, ... are never copied
 };
 
 // Byte offset of 16-byte chunk c of row r in a [rows][cols] 16-bit tile kept
@@ -142,9 +144,9 @@ __device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
 __device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
 }
-// Wait for the mbarrier phase `parity`.  False after 0.2 s of wall-clock time
-// (the abort flag is then raised) or as soon as another role raised it.
-__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, volatile int* abort) {
+// Wait for the mbarrier phase `parity`.  False after `limit_ns` of wall-clock
+// time (the abort flag is then raised) or as soon as another role raised it.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
         uint32_t ok;
@@ -157,7 +159,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, volati
             const uint64_t now = global_ns();
             if (t0 == 0) {
                 t0 = now;
-            } else if (now - t0 > kPfWaitNs) {
+            } else if (now - t0 > limit_ns) {
                 if (abort) *abort = 1;
                 return false;
             }
@@ -384,7 +386,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
 #pragma unroll 1
             for (int i = 0; i < ntiles; ++i) {
                 const int kt = kt0 + i * kstep;
-                bool ok = !failed && mbar_wait(bar(kBarS + X), i & 1, abort);
+                bool ok = !failed && mbar_wait(bar(kBarS + X), i & 1, abort, p.wait_ns);
                 ok = __all_sync(kFull, ok);
                 float sc[kPfTok / 2];
                 float pm = -INFINITY;
@@ -424,7 +426,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                 }
                 l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
                 if (i > 0) {  // P V of the previous tile done: its P buffer is free, O is settled
-                    ok = mbar_wait(bar(kBarO + X), (i - 1) & 1, abort);
+                    ok = mbar_wait(bar(kBarO + X), (i - 1) & 1, abort, p.wait_ns);
                     ok = __all_sync(kFull, ok);
                     if (ok) {
                         tc_after_sync();
@@ -466,10 +468,10 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
             }
             // ---- the last P V, then normalise (the halves' sums combined; a
             // split unit also merges group 1's partial result) and store
-            bool ok = !failed && (ntiles == 0 || mbar_wait(bar(kBarO + X), (ntiles - 1) & 1, abort));
+            bool ok = !failed && (ntiles == 0 || mbar_wait(bar(kBarO + X), (ntiles - 1) & 1, abort, p.wait_ns));
             // (group 1's last P V, read in the merge: after group 0's own last
             // one, at most that phase of group 1 is outstanding)
-            if (split && X == 0 && nkv > 1) ok = ok && mbar_wait(bar(kBarO + 1), ((nkv >> 1) - 1) & 1, abort);
+            if (split && X == 0 && nkv > 1) ok = ok && mbar_wait(bar(kBarO + 1), ((nkv >> 1) - 1) & 1, abort, p.wait_ns);
             ok = __all_sync(kFull, ok);
             xsum[X][half][row] = l;
             if (split && X == 1 && half == 0) xref[row] = mref;
@@ -547,11 +549,11 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                                   (acc || part > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(bar(kBarO + X));
             };
-            bool ok = mbar_wait(bar(kBarQ), 0, abort);
+            bool ok = mbar_wait(bar(kBarQ), 0, abort, p.wait_ns);
             if (!split) {
                 // paired units: every tile serves both; per tile
                 // O_0 += P_0 V, S_0' = Q_0 K'^T, O_1 += P_1 V, S_1' = Q_1 K'^T
-                ok = ok && mbar_wait(bar(kBarKFull), 0, abort);
+                ok = ok && mbar_wait(bar(kBarKFull), 0, abort, p.wait_ns);
                 if (ok) {
                     tc_after_sync();
                     issue_s(0, 0);
@@ -562,22 +564,22 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                 for (int kt = 0; ok && kt < nkv; ++kt) {
                     const int st = stg(kt), sn = stg(kt + 1);
                     const bool a1 = kt < U1.nkv, a1n = kt + 1 < U1.nkv;
-                    ok = mbar_wait(bar(kBarVFull + st), pass(kt), abort) &&
-                         (kt != nkv - 1 || !need_fix || mbar_wait(bar(kBarVFix), 0, abort)) &&
-                         mbar_wait(bar(kBarP), kt & 1, abort);
+                    ok = mbar_wait(bar(kBarVFull + st), pass(kt), abort, p.wait_ns) &&
+                         (kt != nkv - 1 || !need_fix || mbar_wait(bar(kBarVFix), 0, abort, p.wait_ns)) &&
+                         mbar_wait(bar(kBarP), kt & 1, abort, p.wait_ns);
                     if (!ok) break;
                     tc_after_sync();
                     issue_pv(0, st, kt > 0);
                     if (!a1) tc_commit(bar(kBarVEmpty + st));
                     if (kt + 1 < nkv) {
-                        ok = mbar_wait(bar(kBarKFull + sn), pass(kt + 1), abort);
+                        ok = mbar_wait(bar(kBarKFull + sn), pass(kt + 1), abort, p.wait_ns);
                         if (!ok) break;
                         tc_after_sync();
                         issue_s(0, sn);
                         if (!a1n) tc_commit(bar(kBarKEmpty + sn));
                     }
                     if (a1) {
-                        ok = mbar_wait(bar(kBarP + 1), kt & 1, abort);
+                        ok = mbar_wait(bar(kBarP + 1), kt & 1, abort, p.wait_ns);
                         if (!ok) break;
                         tc_after_sync();
                         issue_pv(1, st, kt > 0);
@@ -593,7 +595,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                 // O_0 += P_0 V_2i, S_0 = Q K_2i+2^T, O_1 += P_1 V_2i+1, S_1 = Q K_2i+3^T
 #pragma unroll 1
                 for (int X = 0; ok && X < 2 && X < nkv; ++X) {
-                    ok = mbar_wait(bar(kBarKFull + stg(X)), pass(X), abort);
+                    ok = mbar_wait(bar(kBarKFull + stg(X)), pass(X), abort, p.wait_ns);
                     if (!ok) break;
                     tc_after_sync();
                     issue_s(X, stg(X));
@@ -605,15 +607,15 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                     for (int X = 0; X < 2; ++X) {
                         const int kt = 2 * i + X;
                         if (kt >= nkv) break;
-                        ok = mbar_wait(bar(kBarVFull + stg(kt)), pass(kt), abort) &&
-                             (kt != nkv - 1 || !need_fix || mbar_wait(bar(kBarVFix), 0, abort)) &&
-                             mbar_wait(bar(kBarP + X), i & 1, abort);
+                        ok = mbar_wait(bar(kBarVFull + stg(kt)), pass(kt), abort, p.wait_ns) &&
+                             (kt != nkv - 1 || !need_fix || mbar_wait(bar(kBarVFix), 0, abort, p.wait_ns)) &&
+                             mbar_wait(bar(kBarP + X), i & 1, abort, p.wait_ns);
                         if (!ok) break;
                         tc_after_sync();
                         issue_pv(X, stg(kt), i > 0);
                         tc_commit(bar(kBarVEmpty + stg(kt)));
                         if (kt + 2 < nkv) {
-                            ok = mbar_wait(bar(kBarKFull + stg(kt + 2)), pass(kt + 2), abort);
+                            ok = mbar_wait(bar(kBarKFull + stg(kt + 2)), pass(kt + 2), abort, p.wait_ns);
                             if (!ok) break;
                             tc_after_sync();
                             issue_s(X, stg(kt + 2));
@@ -623,7 +625,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                 }
             }
             tc_commit(bar(kBarDrain));  // every product issued has finished before tensor memory is freed
-            mbar_wait(bar(kBarDrain), 0, nullptr);
+            mbar_wait(bar(kBarDrain), 0, nullptr, p.wait_ns);
         }
         __syncwarp();
     } else if (warp == kPfLoadWarp) {
@@ -645,8 +647,9 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
             const int32_t* trow = p.tables + (int64_t)s * p.mbps;
             const int lg_bs = p.bs == 16 ? 4 : 5;
             const int nblk = kPfTok >> lg_bs;
+            const int kt_end = p.stop_tile < 0 ? nkv : min(nkv, p.stop_tile);
 #pragma unroll 1
-            for (int kt = 0; kt < nkv; ++kt) {
+            for (int kt = 0; kt < kt_end; ++kt) {
                 const int st = stg(kt);
                 int phys[kPfTok / 16];
                 int nb = 0;
@@ -665,7 +668,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                     }
                 }
                 const uint32_t bytes = (uint32_t)(nb * p.bs * D * 2);
-                if (kt >= kPfStages && !(ok = mbar_wait(bar(kBarKEmpty + st), pass(kt - kPfStages), abort))) break;
+                if (kt >= kPfStages && !(ok = mbar_wait(bar(kBarKEmpty + st), pass(kt - kPfStages), abort, p.wait_ns))) break;
                 mbar_expect_tx(bar(kBarKFull + st), bytes);
 #pragma unroll 1
                 for (int jb = 0; jb < nb; ++jb)
@@ -674,7 +677,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                         tma_load3(smem_u32(ksm + st * SM::kTile + cb * kPfTok * 128 + jb * p.bs * 128), &tmap_k,
                                   cb * 64, kh, phys[jb] * p.bs, bar(kBarKFull + st));
                 ++nk[st];
-                if (kt >= kPfStages && !(ok = mbar_wait(bar(kBarVEmpty + st), pass(kt - kPfStages), abort))) break;
+                if (kt >= kPfStages && !(ok = mbar_wait(bar(kBarVEmpty + st), pass(kt - kPfStages), abort, p.wait_ns))) break;
                 mbar_expect_tx(bar(kBarVFull + st), bytes);
 #pragma unroll 1
                 for (int jb = 0; jb < nb; ++jb)
@@ -684,11 +687,12 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                                   cb * 64, kh, phys[jb] * p.bs, bar(kBarVFull + st));
                 ++nv[st];
             }
+            if (kt_end < nkv) ok = false;  // (timeout test) the other roles wait for the missing tiles
             if (!ok) {  // let the copies in flight land before the CTA ends
-                mbar_wait(bar(kBarQ), 0, nullptr);
+                mbar_wait(bar(kBarQ), 0, nullptr, p.wait_ns);
                 for (int st = 0; st < kPfStages; ++st) {
-                    if (nk[st]) mbar_wait(bar(kBarKFull + st), (nk[st] - 1) & 1, nullptr);
-                    if (nv[st]) mbar_wait(bar(kBarVFull + st), (nv[st] - 1) & 1, nullptr);
+                    if (nk[st]) mbar_wait(bar(kBarKFull + st), (nk[st] - 1) & 1, nullptr, p.wait_ns);
+                    if (nv[st]) mbar_wait(bar(kBarVFull + st), (nv[st] - 1) & 1, nullptr, p.wait_ns);
                 }
             }
         }
@@ -696,7 +700,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         ok = __shfl_sync(kFull, ok, 0);
         if (need_fix) {  // zero the last V tile's rows at and past the unit's end
             const int kl = nkv - 1, st = stg(kl);
-            bool fine = ok && mbar_wait(bar(kBarVFull + st), pass(kl), abort);
+            bool fine = ok && mbar_wait(bar(kBarVFull + st), pass(kl), abort, p.wait_ns);
             fine = __all_sync(kFull, fine);
             if (fine) {
                 const int r0 = U0.kv_end - kl * kPfTok;
@@ -779,10 +783,24 @@ pkv_status launch_prefill(const PrefillParams& p, const void* query, const void*
     return PKV_OK;
 }
 
+// A timeout test armed by pkv_testing_prefill_timeout for the next
+// pkv_paged_prefill call on this thread (stop_tile < 0: not armed).
+thread_local int t_test_stop_tile = -1;
+thread_local uint64_t t_test_wait_ns = 0;
+
 }  // namespace
 }  // namespace pkv
 
 using namespace pkv;
+
+extern "C" pkv_status pkv_testing_prefill_timeout(int stop_tile, uint64_t wait_ns) {
+    if (stop_tile < 0) return fail(PKV_EINVAL, "stop_tile < 0");
+    if (wait_ns < 100000ull || wait_ns > kPfWaitNs)
+        return fail(PKV_EINVAL, "wait_ns outside [1e5, %llu]", (unsigned long long)kPfWaitNs);
+    t_test_stop_tile = stop_tile;
+    t_test_wait_ns = wait_ns;
+    return PKV_OK;
+}
 
 extern "C" pkv_status pkv_paged_prefill(void* out, const void* query, pkv_dtype q_dtype,
                                         const void* key_cache, const void* value_cache,
@@ -792,6 +810,11 @@ extern "C" pkv_status pkv_paged_prefill(void* out, const void* query, pkv_dtype 
                                         int64_t num_query_tokens, int num_heads, int num_kv_heads,
                                         int head_dim, int block_size, int64_t num_blocks, float scale,
                                         pkv_stream_t stream) {
+    // a timeout test applies to this call only, whatever it returns
+    const int stop_tile = t_test_stop_tile;
+    const uint64_t wait_ns = t_test_wait_ns ? t_test_wait_ns : kPfWaitNs;
+    t_test_stop_tile = -1;
+    t_test_wait_ns = 0;
     if (num_seqs < 0 || num_query_tokens < 0) return fail(PKV_EINVAL, "negative size");
     if (num_kv_heads <= 0 || num_heads <= 0 || num_heads % num_kv_heads)
         return fail(PKV_EINVAL, "num_heads must be a positive multiple of num_kv_heads");
@@ -824,6 +847,8 @@ extern "C" pkv_status pkv_paged_prefill(void* out, const void* query, pkv_dtype 
     p.mbps = max_blocks_per_seq;
     p.bs = block_size;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.wait_ns = wait_ns;
+    p.stop_tile = stop_tile;
     // unit pairs: sum_s ceil(ceil(C_s g / 128) / 2) <= ceil(T g / 256) + S
     const int64_t pairs = (num_query_tokens * g + 2 * kPfRows - 1) / (2 * kPfRows) + num_seqs;
     const int64_t grid = pairs * num_kv_heads;

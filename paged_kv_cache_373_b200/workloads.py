@@ -17,6 +17,8 @@ length mixes instead:
   cfg5  prefix sharing with copy-on-write: 16 prompts x 8 samples, a
         3000-token shared prefix (187 full blocks + one 8-token block, reference
         count 8), per-sample tails U[32,512], 32/8 heads, D=128, bs=16, bf16
+  short 2048 seqs of U[1,64] tokens, cfg3's shapes (a large-batch test case,
+        not one of the five configurations)
 
 Every sequence's newest token (position seq_len-1) is the decode step's new
 token: its K/V are in ``new_key``/``new_value`` and its slot in
@@ -455,7 +457,17 @@ def prefill_config(budget: int = 8192) -> PrefillWorkload:
                          torch.bfloat16, _seed(6) + budget)
 
 
-CONFIGS = {1: config1, 2: config2, 3: config3, 4: config4, 5: config5}
+def short_batch(num_seqs: int = 2048, lo: int = 1, hi: int = 64) -> DecodeWorkload:
+    """A large batch of short sequences (Llama-3-8B GQA layer shapes, bf16):
+    lengths U[lo, hi], so the per-sequence work (length scans, unit starts,
+    merges) weighs more than in the five configurations."""
+    gen = torch.Generator().manual_seed(_seed(7) * 1000)
+    lens = torch.randint(lo, hi + 1, (num_seqs,), generator=gen).tolist()
+    return build_decode(f"short_llama3_8b_gqa_bf16_b{num_seqs}", lens, 32, 8, 128, 16,
+                        torch.bfloat16, torch.bfloat16, _seed(7))
+
+
+CONFIGS = {1: config1, 2: config2, 3: config3, 4: config4, 5: config5, 7: short_batch}
 
 
 def make_config(cfg: int, **kw) -> DecodeWorkload:

@@ -10,6 +10,7 @@ import torch
 
 import oracle
 import paged_kv_cache_373_b200 as pkv
+from paged_kv_cache_373_b200 import device_inputs
 from paged_kv_cache_373_b200 import workloads as W
 
 TOL_16 = 2e-3   # f16 / bf16 / f32 caches, fp32 accumulation (max-abs vs fp64)
@@ -30,31 +31,11 @@ def half_ulp(x: np.ndarray, dtype: torch.dtype) -> np.ndarray:
 
 def fp8_pool_gpu(wl, dev="cuda"):
     """Quantise the FP8 pool sources on the GPU with reshape_and_cache (all slots)."""
-    NB, bs, Hkv, D = wl.key_src.shape
-    kc = torch.empty((NB, bs, Hkv, D), dtype=torch.uint8, device=dev)
-    vc = torch.empty_like(kc)
-    ks = torch.tensor([wl.k_scale], dtype=torch.float32, device=dev)
-    vs = torch.tensor([wl.v_scale], dtype=torch.float32, device=dev)
-    rows = NB * bs
-    step = max(1, (1 << 28) // (Hkv * D * 2))          # bounded staging (~256 MB of bf16)
-    for r0 in range(0, rows, step):
-        r1 = min(rows, r0 + step)
-        k = wl.key_src.reshape(rows, Hkv, D)[r0:r1].to(dev)
-        v = wl.value_src.reshape(rows, Hkv, D)[r0:r1].to(dev)
-        slots = torch.arange(r0, r1, dtype=torch.int64, device=dev)
-        pkv.reshape_and_cache(k, v, kc, vc, slots, ks, vs)
-    return kc, vc, ks, vs
+    return device_inputs.fp8_pool(wl, dev)
 
 
 def gpu_inputs(wl, dev="cuda"):
-    if wl.is_fp8:
-        kc, vc, ks, vs = fp8_pool_gpu(wl, dev)
-    else:
-        kc, vc = wl.key_cache.to(dev), wl.value_cache.to(dev)
-        ks = vs = None
-    return dict(kc=kc, vc=vc, ks=ks, vs=vs, q=wl.query.to(dev), tables=wl.block_tables.to(dev),
-                lens=wl.seq_lens.to(dev), nk=wl.new_key.to(dev), nv=wl.new_value.to(dev),
-                slots=wl.slot_mapping.to(dev), pairs=wl.cow_pairs.to(dev))
+    return device_inputs.decode_inputs(wl, dev)
 
 
 def gpu_step(wl, g=None, num_ctas: int = 0, dev="cuda"):

@@ -92,11 +92,42 @@ def test_host_validation_without_gpu(L):
 
 def test_decode_step_struct_layout():
     # pkv_decode_step_args: 6 ints, int64, 2 enums, float, int, 7 pointers, int64,
-    # 9 pointers, 5 pointers, size_t
-    assert ctypes.sizeof(pkv.DecodeStepArgs) == 232
+    # 9 pointers, 5 pointers, size_t, 2 pointers (packed inputs)
+    assert ctypes.sizeof(pkv.DecodeStepArgs) == 248
     assert pkv.DecodeStepArgs.num_blocks.offset == 24
     assert pkv.DecodeStepArgs.h_query.offset == 48
     assert pkv.DecodeStepArgs.workspace_bytes.offset == 224
+    assert pkv.DecodeStepArgs.h_packed.offset == 232 and pkv.DecodeStepArgs.d_packed.offset == 240
+
+
+def test_decode_step_layout_offsets(L):
+    # cfg3 shapes: S 256, Hq 32, Hkv 8, D 128, bf16, 512 table entries per sequence
+    lay = pkv.decode_step_layout(256, 32, 8, 128, pkv.PKV_BF16, 512, 0)
+    sizes = [256 * 32 * 128 * 2, 256 * 8 * 128 * 2, 256 * 8 * 128 * 2, 256 * 8, 256 * 512 * 4, 256 * 4, 0]
+    offs = [lay.query, lay.new_key, lay.new_value, lay.slot_mapping, lay.block_tables, lay.seq_lens,
+            lay.cow_pairs]
+    at = 0
+    for off, n in zip(offs, sizes):
+        assert off == at and off % 256 == 0
+        at = (at + n + 255) // 256 * 256
+    assert lay.total == at
+    # copy-on-write pairs and odd sizes stay 256-byte aligned and disjoint
+    lay = pkv.decode_step_layout(3, 6, 2, 64, pkv.PKV_F32, 5, 7)
+    offs = [lay.query, lay.new_key, lay.new_value, lay.slot_mapping, lay.block_tables, lay.seq_lens,
+            lay.cow_pairs, lay.total]
+    assert all(o % 256 == 0 for o in offs) and offs == sorted(offs)
+    assert lay.total - lay.cow_pairs >= 7 * 16
+    with pytest.raises(pkv.PkvError):
+        pkv.decode_step_layout(-1, 6, 2, 64, pkv.PKV_F32, 5, 0)
+    with pytest.raises(pkv.PkvError):
+        pkv.decode_step_layout(3, 6, 2, 64, 9, 5, 0)
+
+
+def test_num_ctas_bound(L):
+    assert pkv.paged_attention_workspace_bytes(4, 8, 2, 128, 1 << 20) > 0
+    assert pkv.paged_attention_workspace_bytes(4, 8, 2, 128, (1 << 20) + 1) == 0
+    assert _decode(L, num_ctas=(1 << 20) + 1) == pkv.PKV_EINVAL
+    assert b"num_ctas" in L.pkv_last_error_message()
 
 
 def _prefill(L, **kw):
@@ -138,3 +169,11 @@ def test_swap_host_validation_without_gpu(L):
     assert swap(block_bytes=0) == pkv.PKV_EINVAL
     assert swap(pairs=0) == pkv.PKV_OK                                     # nothing to do
     assert swap() == pkv.PKV_EINVAL                                        # null pointers
+
+
+def test_prefill_timeout_hook_validation(L):
+    assert L.pkv_testing_prefill_timeout(-1, 1_000_000) == pkv.PKV_EINVAL
+    assert L.pkv_testing_prefill_timeout(0, 10) == pkv.PKV_EINVAL            # below 0.1 ms
+    assert L.pkv_testing_prefill_timeout(0, 10**9) == pkv.PKV_EINVAL         # above the normal 0.2 s
+    assert L.pkv_testing_prefill_timeout(0, 1_000_000) == pkv.PKV_OK
+    assert _prefill(L, num_seqs=0) == pkv.PKV_OK                              # consumes (disarms) it

@@ -192,3 +192,87 @@ def test_full_config_sampled_parity(cfg):
     seqs = _sample(wl, 6, cfg)
     compare(out, oracle_step(wl, seqs=seqs), wl, seqs=seqs)
     assert torch.isfinite(out.float()).all()
+
+
+def _step_args(wl, g, ws, num_ctas):
+    a = pkv.DecodeStepArgs()
+    a.num_seqs, a.num_heads, a.num_kv_heads = wl.num_seqs, wl.num_heads, wl.num_kv_heads
+    a.head_dim, a.block_size, a.max_blocks_per_seq = wl.head_dim, wl.block_size, wl.max_blocks_per_seq
+    a.num_blocks = wl.num_blocks
+    a.q_dtype = pkv.dtype_code(wl.query)
+    a.cache_dtype = pkv.PKV_FP8_E4M3 if wl.is_fp8 else a.q_dtype
+    a.scale, a.num_ctas = wl.scale, num_ctas
+    a.num_cow_pairs = int(wl.cow_pairs.shape[0])
+    a.key_cache, a.value_cache = g["kc"].data_ptr(), g["vc"].data_ptr()
+    a.k_scale = g["ks"].data_ptr() if g["ks"] is not None else None
+    a.v_scale = g["vs"].data_ptr() if g["vs"] is not None else None
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    return a
+
+
+@pytest.mark.parametrize("name", ["cfg5_mini", "fp8_g8_bs32_qbf16", "bf16_gqa4_d128"])
+def test_decode_step_host_packed_and_unpacked(name):
+    """pkv_decode_step_host from host buffers, one copy per input and packed
+    (one copy for all inputs), gives the device path's bits."""
+    wl = SMALL[name]()
+    ref, err, g = gpu_step(wl, num_ctas=37)
+    assert err == 0
+    ws = pkv.alloc_workspace(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, 37)
+    src = dict(q=wl.query, nk=wl.new_key.to(wl.q_dtype), nv=wl.new_value.to(wl.q_dtype),
+               slots=wl.slot_mapping, tables=wl.block_tables, lens=wl.seq_lens, pairs=wl.cow_pairs)
+    # one copy per input
+    h = {k: v.contiguous().pin_memory() for k, v in src.items()}
+    d = {k: torch.empty_like(v, device="cuda") for k, v in src.items()}
+    h_out = torch.full_like(wl.query, float("nan")).pin_memory()
+    d_out = torch.empty_like(ref)
+    a = _step_args(wl, g, ws, 37)
+    a.h_query, a.h_new_key, a.h_new_value = h["q"].data_ptr(), h["nk"].data_ptr(), h["nv"].data_ptr()
+    a.h_slot_mapping, a.h_block_tables = h["slots"].data_ptr(), h["tables"].data_ptr()
+    a.h_seq_lens, a.h_cow_pairs = h["lens"].data_ptr(), h["pairs"].data_ptr()
+    a.d_query, a.d_new_key, a.d_new_value = d["q"].data_ptr(), d["nk"].data_ptr(), d["nv"].data_ptr()
+    a.d_slot_mapping, a.d_block_tables = d["slots"].data_ptr(), d["tables"].data_ptr()
+    a.d_seq_lens, a.d_cow_pairs = d["lens"].data_ptr(), d["pairs"].data_ptr()
+    a.h_out, a.d_out = h_out.data_ptr(), d_out.data_ptr()
+    pkv.decode_step_host(a)
+    assert pkv.get_device_error() == 0
+    assert torch.equal(h_out.view(-1).view(torch.uint8), ref.cpu().view(-1).view(torch.uint8))
+    # packed: every input in one pinned buffer at the layout's offsets
+    lay = pkv.decode_step_layout(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim,
+                                 a.q_dtype, wl.max_blocks_per_seq, a.num_cow_pairs)
+    hb = torch.zeros(lay.total, dtype=torch.uint8).pin_memory()
+    for key, off in (("q", lay.query), ("nk", lay.new_key), ("nv", lay.new_value),
+                     ("slots", lay.slot_mapping), ("tables", lay.block_tables),
+                     ("lens", lay.seq_lens), ("pairs", lay.cow_pairs)):
+        b = src[key].contiguous().view(-1).view(torch.uint8)
+        hb[off:off + b.numel()] = b
+    db = torch.empty(lay.total, dtype=torch.uint8, device="cuda")
+    h_out2 = torch.full_like(wl.query, float("nan")).pin_memory()
+    p = _step_args(wl, g, ws, 37)
+    p.h_packed, p.d_packed = hb.data_ptr(), db.data_ptr()
+    d_out2 = torch.empty_like(ref)
+    p.h_out, p.d_out = h_out2.data_ptr(), d_out2.data_ptr()
+    pkv.decode_step_host(p)
+    assert pkv.get_device_error() == 0
+    assert torch.equal(h_out2.view(-1).view(torch.uint8), ref.cpu().view(-1).view(torch.uint8))
+    compare(h_out2, oracle_step(wl), wl)
+
+
+def test_many_short_sequences():
+    """2048 sequences of 1..64 tokens (plus empty ones): every warp's length
+    scans cover the whole batch and the merge grid sees many unit boundaries."""
+    wl = W.short_batch()
+    lens = wl.seq_lens.clone()
+    out, err, _ = gpu_step(wl)
+    assert err == 0
+    compare(out, oracle_step(wl), wl)
+    for num_ctas in (1, 7, 300):
+        out2, err2, _ = gpu_step(wl, num_ctas=num_ctas)
+        assert err2 == 0
+        compare(out2, oracle_step(wl), wl)
+    # a sprinkle of empty sequences in a large batch
+    wl0 = W.build_decode("short_with_empty", [0 if i % 97 == 3 else int(L) for i, L in enumerate(lens)],
+                         32, 8, 128, 16, torch.bfloat16, torch.bfloat16, seed=62)
+    out3, err3, _ = gpu_step(wl0)
+    assert err3 == 0
+    compare(out3, oracle_step(wl0), wl0)
+    assert float(out3[3].abs().max()) == 0.0

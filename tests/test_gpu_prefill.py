@@ -170,3 +170,24 @@ def test_bad_lengths_and_block_ids_are_flagged():
                           torch.zeros(4, 16, 2, 64, dtype=torch.float16, device="cuda"),
                           torch.zeros(4, 16, 2, 64, dtype=torch.float16, device="cuda"),
                           wl.block_tables.cuda(), wl.seq_lens.cuda(), wl.query_start.cuda(), 0.125)
+
+
+@pytest.mark.parametrize("stop_tile", [0, 2])
+def test_bounded_waits_run_out_then_the_context_recovers(stop_tile):
+    """A test hook makes every CTA's copy lane stop before K/V tile `stop_tile`
+    (after the q rows), so the other roles' bounded waits (1 ms here) run out:
+    the call sets PKV_DEVERR_TIMEOUT and each CTA drains what it issued and
+    frees its tensor memory.  The next, normal call on the same context -- its
+    CTAs allocate the same tensor-memory columns on the same SMs -- completes
+    and matches the oracle."""
+    wl = W.build_prefill("timeout", [0, 300, 1000], [200, 64, 1], 16, 8, 128, 16, torch.bfloat16, seed=23)
+    L = pkv.lib()
+    assert L.pkv_testing_prefill_timeout(stop_tile, 1_000_000) == pkv.PKV_OK
+    out, err, kc, vc = gpu_prefill(wl)
+    assert err & pkv.DEVERR_TIMEOUT, f"device error word {err:#x}"
+    assert err & ~pkv.DEVERR_TIMEOUT == 0
+    out2, err2, _, _ = gpu_prefill(wl, kc, vc)       # disarmed after one call
+    assert err2 == 0
+    kh, vh = oracle_caches(wl)
+    ref = oracle.paged_prefill(wl.query, kh, vh, wl.block_tables, wl.seq_lens, wl.query_start, wl.scale)
+    check(out2, ref, torch.bfloat16)

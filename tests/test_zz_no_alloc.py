@@ -75,3 +75,29 @@ def test_noalloc_rejects_oversize_request():
         wl.num_blocks, 0.1, None, None, 0, None)
     assert st == pkv.PKV_EINVAL
     assert b"static scratch" in pkv.lib().pkv_last_error_message()
+
+
+def test_noalloc_warmup_then_no_device_allocation():
+    """The set-up the header asks for: one num_seqs = 0 call per device (it
+    commits the static scratch under lazy module loading); after it, decode
+    calls leave the device's free memory unchanged."""
+    wl = W.build_decode("noalloc_mem", [3, 90, 700, 1600], 32, 8, 128, 16, torch.bfloat16,
+                        torch.bfloat16, seed=55)
+    ref, err, g = gpu_step(wl)                       # loads the decode kernels, allocates the inputs
+    assert err == 0
+    NB, bs, Hkv, D = g["kc"].shape
+    st = pkv.lib().pkv_paged_attention_decode_noalloc(
+        None, None, pkv.PKV_BF16, None, None, pkv.PKV_BF16, None, g["tables"].shape[1], None, 0,
+        32, Hkv, D, bs, NB, wl.scale, None, None, 0, torch.cuda.current_stream().cuda_stream)
+    assert st == pkv.PKV_OK
+    outs = [torch.empty_like(ref) for _ in range(2)]
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for out in outs:
+        assert _noalloc(wl, g, out) == pkv.PKV_OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, f"device free memory changed by {free0 - free1} bytes"
+    assert pkv.get_device_error() == 0
+    for out in outs:
+        compare(out, ref.double().cpu().numpy(), wl)
