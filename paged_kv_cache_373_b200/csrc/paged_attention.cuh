@@ -87,44 +87,80 @@ struct Lens {
     const int32_t* len;
     const int32_t* start;
     int S, units, cap;
-    __device__ __forceinline__ int first(int s) const {
+    // raw seq_lens / start entries of sequence s (start 0 when kStart is false)
+    __device__ __forceinline__ int raw_len(int s) const { return __ldg(len + s); }
+    __device__ __forceinline__ int raw_start(int s) const {
+        if constexpr (!kStart) return 0;
+        else return __ldg(start + s);
+    }
+    // first attended token and attended length from the raw entries
+    __device__ __forceinline__ int first_of(int st) const { return (kStart && st > 0) ? st : 0; }
+    __device__ __forceinline__ int eff_of(int L, int st) const {
+        const int Lc = clamp_len(L, cap);
         if constexpr (!kStart) {
-            return 0;
+            return Lc;
         } else {
-            const int st = __ldg(start + s);
-            return st < 0 ? 0 : st;
+            const int f = first_of(st);
+            return f >= Lc ? 0 : Lc - f;
         }
     }
-    __device__ __forceinline__ int full(int s) const { return clamp_len(__ldg(len + s), cap); }
-    // attended length (tokens after the start)
-    __device__ __forceinline__ int eff(int s) const {
-        if constexpr (!kStart) {
-            return full(s);
-        } else {
-            const int L = full(s), st = first(s);
-            return st >= L ? 0 : L - st;
-        }
-    }
+    __device__ __forceinline__ int first(int s) const { return first_of(raw_start(s)); }
+    __device__ __forceinline__ int eff(int s) const { return eff_of(raw_len(s), raw_start(s)); }
 };
 template <int TT>
 __device__ __forceinline__ int ntiles_of(int L) { return (L + TT - 1) / TT; }
 
-// Warp-collective: total tiles W = units_per_seq * sum_s ceil(L_s / 16);
+// Entries [s0, s0 + E) of an int32 array (0 past n): 16-byte loads when the
+// run is whole and aligned, else one load per entry; all in flight together.
+template <int E>
+__device__ __forceinline__ void load_run(const int32_t* a, int s0, int n, int (&v)[E]) {
+    static_assert(E % 4 == 0, "whole 16-byte loads");
+    if (s0 + E <= n && (reinterpret_cast<uintptr_t>(a + s0) & 15) == 0) {
+#pragma unroll
+        for (int k = 0; k < E; k += 4) {
+            const int4 x = __ldg(reinterpret_cast<const int4*>(a + s0 + k));
+            v[k] = x.x; v[k + 1] = x.y; v[k + 2] = x.z; v[k + 3] = x.w;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < E; ++k) v[k] = (s0 + k < n) ? __ldg(a + s0 + k) : 0;
+    }
+}
+
+// Sequences per lane in one round of the warp-wide length scans (32 x 32 =
+// 1024 sequences per round: one round of loads for batches up to 1024).
+constexpr int kScanPerLane = 32;
+
+// Raw lengths (and starts) of the lane's sequences of the round at s0.
+template <class LN>
+__device__ __forceinline__ void load_lens(const LN& ln, int s0, int (&v)[kScanPerLane], int (&st)[kScanPerLane]) {
+    load_run<kScanPerLane>(ln.len, s0, ln.S, v);
+    if constexpr (LN::kHasStart) {
+        load_run<kScanPerLane>(ln.start, s0, ln.S, st);
+    } else {
+#pragma unroll
+        for (int k = 0; k < kScanPerLane; ++k) st[k] = 0;
+    }
+}
+
+// Warp-collective: total tiles W = units_per_seq * sum_s ceil(L_s / TT);
 // *bad_len is set when some length is negative or overruns its table row.
 template <int TT, class LN>
 __device__ inline int64_t total_tiles(const LN& ln, bool* bad_len = nullptr) {
+    constexpr int E = kScanPerLane;
     const int lane = threadIdx.x & 31;
     int64_t tot = 0;
     bool bad = false;
-    for (int s0 = 0; s0 < ln.S; s0 += 256) {
-        int part = 0;
+    for (int r0 = 0; r0 < ln.S; r0 += 32 * E) {
+        const int s0 = r0 + lane * E;
+        int v[E], st[E];
+        load_lens(ln, s0, v, st);
+        int64_t part = 0;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int s = s0 + lane * 8 + k;
-            if (s < ln.S) {
-                const int L = __ldg(ln.len + s);
-                bad |= (L < 0 || L > ln.cap);
-                part += ntiles_of<TT>(LN::kHasStart ? ln.eff(s) : clamp_len(L, ln.cap));
+        for (int k = 0; k < E; ++k) {
+            if (s0 + k < ln.S) {
+                bad |= (v[k] < 0 || v[k] > ln.cap);
+                part += ntiles_of<TT>(ln.eff_of(v[k], st[k]));
             }
         }
 #pragma unroll
@@ -138,23 +174,24 @@ __device__ inline int64_t total_tiles(const LN& ln, bool* bad_len = nullptr) {
 struct SeqHit {
     int s;          // sequence holding tile P (num_seqs if none)
     int64_t base;   // index of its first tile
-    int L;          // its attended length
+    int L;          // its raw seq_lens entry
+    int st;         // its raw start entry (0 without starts)
 };
 
 // Warp-collective: the sequence whose tiles contain global tile P.
 template <int TT, class LN>
 __device__ inline SeqHit find_seq(const LN& ln, int64_t P) {
+    constexpr int E = kScanPerLane;
     const int lane = threadIdx.x & 31;
     int64_t base = 0;
-    for (int s0 = 0; s0 < ln.S; s0 += 256) {
-        int64_t w[8];
+    for (int r0 = 0; r0 < ln.S; r0 += 32 * E) {
+        const int s0 = r0 + lane * E;
+        int v[E], st[E];
+        load_lens(ln, s0, v, st);
         int64_t part = 0;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int s = s0 + lane * 8 + k;
-            w[k] = (s < ln.S) ? (int64_t)ntiles_of<TT>(ln.eff(s)) * ln.units : 0;
-            part += w[k];
-        }
+        for (int k = 0; k < E; ++k)
+            part += (s0 + k < ln.S) ? (int64_t)ntiles_of<TT>(ln.eff_of(v[k], st[k])) * ln.units : 0;
         int64_t incl = part;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -164,53 +201,65 @@ __device__ inline SeqHit find_seq(const LN& ln, int64_t P) {
         const unsigned hit = __ballot_sync(kFull, base + incl > P);
         if (hit) {
             const int src = __ffs(hit) - 1;
-            int found = 0;
+            int found = 0, fl = 0, fst = 0;
             int64_t at = 0;
             if (lane == src) {
                 int64_t acc = base + incl - part;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    if (!found && acc + w[k] > P) { found = s0 + lane * 8 + k + 1; at = acc; }
-                    acc += w[k];
+                for (int k = 0; k < E; ++k) {
+                    const int64_t w = (s0 + k < ln.S) ? (int64_t)ntiles_of<TT>(ln.eff_of(v[k], st[k])) * ln.units : 0;
+                    if (!found && acc + w > P) { found = s0 + k + 1; at = acc; fl = v[k]; fst = st[k]; }
+                    acc += w;
                 }
             }
             found = max(__shfl_sync(kFull, found, src) - 1, 0);
             at = __shfl_sync(kFull, at, src);
-            return SeqHit{found, at, ln.eff(found)};
+            fl = __shfl_sync(kFull, fl, src);
+            fst = __shfl_sync(kFull, fst, src);
+            return SeqHit{found, at, fl, fst};
         }
         base += __shfl_sync(kFull, incl, 31);
     }
-    return SeqHit{ln.S, base, 0};
+    return SeqHit{ln.S, base, 0, 0};
 }
 
 // First attended token of the walk's current sequence: a field only when
 // ranges may start past token 0.
-template <bool kStart> struct WalkStart { int st; };
+template <bool kStart> struct WalkStart { int st; int nst; };
 template <> struct WalkStart<false> { static constexpr int st = 0; };
 
 // Walk over a worker's tiles (TT tokens each) in order: (sequence, unit j, tile i).
+// The raw entries of the next sequence are loaded when the walk enters a
+// sequence, so moving on does not wait for a load.
 template <int TT, bool kStart = false>
 struct Walk : WalkStart<kStart> {
     int s, L, nt, j, i, seg_i0, ord;  // L: attended length
+    int nl;                           // raw seq_lens entry of sequence s + 1 (prefetched)
     int64_t T, te;
     bool done;
 
+    __device__ void prefetch_next(const Lens<kStart>& ln) {
+        const bool in = s + 1 < ln.S;
+        nl = in ? ln.raw_len(s + 1) : 0;
+        if constexpr (kStart) this->nst = in ? ln.raw_start(s + 1) : 0;
+    }
     __device__ void init(const Lens<kStart>& ln, int64_t tb, int64_t te_) {
         te = te_;
         T = tb;
         done = tb >= te_;
         ord = 0;
-        s = 0; L = 0; nt = 1; j = 0; i = 0; seg_i0 = 0;
-        if constexpr (kStart) this->st = 0;
+        s = 0; L = 0; nt = 1; j = 0; i = 0; seg_i0 = 0; nl = 0;
+        if constexpr (kStart) { this->st = 0; this->nst = 0; }
         if (done) return;
         const SeqHit h = find_seq<TT>(ln, tb);
         s = h.s;
-        L = h.L;
-        if constexpr (kStart) this->st = ln.first(s);
+        L = ln.eff_of(h.L, h.st);
+        if constexpr (kStart) this->st = ln.first_of(h.st);
         nt = ntiles_of<TT>(L);
         j = (int)((tb - h.base) / nt);
         i = (int)((tb - h.base) % nt);
         seg_i0 = i;
+        prefetch_next(ln);
     }
     __device__ bool first() const { return i == seg_i0; }
     __device__ bool last() const { return i == nt - 1 || T == te - 1; }
@@ -225,10 +274,18 @@ struct Walk : WalkStart<kStart> {
                 j = 0;
                 do {  // a later non-empty sequence exists because T < te <= W
                     ++s;
-                    L = (s < ln.S) ? ln.eff(s) : TT;
+                    if (s < ln.S) {
+                        int nst = 0;
+                        if constexpr (kStart) nst = this->nst;
+                        L = ln.eff_of(nl, nst);
+                        if constexpr (kStart) this->st = ln.first_of(nst);
+                        prefetch_next(ln);
+                    } else {
+                        L = TT;
+                        if constexpr (kStart) this->st = 0;
+                    }
                     nt = ntiles_of<TT>(L);
                 } while (nt == 0);
-                if constexpr (kStart) this->st = (s < ln.S) ? ln.first(s) : 0;
             }
         }
     }
@@ -239,7 +296,10 @@ struct Walk : WalkStart<kStart> {
 // ----------------------------------------------------------------------------
 enum class Path { kMma16, kFp8, kF32 };
 
-template <typename KvT, typename QT, int D_, Path P_, int kWarps_, int kStages_, int kTT_ = kTileTokens>
+// kQH_: q heads one q slot holds (>= the unit's heads, min(g, 8)); a slot per
+// ring stage, since the issue walk may be up to kStages-1 units ahead.
+template <typename KvT, typename QT, int D_, Path P_, int kWarps_, int kStages_, int kTT_ = kTileTokens,
+          int kQH_ = kHeadsPerUnit>
 struct Cfg {
     using kv_t = KvT;
     using q_t = QT;
@@ -255,14 +315,17 @@ struct Cfg {
     static constexpr int kNSub = kRowBytes / 128;       // 128-byte columns per row
     static constexpr int kTensorTile = kNSub * kSubBytes;
     static constexpr int kStageBytes = 2 * kTensorTile; // K tile + V tile
-    static constexpr int kQSlot = kHeadsPerUnit * D * kQBytes;
+    static constexpr int kQH = kQH_;
+    static constexpr int kQSlot = kQH * D * kQBytes;
     static constexpr int kWarpBytes = kStages * (kStageBytes + kQSlot);
     static constexpr int kSmemBytes = kWarps * kWarpBytes + 1024;  // + alignment slack
     static constexpr int kChunksPerRow = kRowBytes / 16;
     static constexpr int kRowsPerInst = 32 / kChunksPerRow;         // rows one warp-wide cp.async covers
     static_assert(kTT == 16 || (kTT == 32 && P_ != Path::kF32), "tile sizes");
     static_assert(kRowBytes % 128 == 0, "rows must be whole 128-byte columns");
-    static_assert(kStageBytes % 1024 == 0 && kQSlot % 1024 == 0, "1024-byte stage alignment");
+    // the swizzle only needs each tile and q slot on a 128-byte boundary
+    static_assert(kStageBytes % 128 == 0 && kQSlot % 128 == 0, "128-byte stage alignment");
+    static_assert(kQH >= 1 && kQH <= kHeadsPerUnit, "q slot heads");
     static_assert(kWarps <= kMaxWarpsPerCta, "workspace sizing");
 };
 
@@ -878,7 +941,7 @@ pkv_merge_kernel(const DecodeParams p, int64_t workers, const SuffixArg<kSuffix>
     const int64_t P = b * chunk;
     if (P >= W) return;
     const SeqHit hit = find_seq<TT>(ln, P);
-    const int nt = ntiles_of<TT>(hit.L);
+    const int nt = ntiles_of<TT>(ln.eff_of(hit.L, hit.st));
     const int j = (int)((P - hit.base) / nt);
     const int off = (int)((P - hit.base) % nt);
     const int64_t T0 = hit.base + (int64_t)j * nt;
