@@ -321,6 +321,7 @@ struct Cfg {
     static constexpr int kSmemBytes = kWarps * kWarpBytes + 1024;  // + alignment slack
     static constexpr int kChunksPerRow = kRowBytes / 16;
     static constexpr int kRowsPerInst = 32 / kChunksPerRow;         // rows one warp-wide cp.async covers
+    static_assert(16 % kRowsPerInst == 0, "a cp.async row group never straddles a 16-token block");
     static_assert(kTT == 16 || (kTT == 32 && P_ != Path::kF32), "tile sizes");
     static_assert(kRowBytes % 128 == 0, "rows must be whole 128-byte columns");
     // the swizzle only needs each tile and q slot on a 128-byte boundary
@@ -401,6 +402,31 @@ struct MmaConsumer {
     float acc[MT][4];    // O^T fragments
     float m0, m1, l0, l1;
     float sl0, sl1;      // per-head score multipliers (log2 domain)
+    // This lane's swizzled byte offsets inside a tile, fixed for the kernel:
+    // 16-bit path: ldmatrix row addresses of k-step / head_dim tile k4 (mod 4)
+    // of the first 16 tokens (later k-steps add a 128-byte column block,
+    // later 16-token m-tiles add 2 KB); FP8 path: the 16-byte K and V chunks
+    // the lane reads for its first rows.
+    uint32_t ko[4], vo[4];
+
+    __device__ void init_lane() {
+        const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+        if constexpr (!kFp8) {
+            const int r = lane & 7, mtx = lane >> 3;
+            const int tk = r + ((mtx & 1) << 3), tv = r + ((mtx >> 1) << 3);
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+                ko[k4] = sw_off<C::kTT>(tk, 2 * k4 + (mtx >> 1));
+                vo[k4] = sw_off<C::kTT>(tv, 2 * k4 + (mtx & 1));
+            }
+        } else {
+            ko[0] = sw_off<C::kTT>(gid, 2 * tig);
+            ko[1] = sw_off<C::kTT>(gid, 2 * tig + 1);
+            vo[0] = sw_off<C::kTT>(2 * tig, gid);
+            vo[1] = sw_off<C::kTT>(2 * tig + 1, gid);
+            ko[2] = ko[3] = vo[2] = vo[3] = 0;
+        }
+    }
 
     __device__ void reset() {
 #pragma unroll
@@ -463,22 +489,21 @@ struct MmaConsumer {
         for (int m = 0; m < NM; ++m) {
             float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
             if constexpr (!kFp8) {
-                const int r = lane & 7, mtx = lane >> 3;
-                const int t = 16 * m + r + ((mtx & 1) << 3);
+                // row t = 16m + (lane's row): the XOR part of the swizzle only
+                // sees t mod 8, so m and the column block are plain offsets
 #pragma unroll
                 for (int kk = 0; kk < KS; ++kk) {
                     uint32_t a[4];
-                    ldsm_x4(a, kb + sw_off<TT>(t, 2 * kk + (mtx >> 1)));
+                    ldsm_x4(a, kb + ko[kk & 3] + (kk >> 2) * (TT * 128) + m * 2048);
                     if (kk & 1) mma16816<kOpBf16>(sb, a, qf[kk][0], qf[kk][1]);
                     else        mma16816<kOpBf16>(sa, a, qf[kk][0], qf[kk][1]);
                 }
             } else {
                 // K rows gid and gid+8 of the m-tile, bytes [32*tig, 32*tig+32).
-                const int t0 = 16 * m + gid, t1 = t0 + 8;
-                const uint4 r0a = *reinterpret_cast<const uint4*>(kt + sw_off<TT>(t0, 2 * tig));
-                const uint4 r0b = *reinterpret_cast<const uint4*>(kt + sw_off<TT>(t0, 2 * tig + 1));
-                const uint4 r1a = *reinterpret_cast<const uint4*>(kt + sw_off<TT>(t1, 2 * tig));
-                const uint4 r1b = *reinterpret_cast<const uint4*>(kt + sw_off<TT>(t1, 2 * tig + 1));
+                const uint4 r0a = *reinterpret_cast<const uint4*>(kt + ko[0] + m * 2048);
+                const uint4 r0b = *reinterpret_cast<const uint4*>(kt + ko[1] + m * 2048);
+                const uint4 r1a = *reinterpret_cast<const uint4*>(kt + ko[0] + m * 2048 + 1024);
+                const uint4 r1b = *reinterpret_cast<const uint4*>(kt + ko[1] + m * 2048 + 1024);
                 const uint32_t w0[8] = {r0a.x, r0a.y, r0a.z, r0a.w, r0b.x, r0b.y, r0b.z, r0b.w};
                 const uint32_t w1[8] = {r1a.x, r1a.y, r1a.z, r1a.w, r1b.x, r1b.y, r1b.z, r1b.w};
 #pragma unroll
@@ -550,12 +575,10 @@ struct MmaConsumer {
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
             if constexpr (!kFp8) {
-                const int r = lane & 7, mtx = lane >> 3;
-                const int t = 16 * m + r + ((mtx >> 1) << 3);
 #pragma unroll
                 for (int mi = 0; mi < MT; ++mi) {
                     uint32_t a[4];
-                    ldsm_x4_trans(a, vb + sw_off<TT>(t, 2 * mi + (mtx & 1)));
+                    ldsm_x4_trans(a, vb + vo[mi & 3] + (mi >> 2) * (TT * 128) + m * 2048);
                     mma16816<kOpBf16>(acc[mi], a, b0[m], b1[m]);
                     if constexpr (kOpBf16) mma16816<true>(acc[mi], a, c0[m], c1[m]);
                 }
@@ -563,11 +586,10 @@ struct MmaConsumer {
                 // V^T fragments: thread gid owns d in [16*gid, 16*gid+16) (one chunk),
                 // rows 2tig, 2tig+1, 2tig+8, 2tig+9 of the m-tile; m-tile mi covers
                 // d = 16*gid + 2*mi (row gid) and 16*gid + 2*mi + 1 (row gid+8).
-                const int tb = 16 * m + 2 * tig;
-                const uint4 R0 = *reinterpret_cast<const uint4*>(vt + sw_off<TT>(tb, gid));
-                const uint4 R1 = *reinterpret_cast<const uint4*>(vt + sw_off<TT>(tb + 1, gid));
-                const uint4 R8 = *reinterpret_cast<const uint4*>(vt + sw_off<TT>(tb + 8, gid));
-                const uint4 R9 = *reinterpret_cast<const uint4*>(vt + sw_off<TT>(tb + 9, gid));
+                const uint4 R0 = *reinterpret_cast<const uint4*>(vt + vo[0] + m * 2048);
+                const uint4 R1 = *reinterpret_cast<const uint4*>(vt + vo[1] + m * 2048);
+                const uint4 R8 = *reinterpret_cast<const uint4*>(vt + vo[0] + m * 2048 + 1024);
+                const uint4 R9 = *reinterpret_cast<const uint4*>(vt + vo[1] + m * 2048 + 1024);
                 const uint32_t q0[4] = {R0.x, R0.y, R0.z, R0.w}, q1[4] = {R1.x, R1.y, R1.z, R1.w};
                 const uint32_t q8[4] = {R8.x, R8.y, R8.z, R8.w}, q9[4] = {R9.x, R9.y, R9.z, R9.w};
 #pragma unroll
@@ -646,6 +668,7 @@ struct F32Consumer {
             l[h] = 0.f;
         }
     }
+    __device__ void init_lane() {}
     __device__ void load_q(const uint8_t* qs, int nh_, float scale_log2, float) {
         const int lane = threadIdx.x & 31, c = lane % CPR;
         nh = nh_;
@@ -781,34 +804,79 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+// kv head and head chunk of unit j (no division in the common nch == 1 case)
+__device__ __forceinline__ int2 unit_head(int j, int nch) {
+    if (nch == 1) return make_int2(j, 0);
+    const int kh = j / nch;
+    return make_int2(kh, j - kh * nch);
+}
+
+// This lane's part of a tile's cp.async loads, fixed for the kernel: the
+// swizzled shared-memory offsets of its rows (the swizzle repeats every 8
+// rows, so kP offsets cover a tile; later row groups add 1 KB each) and its
+// byte offset inside a row group of the cache.
+template <class C>
+struct IssueLane {
+    static constexpr int kR = C::kRowsPerInst;
+    static constexpr int kP = 8 / kR;      // distinct swizzle patterns
+    uint32_t so[kP];
+    int64_t goff;                          // r0 * row_stride + 16 * cr
+    int64_t gstep;                         // kR * row_stride
+    __device__ void init(const DecodeParams& p) {
+        const int lane = threadIdx.x & 31;
+        const int cr = lane % C::kChunksPerRow, r0 = lane / C::kChunksPerRow;
+#pragma unroll
+        for (int k = 0; k < kP; ++k) so[k] = sw_off<C::kTT>(k * kR + r0, cr);
+        const int64_t row_stride = (int64_t)p.num_kv_heads * C::kRowBytes;  // bytes between tokens
+        goff = r0 * row_stride + 16 * cr;
+        gstep = kR * row_stride;
+    }
+};
+
 // Issue the async loads of the walk's current tile (and, on a unit's first
-// tile, of its q rows) into stage `stg` / q slot `qslot`.
+// tile, of its q rows) into stage `stg` / q slot `qslot`.  lg_bs: log2 of
+// the block size (16 or 32 tokens).
 template <class C, bool kStart>
 __device__ __forceinline__ void issue_tile(const DecodeParams& p, const Walk<C::kTT, kStart>& w, TablePrefetch& tp,
-                                           uint8_t* stg, uint8_t* qslot) {
+                                           const IssueLane<C>& il, int lg_bs, uint8_t* stg, uint8_t* qslot) {
     const int lane = threadIdx.x & 31;
-    const int kh = w.j / p.nch, c = w.j % p.nch;
-    const int tok = w.st + w.i * C::kTT;  // absolute token of the tile's first row
-    const int nblk = (w.st + w.L + p.block_size - 1) / p.block_size;
-    int phys = tp.get(p, w.s, tok / p.block_size, nblk, lane);
-    if (phys < 0 || phys >= p.num_blocks) {
-        if (lane == 0) raise_error(p.err, PKV_DEVERR_BLOCK_ID);
-        phys = 0;
+    const int2 hc = unit_head(w.j, p.nch);
+    const int kh = hc.x, c = hc.y;
+    const int tok = w.st + w.i * C::kTT;  // absolute token of the tile's first row (a multiple of 16)
+    const int bmask = (1 << lg_bs) - 1;
+    const int nblk = (w.st + w.L + bmask) >> lg_bs;
+    const int b0 = tok >> lg_bs;
+    auto checked = [&](int ph) {
+        if (ph < 0 || ph >= p.num_blocks) {
+            if (lane == 0) raise_error(p.err, PKV_DEVERR_BLOCK_ID);
+            ph = 0;
+        }
+        return ph;
+    };
+    const int phys0 = checked(tp.get(p, w.s, b0, nblk, lane));
+    const int64_t kv_row = (int64_t)p.num_kv_heads * C::kRowBytes;  // bytes between tokens
+    const int64_t base0 = ((((int64_t)phys0 << lg_bs) + (tok & bmask)) * p.num_kv_heads + kh) * C::kRowBytes;
+    // A 32-token tile over 16-token blocks covers two blocks: rows 16.. come
+    // from the next one (or, past the sequence's last block, again from the
+    // first: those rows are masked).  base1 is offset so that row t reads
+    // base1 + t * row_stride.
+    int64_t base1 = base0;
+    if constexpr (C::kTT > 16) {
+        if (lg_bs == 4) {
+            const int phys1 = b0 + 1 < nblk ? checked(tp.get(p, w.s, b0 + 1, nblk, lane)) : phys0;
+            base1 = (((int64_t)phys1 << lg_bs) * p.num_kv_heads + kh) * C::kRowBytes - 16 * kv_row;
+        }
     }
-    const int tok0 = tok % p.block_size;
-    const int64_t row_stride = (int64_t)p.num_kv_heads * C::kRowBytes;  // bytes between tokens
-    const int64_t base = (((int64_t)phys * p.block_size + tok0) * p.num_kv_heads + kh) * C::kRowBytes;
-    const uint8_t* ksrc = p.key_cache + base;
-    const uint8_t* vsrc = p.value_cache + base;
     const uint32_t kdst = smem_u32(stg), vdst = smem_u32(stg + C::kTensorTile);
-    const int cr = lane % C::kChunksPerRow, r0 = lane / C::kChunksPerRow;
+    const uint8_t* kl = p.key_cache + il.goff;
+    const uint8_t* vl = p.value_cache + il.goff;
 #pragma unroll
     for (int it = 0; it < C::kTT / C::kRowsPerInst; ++it) {
-        const int t = it * C::kRowsPerInst + r0;
-        const int64_t off = t * row_stride + cr * 16;
-        const uint32_t so = sw_off<C::kTT>(t, cr);
-        cp_async16(kdst + so, ksrc + off);
-        cp_async16(vdst + so, vsrc + off);
+        // rows >= 16 exactly when it * kRowsPerInst >= 16
+        const int64_t off = (it * C::kRowsPerInst >= 16 ? base1 : base0) + it * il.gstep;
+        const uint32_t so = il.so[it % IssueLane<C>::kP] + (it / IssueLane<C>::kP) * 1024;
+        cp_async16(kdst + so, kl + off);
+        cp_async16(vdst + so, vl + off);
     }
     if (w.first()) {
         const int nh = min(kHeadsPerUnit, p.g - kHeadsPerUnit * c);
@@ -853,26 +921,31 @@ pkv_decode_kernel(const DecodeParams p, const SuffixArg<kSuffix> sx) {
     iw.init(ln, tb, te);
     cw = iw;
     TablePrefetch tp;
+    IssueLane<C> il;
+    il.init(p);
+    const int lg_bs = 31 - __clz(p.block_size);
 #pragma unroll 1
     for (int k = 0; k < C::kStages - 1; ++k) {
         if (!iw.done)
-            issue_tile<C>(p, iw, tp, stages + k * C::kStageBytes, qslots + (iw.ord % C::kStages) * C::kQSlot);
+            issue_tile<C>(p, iw, tp, il, lg_bs, stages + k * C::kStageBytes, qslots + (iw.ord % C::kStages) * C::kQSlot);
         cp_async_commit();
         iw.advance(ln);
     }
     const float kscale = (C::kPath == Path::kFp8 && p.k_scale) ? __ldg(p.k_scale) : 1.f;
     const float vscale = (C::kPath == Path::kFp8 && p.v_scale) ? __ldg(p.v_scale) : 1.f;
     ConsumerOf<C> cs;
+    cs.init_lane();
 #pragma unroll 1
     for (int n = 0; !cw.done; ++n) {
         if (!iw.done)
-            issue_tile<C>(p, iw, tp, stages + ((n + C::kStages - 1) % C::kStages) * C::kStageBytes,
+            issue_tile<C>(p, iw, tp, il, lg_bs, stages + ((n + C::kStages - 1) % C::kStages) * C::kStageBytes,
                           qslots + (iw.ord % C::kStages) * C::kQSlot);
         cp_async_commit();
         iw.advance(ln);
         cp_async_wait<C::kStages - 1>();
         __syncwarp();
-        const int kh = cw.j / p.nch, c = cw.j % p.nch;
+        const int2 hc = unit_head(cw.j, p.nch);
+        const int kh = hc.x, c = hc.y;
         const int nh = min(kHeadsPerUnit, p.g - kHeadsPerUnit * c);
         if (cw.first()) {
             cs.load_q(qslots + (cw.ord % C::kStages) * C::kQSlot, nh, p.scale_log2, kscale);
