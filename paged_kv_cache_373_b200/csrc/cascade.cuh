@@ -119,6 +119,20 @@ struct MmaRowsConsumer {
     float m[NT][2], l[NT][2];
     uint32_t qb;  // shared address of the unit's q rows (swizzled, R rows)
     float sl;
+    // this lane's swizzled ldmatrix offsets (k-step / head_dim tile mod 4) in a
+    // K tile, a V tile and the q slot; fixed for the kernel
+    uint32_t ko[4], vo[4], qo[4];
+
+    __device__ void init_lane() {
+        const int lane = threadIdx.x & 31;
+        const int r = lane & 7, mtx = lane >> 3;
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+            ko[k4] = sw_off<16>(r + ((mtx & 1) << 3), 2 * k4 + (mtx >> 1));
+            vo[k4] = sw_off<16>(r + ((mtx >> 1) << 3), 2 * k4 + (mtx & 1));
+            qo[k4] = sw_off<R>(8 * (mtx >> 1) + r, 2 * k4 + (mtx & 1));
+        }
+    }
 
     __device__ void reset() {
 #pragma unroll
@@ -151,11 +165,11 @@ struct MmaRowsConsumer {
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
             uint32_t a[4];
-            ldsm_x4(a, kb + sw_off<16>(r + ((mtx & 1) << 3), 2 * kk + (mtx >> 1)));
+            ldsm_x4(a, kb + ko[kk & 3] + (kk >> 2) * 2048);
 #pragma unroll
             for (int n2 = 0; n2 < NT / 2; ++n2) {
                 uint32_t b[4];  // b0, b1 of n-tile 2*n2 and of 2*n2+1
-                ldsm_x4(b, qb + sw_off<R>(8 * (2 * n2 + (mtx >> 1)) + r, 2 * kk + (mtx & 1)));
+                ldsm_x4(b, qb + qo[kk & 3] + (kk >> 2) * (R * 128) + n2 * 2048);
                 mma16816<kOpBf16>(s[2 * n2], a, b[0], b[1]);
                 mma16816<kOpBf16>(s[2 * n2 + 1], a, b[2], b[3]);
             }
@@ -203,11 +217,10 @@ struct MmaRowsConsumer {
                 acc[mi][n][2] *= al[n][0]; acc[mi][n][3] *= al[n][1];
             }
         }
-        const int t = r + ((mtx >> 1) << 3);
 #pragma unroll
         for (int mi = 0; mi < MT; ++mi) {
             uint32_t a[4];
-            ldsm_x4_trans(a, vb + sw_off<16>(t, 2 * mi + (mtx & 1)));
+            ldsm_x4_trans(a, vb + vo[mi & 3] + (mi >> 2) * 2048);
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
                 mma16816<kOpBf16>(acc[mi][n], a, b0[n], b1[n]);
@@ -290,28 +303,30 @@ pkv_prefix_kernel(const DecodeParams p, const CascadeParams c) {
         u.first_member = __ldg(c.grp_members + u.o0);
     };
     UnitInfo iu, cu;  // issue walk's and compute walk's units
+    IssueLane<C> il;
+    il.init(p);
+    const int lg_bs = 31 - __clz(p.block_size);
     auto issue = [&](const Walk<16>& w, TablePrefetch& tp, uint8_t* stg, uint8_t* qslot) {
         unit_rows(w, iu);
         const int kh = iu.kh, rc = iu.rc, nrows = iu.nrows, o0 = iu.o0, first_member = iu.first_member;
         const int tok = w.i * 16;
-        const int nblk = (w.L + p.block_size - 1) / p.block_size;
-        int phys = tp.get(p, first_member, tok / p.block_size, nblk, lane);
+        const int bmask = (1 << lg_bs) - 1;
+        const int nblk = (w.L + bmask) >> lg_bs;
+        int phys = tp.get(p, first_member, tok >> lg_bs, nblk, lane);
         if (phys < 0 || phys >= p.num_blocks) {
             if (lane == 0) raise_error(p.err, PKV_DEVERR_BLOCK_ID);
             phys = 0;
         }
-        const int tok0 = tok % p.block_size;
-        const int64_t row_stride = (int64_t)p.num_kv_heads * C::kRowBytes;
-        const int64_t base = (((int64_t)phys * p.block_size + tok0) * p.num_kv_heads + kh) * C::kRowBytes;
+        const int64_t base = ((((int64_t)phys << lg_bs) + (tok & bmask)) * p.num_kv_heads + kh) * C::kRowBytes;
         const uint32_t kdst = smem_u32(stg), vdst = smem_u32(stg + C::kTensorTile);
-        const int cr = lane % C::kChunksPerRow, r0 = lane / C::kChunksPerRow;
+        const uint8_t* kl = p.key_cache + il.goff;
+        const uint8_t* vl = p.value_cache + il.goff;
 #pragma unroll
         for (int it = 0; it < 16 / C::kRowsPerInst; ++it) {
-            const int t = it * C::kRowsPerInst + r0;
-            const int64_t off = t * row_stride + cr * 16;
-            const uint32_t so = sw_off<16>(t, cr);
-            cp_async16(kdst + so, p.key_cache + base + off);
-            cp_async16(vdst + so, p.value_cache + base + off);
+            const int64_t off = base + it * il.gstep;
+            const uint32_t so = il.so[it % IssueLane<C>::kP] + (it / IssueLane<C>::kP) * 1024;
+            cp_async16(kdst + so, kl + off);
+            cp_async16(vdst + so, vl + off);
         }
         if (w.first()) {
             constexpr int CPR = C::kRowBytes / 16;
@@ -337,6 +352,7 @@ pkv_prefix_kernel(const DecodeParams p, const CascadeParams c) {
         iw.advance(ln);
     }
     MmaRowsConsumer<C, NT> cs;
+    cs.init_lane();
 #pragma unroll 1
     for (int n = 0; !cw.done; ++n) {
         if (!iw.done)
@@ -410,7 +426,7 @@ pkv_cascade_combine_kernel(const DecodeParams p, const CascadeParams c) {
     const Lens<false> ln{c.prefix_eff, nullptr, c.num_groups, p.num_kv_heads * c.row_chunks, 0x7fffffff};
     const int j = kh * c.row_chunks + rc;                   // unit of the group
     const int nt = ntiles_of<16>(ln.eff(g));
-    const int64_t W = total_tiles<16>(ln);
+    const int64_t W = total_tiles<16, kMergeScanPerLane>(ln);
     const int64_t chunk = (W + c.prefix_workers - 1) / c.prefix_workers;
     const int64_t T0 = group_tile_base(ln, g) + (int64_t)j * nt;
     const int64_t bf = T0 / chunk, bl = (T0 + nt - 1) / chunk;

@@ -127,34 +127,36 @@ __device__ __forceinline__ void load_run(const int32_t* a, int s0, int n, int (&
     }
 }
 
-// Sequences per lane in one round of the warp-wide length scans (32 x 32 =
-// 1024 sequences per round: one round of loads for batches up to 1024).
+// Sequences per lane in one round of the decode kernel's warp-wide length
+// scans (32 x 32 = 1024 sequences per round: one round of loads for batches
+// up to 1024).  The merge kernel scans 8 per lane: its CTAs are scheduled
+// beside the running decode CTAs, so it keeps to a small register budget.
 constexpr int kScanPerLane = 32;
+constexpr int kMergeScanPerLane = 8;
 
 // Raw lengths (and starts) of the lane's sequences of the round at s0.
-template <class LN>
-__device__ __forceinline__ void load_lens(const LN& ln, int s0, int (&v)[kScanPerLane], int (&st)[kScanPerLane]) {
-    load_run<kScanPerLane>(ln.len, s0, ln.S, v);
+template <int E, class LN>
+__device__ __forceinline__ void load_lens(const LN& ln, int s0, int (&v)[E], int (&st)[E]) {
+    load_run<E>(ln.len, s0, ln.S, v);
     if constexpr (LN::kHasStart) {
-        load_run<kScanPerLane>(ln.start, s0, ln.S, st);
+        load_run<E>(ln.start, s0, ln.S, st);
     } else {
 #pragma unroll
-        for (int k = 0; k < kScanPerLane; ++k) st[k] = 0;
+        for (int k = 0; k < E; ++k) st[k] = 0;
     }
 }
 
 // Warp-collective: total tiles W = units_per_seq * sum_s ceil(L_s / TT);
 // *bad_len is set when some length is negative or overruns its table row.
-template <int TT, class LN>
+template <int TT, int E = kScanPerLane, class LN>
 __device__ inline int64_t total_tiles(const LN& ln, bool* bad_len = nullptr) {
-    constexpr int E = kScanPerLane;
     const int lane = threadIdx.x & 31;
     int64_t tot = 0;
     bool bad = false;
     for (int r0 = 0; r0 < ln.S; r0 += 32 * E) {
         const int s0 = r0 + lane * E;
         int v[E], st[E];
-        load_lens(ln, s0, v, st);
+        load_lens<E>(ln, s0, v, st);
         int64_t part = 0;
 #pragma unroll
         for (int k = 0; k < E; ++k) {
@@ -179,15 +181,14 @@ struct SeqHit {
 };
 
 // Warp-collective: the sequence whose tiles contain global tile P.
-template <int TT, class LN>
+template <int TT, int E = kScanPerLane, class LN>
 __device__ inline SeqHit find_seq(const LN& ln, int64_t P) {
-    constexpr int E = kScanPerLane;
     const int lane = threadIdx.x & 31;
     int64_t base = 0;
     for (int r0 = 0; r0 < ln.S; r0 += 32 * E) {
         const int s0 = r0 + lane * E;
         int v[E], st[E];
-        load_lens(ln, s0, v, st);
+        load_lens<E>(ln, s0, v, st);
         int64_t part = 0;
 #pragma unroll
         for (int k = 0; k < E; ++k)
@@ -624,6 +625,40 @@ struct MmaConsumer {
             a1 += __shfl_xor_sync(kFull, a1, o);
         }
         const int h0 = 2 * tig, h1 = 2 * tig + 1;
+        bool to_out = !k.split;
+        if constexpr (kPart) to_out = to_out && !k.part;
+        if (to_out) {
+            // the output rows, normalised and rounded RNE to the q dtype, two
+            // adjacent head_dim elements per 32-bit store
+            constexpr bool kQb = std::is_same<QT, __nv_bfloat16>::value;
+            const float s0 = a0 > 0.f ? vscale / a0 : 0.f, s1 = a1 > 0.f ? vscale / a1 : 0.f;
+            QT* out = reinterpret_cast<QT*>(p.out) + k.row0 * D;
+            if constexpr (!kFp8) {
+                // O^T fragments hold (d = 16 mi + gid (+8), heads 2 tig, 2 tig + 1):
+                // transposed, lane (gid, tig) holds head gid at d = 2 tig, 2 tig + 1
+#pragma unroll
+                for (int mi = 0; mi < MT; ++mi) {
+                    const uint32_t lo = movm_trans(pack2<kQb>(acc[mi][0] * s0, acc[mi][1] * s1));
+                    const uint32_t hi = movm_trans(pack2<kQb>(acc[mi][2] * s0, acc[mi][3] * s1));
+                    if (gid < k.nh) {
+                        *reinterpret_cast<uint32_t*>(out + gid * D + 16 * mi + 2 * tig) = lo;
+                        *reinterpret_cast<uint32_t*>(out + gid * D + 16 * mi + 8 + 2 * tig) = hi;
+                    }
+                }
+            } else {
+                // FP8 path: lane holds d = 16 gid + 2 mi and the next one of heads h0, h1
+#pragma unroll
+                for (int mi = 0; mi < MT; ++mi) {
+                    if (h0 < k.nh)
+                        *reinterpret_cast<uint32_t*>(out + h0 * D + 16 * gid + 2 * mi) =
+                            pack2<kQb>(acc[mi][0] * s0, acc[mi][2] * s0);
+                    if (h1 < k.nh)
+                        *reinterpret_cast<uint32_t*>(out + h1 * D + 16 * gid + 2 * mi) =
+                            pack2<kQb>(acc[mi][1] * s1, acc[mi][3] * s1);
+                }
+            }
+            return;
+        }
 #pragma unroll
         for (int mi = 0; mi < MT; ++mi) {
             int d0, d1;
@@ -976,7 +1011,7 @@ pkv_decode_kernel(const DecodeParams p, const SuffixArg<kSuffix> sx) {
 // row; CTA 0 zeroes the empty sequences.  Partials are folded in worker order, four segments
 // per step (their loads in flight together, M updated once per step).
 // ----------------------------------------------------------------------------
-template <typename QT, int D, int TT, bool kSuffix>
+template <typename QT, int D, int TT, bool kSuffix, int kScanE = kMergeScanPerLane>
 __global__ void __launch_bounds__(256)
 pkv_merge_kernel(const DecodeParams p, int64_t workers, const SuffixArg<kSuffix> sx) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1009,11 +1044,11 @@ pkv_merge_kernel(const DecodeParams p, int64_t workers, const SuffixArg<kSuffix>
     }
     if (b >= workers) return;
     // every warp locates the boundary's unit itself (no block barrier)
-    const int64_t W = total_tiles<TT>(ln);
+    const int64_t W = total_tiles<TT, kScanE>(ln);
     const int64_t chunk = (W + workers - 1) / workers;
     const int64_t P = b * chunk;
     if (P >= W) return;
-    const SeqHit hit = find_seq<TT>(ln, P);
+    const SeqHit hit = find_seq<TT, kScanE>(ln, P);
     const int nt = ntiles_of<TT>(ln.eff_of(hit.L, hit.st));
     const int j = (int)((P - hit.base) / nt);
     const int off = (int)((P - hit.base) % nt);
