@@ -224,6 +224,21 @@ __device__ inline SeqHit find_seq(const LN& ln, int64_t P) {
     return SeqHit{ln.S, base, 0, 0};
 }
 
+// The scans with their width chosen by the batch: 8 lengths per lane (one
+// round, a short prologue) for batches of up to 256 sequences, 32 per lane
+// (4x fewer rounds) for larger ones.  Every warp of a grid takes the same
+// branch, so they all agree on W and on the tile split.
+template <int TT, class LN>
+__device__ inline int64_t total_tiles_any(const LN& ln, bool* bad_len = nullptr) {
+    if (ln.S <= 256) return total_tiles<TT, kMergeScanPerLane>(ln, bad_len);
+    return total_tiles<TT, kScanPerLane>(ln, bad_len);
+}
+template <int TT, class LN>
+__device__ inline SeqHit find_seq_any(const LN& ln, int64_t P) {
+    if (ln.S <= 256) return find_seq<TT, kMergeScanPerLane>(ln, P);
+    return find_seq<TT, kScanPerLane>(ln, P);
+}
+
 // First attended token of the walk's current sequence: a field only when
 // ranges may start past token 0.
 template <bool kStart> struct WalkStart { int st; int nst; };
@@ -252,7 +267,7 @@ struct Walk : WalkStart<kStart> {
         s = 0; L = 0; nt = 1; j = 0; i = 0; seg_i0 = 0; nl = 0;
         if constexpr (kStart) { this->st = 0; this->nst = 0; }
         if (done) return;
-        const SeqHit h = find_seq<TT>(ln, tb);
+        const SeqHit h = find_seq_any<TT>(ln, tb);
         s = h.s;
         L = ln.eff_of(h.L, h.st);
         if constexpr (kStart) this->st = ln.first_of(h.st);
@@ -946,7 +961,7 @@ pkv_decode_kernel(const DecodeParams p, const SuffixArg<kSuffix> sx) {
     const int64_t workers = (int64_t)gridDim.x * C::kWarps;
     const int64_t wid = (int64_t)blockIdx.x * C::kWarps + warp;
     bool bad_len = false;
-    const int64_t W = total_tiles<C::kTT>(ln, &bad_len);
+    const int64_t W = total_tiles_any<C::kTT>(ln, &bad_len);
     if (bad_len && wid == 0 && lane == 0) raise_error(p.err, PKV_DEVERR_SEQ_LEN);
     const int64_t chunk = (W + workers - 1) / workers;
     const int64_t tb = min(W, wid * chunk), te = min(W, tb + chunk);
