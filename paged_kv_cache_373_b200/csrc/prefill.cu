@@ -50,7 +50,7 @@ constexpr int kPfTok = 64;          // KV tokens per tile (N of S, K of P V)
 constexpr int kPfGroup = 256;       // softmax threads per unit: two per row
 constexpr int kPfMmaWarp = 16;      // issues the tensor-core products, owns tensor memory
 constexpr int kPfLoadWarp = 17;     // issues the TMA copies
-constexpr int kPfConvWarp = 18;     // bf16 caches: converts each V tile to f16 (single-part P V)
+constexpr int kPfThreads = 18 * 32;
 constexpr int kPfStages = 3;        // K and V ring depth
 constexpr int kPfTmemCols = 512;    // unit u: S in columns 256 u + [0, 64), O from 256 u + 64,
 constexpr int kPfTmemP = 192;       //   P (hi, lo: 32 columns each) from 256 (1 - u) + 192: the
@@ -69,8 +69,7 @@ enum : int {
     kBarP = kBarS + 2,                     // [unit] P written (and S read): kPfGroup arrivals
     kBarO = kBarP + 2,                     // [unit] P V finished
     kBarDrain = kBarO + 2,                 // products drained (abort path)
-    kBarVConv = kBarDrain + 1,             // [stage] bf16 caches: the V tile's f16 copy written
-    kNumBars = kBarVConv + kPfStages
+    kNumBars = kBarDrain + 1
 };
 
 struct PrefillParams {
@@ -248,11 +247,10 @@ __device__ __forceinline__ void tc_after_sync() { asm volatile("tcgen05.fence::a
 
 template <typename T, int D>
 struct PfSmem {
-    static constexpr bool kConv = std::is_same<T, __nv_bfloat16>::value;  // V tiles converted to f16
-    static constexpr int kThreads = (kConv ? 19 : 18) * 32;
     static constexpr int kQ = kPfRows * D * 2;     // one unit's q rows
     static constexpr int kTile = kPfTok * D * 2;   // one K or V tile
-    static constexpr int kData = 2 * kQ + (2 + (kConv ? 1 : 0)) * kPfStages * kTile + 1024;  // + alignment
+    static constexpr int kParts = std::is_same<T, __nv_bfloat16>::value ? 2 : 1;  // P hi (+ lo)
+    static constexpr int kData = 2 * kQ + 2 * kPfStages * kTile + 1024;           // + alignment
     // at least 120 KB, so one CTA (and its 512 tensor-memory columns) per SM
     static constexpr int kBytes = kData > 120 * 1024 ? kData : 120 * 1024;
 };
@@ -263,7 +261,7 @@ struct PfUnit {
 };
 
 template <typename T, int D>
-__global__ void __launch_bounds__(PfSmem<T, D>::kThreads, 1)
+__global__ void __launch_bounds__(kPfThreads, 1)
 pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v) {
     using SM = PfSmem<T, D>;
@@ -274,11 +272,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     uint8_t* qsm = sm;                          // [2 units]
     uint8_t* ksm = qsm + 2 * SM::kQ;            // [stage]
     uint8_t* vsm = ksm + kPfStages * SM::kTile; // [stage]
-    uint8_t* vhsm = vsm + kPfStages * SM::kTile; // [stage] bf16 caches: f16 copies of the V tiles
     __shared__ __align__(8) uint64_t bars[kNumBars];
-    __shared__ int vmode[kPfStages];            // bf16 caches: 0 = the f16 copy of the stage's V tile is
-                                                // exact, 1 = a value is past f16's range: P V reads the
-                                                // bf16 tile with P as hi + lo parts
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     __shared__ float xmax[2][2][2][kPfRows];    // [unit][tile parity][half][row] partial row maxima
@@ -448,40 +442,25 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                         }
                     }
                 }
-                // bf16 caches: the tile's V is read as an exact f16 copy unless a
-                // value is past f16's range (vmode), which sets P's format
-                bool pf16 = !kBf16;
-                if constexpr (kBf16) {
-                    if (ok) {
-                        ok = mbar_wait(bar(kBarVConv + stg(kt)), pass(kt), abort, p.wait_ns);
-                        ok = __all_sync(kFull, ok);
-                        if (ok) pf16 = vmode[stg(kt)] == 0;
-                    }
-                }
                 if (!ok) {
                     failed = true;
                     continue;  // the next tile's group barrier ends the loop for the whole group
                 }
                 // ---- this half of P into tensor memory: row = lane, two
-                // tokens per 32-bit column (f16 in one part; with a bf16 V tile
-                // bf16 as hi + lo parts, 32 columns apart)
+                // tokens per 32-bit column (bf16 as hi + lo parts, 32 columns apart)
                 {
                     uint32_t h[kPfTok / 4], lo[kPfTok / 4];
-                    if (pf16) {
 #pragma unroll
-                        for (int e = 0; e < kPfTok / 4; ++e) h[e] = pack2<false>(sc[2 * e], sc[2 * e + 1]);
-                        tc_st16u(tP, h);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < kPfTok / 4; ++e) {
-                            const float a = sc[2 * e], b = sc[2 * e + 1];
-                            h[e] = pack2<true>(a, b);
+                    for (int e = 0; e < kPfTok / 4; ++e) {
+                        const float a = sc[2 * e], b = sc[2 * e + 1];
+                        h[e] = pack2<kBf16>(a, b);
+                        if constexpr (kBf16) {
                             const float2 hf = unpack2<true>(h[e]);
                             lo[e] = pack2<true>(a - hf.x, b - hf.y);
                         }
-                        tc_st16u(tP, h);
-                        tc_st16u(tP + kPfTok / 2, lo);
                     }
+                    tc_st16u(tP, h);
+                    if constexpr (kBf16) tc_st16u(tP + kPfTok / 2, lo);
                     tc_wait_st();
                 }
                 tc_before_sync();
@@ -549,8 +528,6 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
             const uint64_t dq1 = tc_desc(smem_u32(qsm + (split ? 0 : SM::kQ)), 16, 1024);
             const uint64_t dk0 = tc_desc(smem_u32(ksm), 16, 1024);
             const uint64_t dv0 = tc_desc(smem_u32(vsm), kPfTok * 128, 1024);
-            const uint64_t dvh0 = tc_desc(smem_u32(vhsm), kPfTok * 128, 1024);
-            const uint32_t id_o16 = tc_idesc<false>(kPfRows, D, 1);
             auto issue_s = [&](int X, int st) {  // S_X = Q_X K^T (a split unit: both groups read q slot 0)
                 const uint64_t qd = X ? dq1 : dq0;
                 const uint64_t kd = desc_add(dk0, (uint32_t)(st * (SM::kTile >> 4)));
@@ -561,27 +538,16 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                            desc_add(kd, ((kk >> 2) * kPfTok * 128 + (kk & 3) * 32) >> 4), id_s, kk > 0);
                 tc_commit(bar(kBarS + X));
             };
-            auto issue_pv = [&](int X, int st, bool acc) {  // O_X (+)= P_X V (P in tensor memory)
-                // f16 V copy and f16 P in one part, or bf16 V with P as hi + lo
-                const bool f16v = !kBf16 || vmode[st] == 0;
-                const uint64_t vd = desc_add(kBf16 && f16v ? dvh0 : dv0, (uint32_t)(st * (SM::kTile >> 4)));
-                const uint32_t id = kBf16 && f16v ? id_o16 : id_o;
-                const int parts = f16v ? 1 : 2;
+            auto issue_pv = [&](int X, int st, bool acc) {  // O_X (+)= P_X V (hi, then lo; P in tensor memory)
+                const uint64_t vd = desc_add(dv0, (uint32_t)(st * (SM::kTile >> 4)));
                 const uint32_t d = tmem + X * 256 + kPfTok, a = tmem + (X ^ 1) * 256 + kPfTmemP;
-#pragma unroll 1
-                for (int part = 0; part < parts; ++part)
+#pragma unroll
+                for (int part = 0; part < SM::kParts; ++part)
 #pragma unroll
                     for (int kk = 0; kk < kPfTok / 16; ++kk)
-                        tc_mma_ts(d, a + part * (kPfTok / 2) + kk * 8, desc_add(vd, (kk * 2048) >> 4), id,
+                        tc_mma_ts(d, a + part * (kPfTok / 2) + kk * 8, desc_add(vd, (kk * 2048) >> 4), id_o,
                                   (acc || part > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(bar(kBarO + X));
-            };
-            // the V tile of tile kt is ready: landed (and its tail zeroed), or,
-            // for bf16 caches, converted
-            auto v_ready = [&](int kt) {
-                if constexpr (kBf16) return mbar_wait(bar(kBarVConv + stg(kt)), pass(kt), abort, p.wait_ns);
-                return mbar_wait(bar(kBarVFull + stg(kt)), pass(kt), abort, p.wait_ns) &&
-                       (kt != nkv - 1 || !need_fix || mbar_wait(bar(kBarVFix), 0, abort, p.wait_ns));
             };
             bool ok = mbar_wait(bar(kBarQ), 0, abort, p.wait_ns);
             if (!split) {
@@ -598,7 +564,9 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                 for (int kt = 0; ok && kt < nkv; ++kt) {
                     const int st = stg(kt), sn = stg(kt + 1);
                     const bool a1 = kt < U1.nkv, a1n = kt + 1 < U1.nkv;
-                    ok = v_ready(kt) && mbar_wait(bar(kBarP), kt & 1, abort, p.wait_ns);
+                    ok = mbar_wait(bar(kBarVFull + st), pass(kt), abort, p.wait_ns) &&
+                         (kt != nkv - 1 || !need_fix || mbar_wait(bar(kBarVFix), 0, abort, p.wait_ns)) &&
+                         mbar_wait(bar(kBarP), kt & 1, abort, p.wait_ns);
                     if (!ok) break;
                     tc_after_sync();
                     issue_pv(0, st, kt > 0);
@@ -639,7 +607,9 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                     for (int X = 0; X < 2; ++X) {
                         const int kt = 2 * i + X;
                         if (kt >= nkv) break;
-                        ok = v_ready(kt) && mbar_wait(bar(kBarP + X), i & 1, abort, p.wait_ns);
+                        ok = mbar_wait(bar(kBarVFull + stg(kt)), pass(kt), abort, p.wait_ns) &&
+                             (kt != nkv - 1 || !need_fix || mbar_wait(bar(kBarVFix), 0, abort, p.wait_ns)) &&
+                             mbar_wait(bar(kBarP + X), i & 1, abort, p.wait_ns);
                         if (!ok) break;
                         tc_after_sync();
                         issue_pv(X, stg(kt), i > 0);
@@ -728,7 +698,7 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         }
         __syncwarp();
         ok = __shfl_sync(kFull, ok, 0);
-        if (!kBf16 && need_fix) {  // zero the last V tile's rows at and past the unit's end (bf16: the converter)
+        if (need_fix) {  // zero the last V tile's rows at and past the unit's end
             const int kl = nkv - 1, st = stg(kl);
             bool fine = ok && mbar_wait(bar(kBarVFull + st), pass(kl), abort, p.wait_ns);
             fine = __all_sync(kFull, fine);
@@ -740,50 +710,6 @@ pkv_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(kBarVFix));
-            }
-        }
-    } else if (kBf16 && warp == kPfConvWarp) {
-        // ================= bf16 caches: each V tile, once landed, copied as f16
-        // into its stage's f16 buffer (same swizzled offsets: both 2-byte types).
-        // bf16 -> f16 is exact up to f16's range (a value below 2^-14 keeps an
-        // absolute error under 2^-25); if any value is past 65504 the stage is
-        // flagged and P V reads the bf16 tile instead.  Rows at and past the
-        // unit's end are zeroed in both buffers.
-        bool ok = true;
-#pragma unroll 1
-        for (int kt = 0; kt < nkv; ++kt) {
-            const int st = stg(kt);
-            ok = mbar_wait(bar(kBarVFull + st), pass(kt), abort, p.wait_ns);
-            ok = __all_sync(kFull, ok);
-            if (!ok) break;
-            const int r_end = (kt == nkv - 1 && need_fix) ? U0.kv_end - kt * kPfTok : kPfTok;
-            uint8_t* vb = vsm + st * SM::kTile;
-            uint8_t* vh = vhsm + st * SM::kTile;
-            bool over = false;
-#pragma unroll 4
-            for (int i = lane; i < kPfTok * CH; i += 32) {
-                const int r = i / CH;
-                const uint32_t off = tc_off(r, i % CH, kPfTok);
-                uint4 x = *reinterpret_cast<const uint4*>(vb + off);
-                if (r >= r_end) {
-                    x = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4*>(vb + off) = x;
-                }
-                uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float2 f = unpack2<true>(w[k]);
-                    over |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
-                    w[k] = pack2<false>(f.x, f.y);
-                }
-                *reinterpret_cast<uint4*>(vh + off) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            const bool any_over = __any_sync(kFull, over);
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                vmode[st] = any_over ? 1 : 0;
-                mbar_arrive(bar(kBarVConv + st));
             }
         }
     }
@@ -851,7 +777,7 @@ pkv_status launch_prefill(const PrefillParams& p, const void* query, const void*
         if (e != cudaSuccess) return fail(PKV_ECUDA, "prefill smem opt-in: %s", cudaGetErrorString(e));
         configured.fetch_or(bit);
     }
-    pkv_prefill_kernel<T, D><<<(unsigned)grid, PfSmem<T, D>::kThreads, kSmem, st>>>(p, tq, tk, tv);
+    pkv_prefill_kernel<T, D><<<(unsigned)grid, kPfThreads, kSmem, st>>>(p, tq, tk, tv);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "prefill launch: %s", cudaGetErrorString(e));
     return PKV_OK;

@@ -172,43 +172,6 @@ def test_bad_lengths_and_block_ids_are_flagged():
                           wl.block_tables.cuda(), wl.seq_lens.cuda(), wl.query_start.cuda(), 0.125)
 
 
-def test_bf16_values_past_f16_range_take_the_bf16_path():
-    """bf16 V tiles are read as exact f16 copies (P in one f16 part) unless a
-    value is past f16's range: such tiles' P.V reads the bf16 tile with P as
-    hi + lo parts.  Sequence 0 has one 64-token tile of values up to ~1e5 among
-    ordinary tiles, sequence 1 a few such values among its chunk's own tokens,
-    sequence 2 none.  Rows of sequences 0 and 1 are checked with the tolerance
-    scaled by their largest |V| (the rounding of P then dominates); sequence 2,
-    in the same call, with the plain bound."""
-    wl = W.build_prefill("f16range", [300, 0, 100], [90, 130, 40], 16, 8, 128, 16, torch.bfloat16, seed=24)
-    vc = wl.value_cache.clone()
-    t = torch.arange(64, 128)
-    blk = wl.block_tables[0].long()[t // 16]
-    vc[blk, t % 16] = (vc[blk, t % 16].float() * 3e4).to(torch.bfloat16)
-    wl.value_cache = vc
-    nv = wl.new_value.clone()
-    nv[95:100] = (nv[95:100].float() * 5e4).to(torch.bfloat16)        # tokens of sequence 1's chunk
-    wl.new_value = nv
-    assert float(vc.float().abs().max()) > 65504 and float(nv.float().abs().max()) > 65504
-    out, err, _, _ = gpu_prefill(wl)
-    assert err == 0
-    kc, vc2 = oracle_caches(wl)
-    ref = oracle.paged_prefill(wl.query, kc, vc2, wl.block_tables, wl.seq_lens, wl.query_start, wl.scale)
-    g = out.float().cpu().double().numpy()
-    assert np.isfinite(g).all()
-    qs = wl.query_start.tolist()
-    for s_ in range(3):
-        L = int(wl.seq_lens[s_])
-        tt = torch.arange(L)
-        vmax = float(vc2[wl.block_tables[s_].long()[tt // 16], tt % 16].float().abs().max())
-        rows = slice(qs[s_], qs[s_ + 1])
-        e = np.abs(g[rows] - ref[rows])
-        bound = TOL_16 * max(1.0, vmax) + half_ulp(ref[rows], torch.bfloat16)
-        assert float((e - bound).max()) <= 0.0, (s_, vmax, float(e.max()))
-    assert float(vc2.float().abs().max()) > 65504
-    check(out[qs[2]:qs[3]], ref[qs[2]:qs[3]], torch.bfloat16)
-
-
 @pytest.mark.parametrize("stop_tile", [0, 2])
 def test_bounded_waits_run_out_then_the_context_recovers(stop_tile):
     """A test hook makes every CTA's copy lane stop before K/V tile `stop_tile`
