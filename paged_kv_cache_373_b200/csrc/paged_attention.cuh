@@ -317,7 +317,7 @@ enum class Path { kMma16, kFp8, kF32 };
 // kQH_: q heads one q slot holds (>= the unit's heads, min(g, 8)); a slot per
 // ring stage, since the issue walk may be up to kStages-1 units ahead.
 template <typename KvT, typename QT, int D_, Path P_, int kWarps_, int kStages_, int kTT_ = kTileTokens,
-          int kQH_ = kHeadsPerUnit, bool kQ8_ = false>
+          int kQH_ = kHeadsPerUnit>
 struct Cfg {
     using kv_t = KvT;
     using q_t = QT;
@@ -334,10 +334,6 @@ struct Cfg {
     static constexpr int kTensorTile = kNSub * kSubBytes;
     static constexpr int kStageBytes = 2 * kTensorTile; // K tile + V tile
     static constexpr int kQH = kQH_;
-    // FP8 caches: q.K^T on E4M3 tensor cores (q as E4M3 hi + lo parts, K
-    // codes as stored) instead of converting K to f16
-    static constexpr bool kQ8 = kQ8_;
-    static_assert(!kQ8_ || P_ == Path::kFp8, "E4M3 q.K^T needs an FP8 cache");
     static constexpr int kQSlot = kQH * D * kQBytes;
     static constexpr int kWarpBytes = kStages * (kStageBytes + kQSlot);
     static constexpr int kSmemBytes = kWarps * kWarpBytes + 1024;  // + alignment slack
@@ -469,48 +465,6 @@ struct MmaConsumer {
                 qf[kk][1] = on ? q32[(gid * D + 16 * kk + 2 * tig + 8) / 2] : 0u;
             }
             sl0 = sl1 = scale_log2;
-        } else if constexpr (C::kQ8) {
-            // K stays E4M3 for q.K^T (m16n8k32): q of each head is scaled by a
-            // power of two to below 2^8 and split into E4M3 hi + lo parts (about
-            // 8 significant bits); products accumulate in fp32.  Thread
-            // (gid, tig), k-step kk holds d = 32*tig + 8*kk + {0..3} (first B
-            // register) and + {4..7} (second): the same permutation of the
-            // contraction index as its K fragments.
-            using QT = typename C::q_t;
-            const QT* qh = reinterpret_cast<const QT*>(qs) + gid * D + 32 * tig;
-            float v[32];
-            float amax = 0.f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                v[i] = (gid < nh) ? static_cast<float>(qh[i]) : 0.f;
-                amax = fmaxf(amax, fabsf(v[i]));
-            }
-            amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
-            amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
-            int e = 0;
-            if (amax > 0.f && isfinite(amax)) frexpf(amax, &e);  // amax in [2^(e-1), 2^e)
-            const float sc = ldexpf(1.f, 8 - e);
-#pragma unroll
-            for (int kk = 0; kk < KS / 2; ++kk) {
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const int i0 = 8 * kk + 4 * r;
-                    float x[4], h[4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) x[j] = v[i0 + j] * sc;
-                    const uint16_t h01 = f32x2_to_e4m3x2(x[0], x[1]), h23 = f32x2_to_e4m3x2(x[2], x[3]);
-                    const float2 a01 = unpack2<false>(e4m3x2_to_f16x2(h01)), a23 = unpack2<false>(e4m3x2_to_f16x2(h23));
-                    h[0] = a01.x; h[1] = a01.y; h[2] = a23.x; h[3] = a23.y;
-                    const uint16_t l01 = f32x2_to_e4m3x2(x[0] - h[0], x[1] - h[1]);
-                    const uint16_t l23 = f32x2_to_e4m3x2(x[2] - h[2], x[3] - h[3]);
-                    qf[kk][r] = (uint32_t)h01 | ((uint32_t)h23 << 16);           // hi part
-                    qf[KS / 2 + kk][r] = (uint32_t)l01 | ((uint32_t)l23 << 16);  // lo part
-                }
-            }
-            // an infinite q element makes the head's scores NaN (as exact arithmetic would)
-            const float mine = isfinite(amax) ? ldexpf(kscale * scale_log2, e - 8) : NAN;
-            sl0 = __shfl_sync(kFull, mine, (2 * tig) * 4);
-            sl1 = __shfl_sync(kFull, mine, (2 * tig + 1) * 4);
         } else {
             // q is f16 or bf16; K is converted to f16, so q goes to f16 too,
             // pre-scaled by a power of two per head (exact) to stay in range.
@@ -570,15 +524,6 @@ struct MmaConsumer {
                 const uint4 r1b = *reinterpret_cast<const uint4*>(kt + ko[1] + m * 2048 + 1024);
                 const uint32_t w0[8] = {r0a.x, r0a.y, r0a.z, r0a.w, r0b.x, r0b.y, r0b.z, r0b.w};
                 const uint32_t w1[8] = {r1a.x, r1a.y, r1a.z, r1a.w, r1b.x, r1b.y, r1b.z, r1b.w};
-                if constexpr (C::kQ8) {
-                    // A fragments straight from the codes: k-step kk uses words 2kk, 2kk+1
-#pragma unroll
-                    for (int kk = 0; kk < KS / 2; ++kk) {
-                        const uint32_t a[4] = {w0[2 * kk], w1[2 * kk], w0[2 * kk + 1], w1[2 * kk + 1]};
-                        mma16832_e4m3(kk & 1 ? sb : sa, a, qf[kk][0], qf[kk][1]);
-                        mma16832_e4m3(kk & 1 ? sb : sa, a, qf[KS / 2 + kk][0], qf[KS / 2 + kk][1]);
-                    }
-                } else {
 #pragma unroll
                 for (int kk = 0; kk < KS; ++kk) {
                     uint32_t a[4];
@@ -588,7 +533,6 @@ struct MmaConsumer {
                     a[3] = e4m3x2_to_f16x2((uint16_t)(w1[kk] >> 16));
                     if (kk & 1) mma16816<false>(sb, a, qf[kk][0], qf[kk][1]);
                     else        mma16816<false>(sa, a, qf[kk][0], qf[kk][1]);
-                }
                 }
             }
             // scores S^T[token][head]: (gid, 2tig), (gid, 2tig+1), (gid+8, 2tig), (gid+8, 2tig+1)
