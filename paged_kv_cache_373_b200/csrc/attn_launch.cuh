@@ -29,8 +29,25 @@ pkv_status launch_decode_k(const DecodeLaunchArgs& a, cudaStream_t st) {
     const DecodeParams& p = *a.params;
     SuffixArg<kSuffix> sx{};
     if constexpr (kSuffix) sx = SuffixArg<true>{a.seq_start, a.part_o, a.part_ml};
-    pkv_decode_kernel<C, kSuffix><<<a.grid, C::kWarps * 32, C::kSmemBytes, st>>>(p, sx);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = cudaSuccess;
+    if constexpr (kSuffix) {
+        // the cascade suffix pass: a programmatic dependent of the prefix pass
+        // (it may start on SMs the prefix pass leaves; see WaitPrimaryAtExit)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)a.grid);
+        cfg.blockDim = dim3(C::kWarps * 32);
+        cfg.dynamicSmemBytes = C::kSmemBytes;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, pkv_decode_kernel<C, kSuffix>, p, sx);
+    } else {
+        pkv_decode_kernel<C, kSuffix><<<a.grid, C::kWarps * 32, C::kSmemBytes, st>>>(p, sx);
+    }
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "decode launch: %s", cudaGetErrorString(e));
     // the merge kernel is a programmatic dependent launch: its CTAs start
     // while the decode grid drains, locate their unit from the lengths (which

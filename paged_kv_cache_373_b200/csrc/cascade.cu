@@ -10,6 +10,25 @@ namespace {
 
 constexpr int kMaxSmem = 227 * 1024;
 
+// Launch `kern` as a programmatic dependent of the previous kernel on `st`
+// (the kernel waits for it with griddepcontrol.wait before reading its results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    return e == cudaSuccess ? cudaGetLastError() : e;
+}
+
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct CascadeLayout {
@@ -64,8 +83,7 @@ pkv_status launch_prefix(const DecodeParams& p, const CascadeParams& c, int grid
         if (e != cudaSuccess) return fail(PKV_ECUDA, "prefix smem opt-in: %s", cudaGetErrorString(e));
         configured.fetch_or(bit);
     }
-    pkv_prefix_kernel<C, NT><<<grid, C::kWarps * 32, kSmem, st>>>(p, c);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_dependent(pkv_prefix_kernel<C, NT>, dim3(grid), dim3(C::kWarps * 32), kSmem, st, p, c);
     if (e != cudaSuccess) return fail(PKV_ECUDA, "prefix launch: %s", cudaGetErrorString(e));
     return PKV_OK;
 }
@@ -86,9 +104,8 @@ pkv_status launch_prefix_t(const DecodeParams& p, const CascadeParams& c, int nt
 template <typename QT, int D>
 pkv_status launch_combine(const DecodeParams& p, const CascadeParams& c, int nt, cudaStream_t st) {
     const dim3 grid((unsigned)p.num_seqs, (unsigned)((p.num_heads + 7) / 8));  // a warp per (member, head)
-    if (nt == 2) pkv_cascade_combine_kernel<QT, D, 2><<<grid, 256, 0, st>>>(p, c);
-    else pkv_cascade_combine_kernel<QT, D, 4><<<grid, 256, 0, st>>>(p, c);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = nt == 2 ? launch_dependent(pkv_cascade_combine_kernel<QT, D, 2>, grid, dim3(256), 0, st, p, c)
+                                  : launch_dependent(pkv_cascade_combine_kernel<QT, D, 4>, grid, dim3(256), 0, st, p, c);
     if (e != cudaSuccess) return fail(PKV_ECUDA, "combine launch: %s", cudaGetErrorString(e));
     return PKV_OK;
 }

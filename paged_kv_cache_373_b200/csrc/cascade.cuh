@@ -55,6 +55,9 @@ struct CascadeParams {
 // effective prefix, scattered to its members as their suffix start.
 __global__ void __launch_bounds__(256)
 pkv_cascade_setup_kernel(const DecodeParams p, const CascadeParams c) {
+    // the prefix pass (a programmatic dependent launch) may be scheduled now;
+    // it waits for this grid before reading anything it writes
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ int s_min, s_diff, s_bad;
     const int g = blockIdx.x, tid = threadIdx.x;
     const int cap = p.max_blocks_per_seq * p.block_size;
@@ -261,6 +264,11 @@ struct MmaRowsConsumer {
 template <class C, int NT>
 __global__ void __launch_bounds__(C::kWarps * 32, 1)
 pkv_prefix_kernel(const DecodeParams p, const CascadeParams c) {
+    // launched as a programmatic dependent of the setup pass: its results
+    // (prefix_eff, seq_start, member_info) are complete and visible only after
+    // the wait; then the suffix pass may be scheduled (it reads seq_start)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr int R = 8 * NT;
     constexpr int kQSlot = R * C::kRowBytes;
     extern __shared__ uint8_t smem_raw[];
@@ -411,6 +419,10 @@ __device__ inline int64_t group_tile_base(const Lens<false>& ln, int g) {
 template <typename QT, int D, int NT>
 __global__ void __launch_bounds__(256)
 pkv_cascade_combine_kernel(const DecodeParams p, const CascadeParams c) {
+    // a programmatic dependent of the suffix pass's merge: every partial (the
+    // prefix pass's included, which the suffix pass waited for) is complete
+    // and visible after the wait
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     constexpr int R = 8 * NT;
     constexpr int PER = D / 32;
     const int k = blockIdx.x;  // member slot

@@ -944,9 +944,21 @@ __device__ __forceinline__ void issue_tile(const DecodeParams& p, const Walk<C::
 // ----------------------------------------------------------------------------
 // kSuffix: the cascade suffix pass (per-sequence start tokens, partial
 // output); false compiles the plain decode path without either.
+// The cascade suffix pass is a programmatic dependent of the prefix pass,
+// whose results it does not read: it may run beside the prefix pass's last
+// CTAs, but it completes only after that grid, so that the passes after it
+// see every prefix partial.  Every exit of a suffix CTA waits.
+template <bool kSuffix>
+struct WaitPrimaryAtExit {
+    __device__ ~WaitPrimaryAtExit() {
+        if constexpr (kSuffix) asm volatile("griddepcontrol.wait;" ::: "memory");
+    }
+};
+
 template <class C, bool kSuffix>
 __global__ void __launch_bounds__(C::kWarps * 32, 1)
 pkv_decode_kernel(const DecodeParams p, const SuffixArg<kSuffix> sx) {
+    const WaitPrimaryAtExit<kSuffix> wait_at_exit;
     // let the merge grid (a programmatic dependent launch) be scheduled now:
     // its CTAs locate their units while this grid runs and wait for its
     // completion before reading any partial result
@@ -1031,6 +1043,9 @@ pkv_decode_kernel(const DecodeParams p, const SuffixArg<kSuffix> sx) {
 template <typename QT, int D, int TT, bool kSuffix, int kScanE = kMergeScanPerLane>
 __global__ void __launch_bounds__(256)
 pkv_merge_kernel(const DecodeParams p, int64_t workers, const SuffixArg<kSuffix> sx) {
+    // a following programmatic dependent (the cascade's combine pass) may be
+    // scheduled now; it waits for this grid before reading
+    if constexpr (kSuffix) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t b = blockIdx.x;
     const Lens<kSuffix> ln{p.seq_lens, sx.seq_start, p.num_seqs, p.num_kv_heads * p.nch,
