@@ -317,17 +317,17 @@ pkv_status pkv_paged_prefill(void* out, const void* query, pkv_dtype q_dtype, co
  *   - Limit: if pkv_paged_attention_workspace_bytes(num_seqs, num_heads,
  *     num_kv_heads, head_dim, num_ctas) exceeds PKV_STATIC_WORKSPACE_BYTES the
  *     call returns PKV_EINVAL and launches nothing.
- *   - Set-up: every call looks up the array's device address on the current
- *     device (cudaGetSymbolAddress).  Under lazy module loading (the CUDA
- *     default) the first lookup on a device is what commits the 16 MiB there,
- *     so the FIRST call on each device may allocate and synchronise.  Make one
- *     warm-up call per device, with that device current, before the KV pool
- *     takes the device memory and before any stream capture: a call with
- *     num_seqs = 0 (dtypes, head_dim, block_size, num_blocks and
- *     max_blocks_per_seq valid; pointers may be NULL) does only that set-up
- *     and returns PKV_OK.  Later calls allocate nothing.  Because the address
- *     is looked up each time, a call after cudaDeviceReset uses the new
- *     context's array (and is again a first call).
+ *   - Set-up: the array's device address is looked up (cudaGetSymbolAddress)
+ *     by the first call in each CUDA context and cached per context.  Under
+ *     lazy module loading (the CUDA default) that first lookup is what commits
+ *     the 16 MiB on the device, so the FIRST call on each device may allocate
+ *     and synchronise.  Make one warm-up call per device, with that device
+ *     current, before the KV pool takes the device memory and before any
+ *     stream capture: a call with num_seqs = 0 (dtypes, head_dim, block_size,
+ *     num_blocks and max_blocks_per_seq valid; pointers may be NULL) does only
+ *     that set-up and returns PKV_OK.  Later calls allocate nothing.  A call
+ *     after cudaDeviceReset runs in a new context: it looks the address up
+ *     again (and is again a first call).
  *   - Sharing: every call on a device uses the same array, which keeps the
  *     last call's contents.  Nothing in it has to start at zero (every value
  *     read is written earlier by the same call), but calls that overlap on the

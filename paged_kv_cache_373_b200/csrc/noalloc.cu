@@ -3,12 +3,12 @@
 //
 // The split-merge scratch lives in one file-scope device array of a fixed
 // size (kStaticWorkspaceBytes).  Host code cannot pass the array's name to a
-// kernel (on the host it is only a stand-in symbol), so every call looks up
-// its device address with cudaGetSymbolAddress on the current device and
-// hands that address to the existing decode path.  The lookup is repeated on
-// every call (after the first it is a table lookup that allocates nothing),
-// so an address never outlives the context it belongs to, e.g. across a
-// cudaDeviceReset.
+// kernel (on the host it is only a stand-in symbol), so its device address is
+// looked up with cudaGetSymbolAddress with the device current and handed to
+// the existing decode path.  The address is cached per context (keyed by the
+// context's unique id): a call in a context it has not seen before -- another
+// device, or the same device after a cudaDeviceReset -- looks it up again, so
+// an address never outlives the context it belongs to.
 //
 // With lazy module loading (the CUDA default, CUDA_MODULE_LOADING=LAZY) the
 // array is committed on a device by the first lookup there, i.e. by the first
@@ -23,14 +23,11 @@ constexpr size_t kStaticWorkspaceBytes = (size_t)PKV_STATIC_WORKSPACE_BYTES;
 
 static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
 
-// Device address of the static scratch on the current device; null on failure.
+// Device address of the static scratch in the current context; null on failure.
 void* static_workspace(pkv_status* st) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_workspace);
-    if (e != cudaSuccess || !p) {
-        *st = fail(PKV_ECUDA, "cudaGetSymbolAddress(static workspace): %s", cudaGetErrorString(e));
-        return nullptr;
-    }
+    static SymbolCache cache;
+    void* p = symbol_address(g_static_workspace, &cache);
+    if (!p) *st = fail(PKV_ECUDA, "cudaGetSymbolAddress(static workspace) failed");
     return p;
 }
 

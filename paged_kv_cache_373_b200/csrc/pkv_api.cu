@@ -5,6 +5,9 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <utility>
+
+#include <cudaTypedefs.h>
 
 #include "paged_attention.cuh"
 #include "pkv_internal.h"
@@ -35,12 +38,57 @@ int dtype_bytes(pkv_dtype d) {
     }
 }
 
-int* device_error_word() {
-    // looked up on every call (a table lookup once the module is loaded), so
-    // the address always belongs to the current device's current context
+namespace {
+
+// The current context's unique id (cuCtxGetId, through the runtime's driver
+// entry points); 0 if there is none or the driver cannot tell.
+unsigned long long current_context_id() {
+    static const auto fns = [] {
+        void* get_current = nullptr;
+        void* get_id = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &get_current, 4000, cudaEnableDefault, &q) !=
+                cudaSuccess || q != cudaDriverEntryPointSuccess)
+            get_current = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &get_id, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            get_id = nullptr;
+        return std::make_pair(reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(get_current),
+                              reinterpret_cast<PFN_cuCtxGetId_v12000>(get_id));
+    }();
+    if (!fns.first || !fns.second) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (fns.first(&ctx) != CUDA_SUCCESS || !ctx || fns.second(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+}  // namespace
+
+void* symbol_address(const void* symbol, SymbolCache* cache) {
+    // the lookup is repeated whenever the current context is not the one the
+    // cached address belongs to (another device, or the same device after a
+    // reset), so an address never outlives its context
+    const unsigned long long ctx = current_context_id();
+    if (ctx != 0) {
+        std::lock_guard<std::mutex> lk(cache->mu);
+        for (const auto& e : cache->entries)
+            if (e.first == ctx) return e.second;
+    }
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_pkv_error) != cudaSuccess) return nullptr;
-    return static_cast<int*>(p);
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess || !p) return nullptr;
+    const unsigned long long ctx2 = ctx != 0 ? ctx : current_context_id();  // the lookup may create it
+    if (ctx2 != 0) {
+        std::lock_guard<std::mutex> lk(cache->mu);
+        if (cache->entries.size() >= 64) cache->entries.erase(cache->entries.begin());
+        cache->entries.emplace_back(ctx2, p);
+    }
+    return p;
+}
+
+int* device_error_word() {
+    static SymbolCache cache;
+    return static_cast<int*>(symbol_address(&g_pkv_error, &cache));
 }
 
 static int default_ctas() {

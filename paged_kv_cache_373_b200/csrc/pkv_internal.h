@@ -5,11 +5,24 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+#include <utility>
+#include <vector>
+
 #include "../../include/pkv.h"
 
 namespace pkv {
 
-// Device address of the static error word on the current device (null on failure).
+// Device address of a file-scope __device__ symbol in the current context,
+// cached per context (keyed by cuCtxGetId): the first call in a context does
+// the cudaGetSymbolAddress lookup; null on failure.
+struct SymbolCache {
+    std::mutex mu;
+    std::vector<std::pair<unsigned long long, void*>> entries;
+};
+void* symbol_address(const void* symbol, SymbolCache* cache);
+
+// Device address of the static error word in the current context (null on failure).
 int* device_error_word();
 
 // Record a message for pkv_last_error_message() and return `st`.
