@@ -115,6 +115,11 @@ __device__ __forceinline__ int ntiles_of(int L) { return (L + TT - 1) / TT; }
 template <int E>
 __device__ __forceinline__ void load_run(const int32_t* a, int s0, int n, int (&v)[E]) {
     static_assert(E % 4 == 0, "whole 16-byte loads");
+    if constexpr (E <= 8) {  // the narrow scan: one straight-line path (a short prologue)
+#pragma unroll
+        for (int k = 0; k < E; ++k) v[k] = (s0 + k < n) ? __ldg(a + s0 + k) : 0;
+        return;
+    }
     if (s0 + E <= n && (reinterpret_cast<uintptr_t>(a + s0) & 15) == 0) {
 #pragma unroll
         for (int k = 0; k < E; k += 4) {
@@ -230,15 +235,20 @@ __device__ inline SeqHit find_seq(const LN& ln, int64_t P) {
 // branch, so they all agree on W and on the tile split.  Ranges with start
 // tokens (the cascade suffix pass, whose warps have few tiles each) keep to
 // the narrow scan: its code is a quarter of the size.
+// (The narrow path is marked the likely one, so it can stay one short
+// straight run of code: kernels that are mostly prologue, such as a tiny
+// batch, start cold on instruction fetches.)
 template <int TT, class LN>
 __device__ inline int64_t total_tiles_any(const LN& ln, bool* bad_len = nullptr) {
-    if (LN::kHasStart || ln.S <= 256) return total_tiles<TT, kMergeScanPerLane>(ln, bad_len);
-    return total_tiles<TT, kScanPerLane>(ln, bad_len);
+    if (__builtin_expect(LN::kHasStart || ln.S <= 256, 1)) return total_tiles<TT, kMergeScanPerLane>(ln, bad_len);
+    if constexpr (!LN::kHasStart) return total_tiles<TT, kScanPerLane>(ln, bad_len);
+    return 0;
 }
 template <int TT, class LN>
 __device__ inline SeqHit find_seq_any(const LN& ln, int64_t P) {
-    if (LN::kHasStart || ln.S <= 256) return find_seq<TT, kMergeScanPerLane>(ln, P);
-    return find_seq<TT, kScanPerLane>(ln, P);
+    if (__builtin_expect(LN::kHasStart || ln.S <= 256, 1)) return find_seq<TT, kMergeScanPerLane>(ln, P);
+    if constexpr (!LN::kHasStart) return find_seq<TT, kScanPerLane>(ln, P);
+    return SeqHit{0, 0, 0, 0};
 }
 
 // First attended token of the walk's current sequence: a field only when
