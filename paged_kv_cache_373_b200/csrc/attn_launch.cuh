@@ -12,7 +12,7 @@
 
 namespace pkv {
 
-template <class C, bool kSuffix, int kMergeScanE = kMergeScanPerLane>
+template <class C, bool kSuffix>
 pkv_status launch_decode_k(const DecodeLaunchArgs& a, cudaStream_t st) {
     static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
     static std::atomic<unsigned long long> configured{0};  // bit per device (< 64)
@@ -64,7 +64,7 @@ pkv_status launch_decode_k(const DecodeLaunchArgs& a, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, pkv_merge_kernel<typename C::q_t, C::D, C::kTT, kSuffix, kMergeScanE>, p,
+    e = cudaLaunchKernelEx(&cfg, pkv_merge_kernel<typename C::q_t, C::D, C::kTT, kSuffix>, p,
                            workers, sx);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "merge launch: %s", cudaGetErrorString(e));

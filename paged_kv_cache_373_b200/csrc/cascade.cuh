@@ -287,7 +287,7 @@ pkv_prefix_kernel(const DecodeParams p, const CascadeParams c) {
     const Lens<false> ln{c.prefix_eff, nullptr, c.num_groups, p.num_kv_heads * c.row_chunks, 0x7fffffff};
     const int64_t workers = (int64_t)gridDim.x * C::kWarps;
     const int64_t wid = (int64_t)blockIdx.x * C::kWarps + warp;
-    const int64_t W = total_tiles_any<16>(ln);
+    const int64_t W = total_tiles<16>(ln);
     const int64_t chunk = (W + workers - 1) / workers;
     const int64_t tb = min(W, wid * chunk), te = min(W, tb + chunk);
     if (tb >= te) return;
@@ -438,7 +438,7 @@ pkv_cascade_combine_kernel(const DecodeParams p, const CascadeParams c) {
     const Lens<false> ln{c.prefix_eff, nullptr, c.num_groups, p.num_kv_heads * c.row_chunks, 0x7fffffff};
     const int j = kh * c.row_chunks + rc;                   // unit of the group
     const int nt = ntiles_of<16>(ln.eff(g));
-    const int64_t W = total_tiles<16, kMergeScanPerLane>(ln);
+    const int64_t W = total_tiles<16>(ln);
     const int64_t chunk = (W + c.prefix_workers - 1) / c.prefix_workers;
     const int64_t T0 = group_tile_base(ln, g) + (int64_t)j * nt;
     const int64_t bf = T0 / chunk, bl = (T0 + nt - 1) / chunk;

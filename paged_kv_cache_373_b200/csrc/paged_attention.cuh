@@ -110,34 +110,18 @@ struct Lens {
 template <int TT>
 __device__ __forceinline__ int ntiles_of(int L) { return (L + TT - 1) / TT; }
 
-// Entries [s0, s0 + E) of an int32 array (0 past n): 16-byte loads when the
-// run is whole and aligned, else one load per entry; all in flight together.
+// Entries [s0, s0 + E) of an int32 array (0 past n), all loads in flight together.
 template <int E>
 __device__ __forceinline__ void load_run(const int32_t* a, int s0, int n, int (&v)[E]) {
-    static_assert(E % 4 == 0, "whole 16-byte loads");
-    if constexpr (E <= 8) {  // the narrow scan: one straight-line path (a short prologue)
 #pragma unroll
-        for (int k = 0; k < E; ++k) v[k] = (s0 + k < n) ? __ldg(a + s0 + k) : 0;
-        return;
-    }
-    if (s0 + E <= n && (reinterpret_cast<uintptr_t>(a + s0) & 15) == 0) {
-#pragma unroll
-        for (int k = 0; k < E; k += 4) {
-            const int4 x = __ldg(reinterpret_cast<const int4*>(a + s0 + k));
-            v[k] = x.x; v[k + 1] = x.y; v[k + 2] = x.z; v[k + 3] = x.w;
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < E; ++k) v[k] = (s0 + k < n) ? __ldg(a + s0 + k) : 0;
-    }
+    for (int k = 0; k < E; ++k) v[k] = (s0 + k < n) ? __ldg(a + s0 + k) : 0;
 }
 
-// Sequences per lane in one round of the decode kernel's warp-wide length
-// scans (32 x 32 = 1024 sequences per round: one round of loads for batches
-// up to 1024).  The merge kernel scans 8 per lane: its CTAs are scheduled
-// beside the running decode CTAs, so it keeps to a small register budget.
-constexpr int kScanPerLane = 32;
-constexpr int kMergeScanPerLane = 8;
+// Sequences per lane in one round of the warp-wide length scans (256 per
+// round).  A wider scan (32 per lane, 16-byte loads) was measured: its larger
+// prologue made a cold-started tiny batch 8 us slower (instruction fetches)
+// and it did not speed up a 2048-sequence batch.
+constexpr int kScanPerLane = 8;
 
 // Raw lengths (and starts) of the lane's sequences of the round at s0.
 template <int E, class LN>
@@ -229,28 +213,6 @@ __device__ inline SeqHit find_seq(const LN& ln, int64_t P) {
     return SeqHit{ln.S, base, 0, 0};
 }
 
-// The scans with their width chosen by the batch: 8 lengths per lane (one
-// round, a short prologue) for batches of up to 256 sequences, 32 per lane
-// (4x fewer rounds) for larger ones.  Every warp of a grid takes the same
-// branch, so they all agree on W and on the tile split.  Ranges with start
-// tokens (the cascade suffix pass, whose warps have few tiles each) keep to
-// the narrow scan: its code is a quarter of the size.
-// (The narrow path is marked the likely one, so it can stay one short
-// straight run of code: kernels that are mostly prologue, such as a tiny
-// batch, start cold on instruction fetches.)
-template <int TT, class LN>
-__device__ inline int64_t total_tiles_any(const LN& ln, bool* bad_len = nullptr) {
-    if (__builtin_expect(LN::kHasStart || ln.S <= 256, 1)) return total_tiles<TT, kMergeScanPerLane>(ln, bad_len);
-    if constexpr (!LN::kHasStart) return total_tiles<TT, kScanPerLane>(ln, bad_len);
-    return 0;
-}
-template <int TT, class LN>
-__device__ inline SeqHit find_seq_any(const LN& ln, int64_t P) {
-    if (__builtin_expect(LN::kHasStart || ln.S <= 256, 1)) return find_seq<TT, kMergeScanPerLane>(ln, P);
-    if constexpr (!LN::kHasStart) return find_seq<TT, kScanPerLane>(ln, P);
-    return SeqHit{0, 0, 0, 0};
-}
-
 // First attended token of the walk's current sequence: a field only when
 // ranges may start past token 0.
 template <bool kStart> struct WalkStart { int st; int nst; };
@@ -279,7 +241,7 @@ struct Walk : WalkStart<kStart> {
         s = 0; L = 0; nt = 1; j = 0; i = 0; seg_i0 = 0; nl = 0;
         if constexpr (kStart) { this->st = 0; this->nst = 0; }
         if (done) return;
-        const SeqHit h = find_seq_any<TT>(ln, tb);
+        const SeqHit h = find_seq<TT>(ln, tb);
         s = h.s;
         L = ln.eff_of(h.L, h.st);
         if constexpr (kStart) this->st = ln.first_of(h.st);
@@ -985,7 +947,7 @@ pkv_decode_kernel(const DecodeParams p, const SuffixArg<kSuffix> sx) {
     const int64_t workers = (int64_t)gridDim.x * C::kWarps;
     const int64_t wid = (int64_t)blockIdx.x * C::kWarps + warp;
     bool bad_len = false;
-    const int64_t W = total_tiles_any<C::kTT>(ln, &bad_len);
+    const int64_t W = total_tiles<C::kTT>(ln, &bad_len);
     if (bad_len && wid == 0 && lane == 0) raise_error(p.err, PKV_DEVERR_SEQ_LEN);
     const int64_t chunk = (W + workers - 1) / workers;
     const int64_t tb = min(W, wid * chunk), te = min(W, tb + chunk);
@@ -1050,7 +1012,7 @@ pkv_decode_kernel(const DecodeParams p, const SuffixArg<kSuffix> sx) {
 // row; CTA 0 zeroes the empty sequences.  Partials are folded in worker order, four segments
 // per step (their loads in flight together, M updated once per step).
 // ----------------------------------------------------------------------------
-template <typename QT, int D, int TT, bool kSuffix, int kScanE = kMergeScanPerLane>
+template <typename QT, int D, int TT, bool kSuffix>
 __global__ void __launch_bounds__(256)
 pkv_merge_kernel(const DecodeParams p, int64_t workers, const SuffixArg<kSuffix> sx) {
     // a following programmatic dependent (the cascade's combine pass) may be
@@ -1086,11 +1048,11 @@ pkv_merge_kernel(const DecodeParams p, int64_t workers, const SuffixArg<kSuffix>
     }
     if (b >= workers) return;
     // every warp locates the boundary's unit itself (no block barrier)
-    const int64_t W = total_tiles<TT, kScanE>(ln);
+    const int64_t W = total_tiles<TT>(ln);
     const int64_t chunk = (W + workers - 1) / workers;
     const int64_t P = b * chunk;
     if (P >= W) return;
-    const SeqHit hit = find_seq<TT, kScanE>(ln, P);
+    const SeqHit hit = find_seq<TT>(ln, P);
     const int nt = ntiles_of<TT>(ln.eff_of(hit.L, hit.st));
     const int j = (int)((P - hit.base) / nt);
     const int off = (int)((P - hit.base) % nt);
