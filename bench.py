@@ -463,7 +463,8 @@ def run_ours(args):
                          "traffic": traffic,
                          "traffic_source": None if traffic is None else
                          "profiles/traffic.json: ncu dram__bytes_read.sum + dram__bytes_write.sum of one "
-                         "attention call (decode + merge kernels) on this workload, not measured in this run"},
+                         "attention call (every kernel of the call: decode + merge, or the cascade's setup, "
+                         "prefix, suffix decode, merge and combine) on this workload, not measured in this run"},
             "clocks": clk.summary(),
             "protocol": proto,
             "gpu_launches": launches_per_step * K,
