@@ -213,6 +213,121 @@ __device__ inline SeqHit find_seq(const LN& ln, int64_t P) {
     return SeqHit{ln.S, base, 0, 0};
 }
 
+// ----------------------------------------------------------------------------
+// CTA-cooperative forms of the two scans: the CTA's threads share one pass
+// over the lengths (kScanPerLane sequences per thread and round) instead of
+// every warp walking all of them.  Every thread of the CTA must call them
+// (they synchronise the CTA); blockDim.x is a multiple of 32, at most
+// kScanThreads.
+// ----------------------------------------------------------------------------
+constexpr int kScanThreads = 256;
+struct BlockScanSmem {
+    int64_t ex[kScanThreads];        // per-thread exclusive tile prefix of a round
+    int64_t wsum[kScanThreads / 32]; // per-warp sums
+};
+
+// Exclusive prefix of v over the CTA's threads in thread order; *total is
+// the CTA's sum.  The caller synchronises before the next call.
+__device__ __forceinline__ int64_t block_excl_sum(int64_t v, BlockScanSmem& sm, int64_t* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int64_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int64_t y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) sm.wsum[warp] = incl;
+    __syncthreads();
+    int64_t before = 0, tot = 0;
+    for (int w = 0; w < nw; ++w) {
+        const int64_t x = sm.wsum[w];
+        before += (w < warp) ? x : 0;
+        tot += x;
+    }
+    *total = tot;
+    return before + incl - v;
+}
+
+// CTA-collective total_tiles.
+template <int TT, class LN>
+__device__ inline int64_t block_total_tiles(const LN& ln, BlockScanSmem& sm, bool* bad_len = nullptr) {
+    constexpr int E = kScanPerLane;
+    int64_t part = 0;
+    bool bad = false;
+    for (int r0 = 0; r0 < ln.S; r0 += blockDim.x * E) {
+        const int s0 = r0 + threadIdx.x * E;
+        int v[E], st[E];
+        load_lens<E>(ln, s0, v, st);
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+            if (s0 + k < ln.S) {
+                bad |= (v[k] < 0 || v[k] > ln.cap);
+                part += ntiles_of<TT>(ln.eff_of(v[k], st[k]));
+            }
+        }
+    }
+    int64_t tot;
+    block_excl_sum(part, sm, &tot);
+    const int any_bad = __syncthreads_or(bad);  // also: every thread has read the warp sums
+    if (bad_len) *bad_len = any_bad != 0;
+    return tot * ln.units;
+}
+
+// CTA-collective find_seq: each warp passes its own tile P and gets the
+// sequence whose tiles contain it (s = num_seqs when P is past the last).
+template <int TT, class LN>
+__device__ inline SeqHit block_find_seq(const LN& ln, int64_t P, BlockScanSmem& sm) {
+    constexpr int E = kScanPerLane;
+    static_assert(E <= 32, "one sequence per lane in the final step");
+    const int lane = threadIdx.x & 31;
+    SeqHit hit{ln.S, 0, 0, 0};
+    bool found = false;
+    int64_t base = 0;
+    for (int r0 = 0; r0 < ln.S; r0 += blockDim.x * E) {
+        const int s0 = r0 + threadIdx.x * E;
+        int v[E], st[E];
+        load_lens<E>(ln, s0, v, st);
+        int64_t cnt = 0;
+#pragma unroll
+        for (int k = 0; k < E; ++k)
+            cnt += (s0 + k < ln.S) ? (int64_t)ntiles_of<TT>(ln.eff_of(v[k], st[k])) * ln.units : 0;
+        int64_t tot;
+        sm.ex[threadIdx.x] = base + block_excl_sum(cnt, sm, &tot);
+        __syncthreads();
+        if (!found && P < base + tot) {  // warp-uniform
+            // the last thread t with ex[t] <= P holds tile P (ex does not decrease)
+            int t = 0;
+            for (int c0 = 0; c0 < (int)blockDim.x; c0 += 32) {
+                const unsigned le = __ballot_sync(kFull, sm.ex[c0 + lane] <= P);
+                if (le) t = c0 + 31 - __clz(le);
+                if (le != kFull) break;
+            }
+            // thread t's sequences, one per lane
+            const int s = r0 + t * E + lane;
+            const bool in = lane < E && s < ln.S;
+            const int L = in ? ln.raw_len(s) : 0;
+            const int sst = in ? ln.raw_start(s) : 0;
+            const int64_t w = in ? (int64_t)ntiles_of<TT>(ln.eff_of(L, sst)) * ln.units : 0;
+            int64_t incl = w;
+#pragma unroll
+            for (int o = 1; o < E; o <<= 1) {
+                const int64_t y = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int64_t at = sm.ex[t] + incl - w;
+            const unsigned h = __ballot_sync(kFull, in && at + w > P);
+            const int src = __ffs(h) - 1;  // h != 0: thread t's sequences hold P
+            hit = SeqHit{__shfl_sync(kFull, s, src), __shfl_sync(kFull, at, src), __shfl_sync(kFull, L, src),
+                         __shfl_sync(kFull, sst, src)};
+            found = true;
+        }
+        base += tot;
+        __syncthreads();  // ex and the warp sums are rewritten by the next round
+    }
+    if (!found) hit.base = base;
+    return hit;
+}
+
 // First attended token of the walk's current sequence: a field only when
 // ranges may start past token 0.
 template <bool kStart> struct WalkStart { int st; int nst; };
@@ -234,6 +349,10 @@ struct Walk : WalkStart<kStart> {
         if constexpr (kStart) this->nst = in ? ln.raw_start(s + 1) : 0;
     }
     __device__ void init(const Lens<kStart>& ln, int64_t tb, int64_t te_) {
+        init(ln, tb, te_, tb < te_ ? find_seq<TT>(ln, tb) : SeqHit{ln.S, 0, 0, 0});
+    }
+    // h: the sequence holding tile tb (find_seq or block_find_seq)
+    __device__ void init(const Lens<kStart>& ln, int64_t tb, int64_t te_, const SeqHit& h) {
         te = te_;
         T = tb;
         done = tb >= te_;
@@ -241,7 +360,6 @@ struct Walk : WalkStart<kStart> {
         s = 0; L = 0; nt = 1; j = 0; i = 0; seg_i0 = 0; nl = 0;
         if constexpr (kStart) { this->st = 0; this->nst = 0; }
         if (done) return;
-        const SeqHit h = find_seq<TT>(ln, tb);
         s = h.s;
         L = ln.eff_of(h.L, h.st);
         if constexpr (kStart) this->st = ln.first_of(h.st);
@@ -327,9 +445,10 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
-// Zero rows [valid, 16) of a V tile (NSUB columns of 16 x 128 B).  Used on a
-// sequence's last tile so the unused slots (never written, any bits) cannot
-// reach the tensor-core P.V product.
+// Zero rows [valid, TT) of a V tile (NSUB columns of TT x 128 B).  Used on a
+// sequence's last tile (FP8 decode tiles, the cascade prefix pass) so the
+// unused slots (never written, any bits) cannot reach the tensor-core P.V
+// product; 16-bit decode tiles zero-fill those rows as they load them.
 template <int kNSub, int TT>
 __device__ __forceinline__ void zero_tail_rows(uint8_t* tile, int valid, int lane) {
     constexpr int kSubBytes = TT * 128;
@@ -472,7 +591,11 @@ struct MmaConsumer {
     __device__ void tile(uint8_t* kt, uint8_t* vt, int valid) {
         constexpr int TT = C::kTT, NM = TT / 16;
         const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
-        if (valid < TT) zero_tail_rows<C::kNSub, TT>(vt, valid, lane);
+        // rows >= valid: zero-filled by issue_tile for 16-bit caches; FP8
+        // codes are loaded as stored and zeroed here, so that unused slots
+        // (never written, any bits) cannot reach the P.V product
+        if constexpr (C::kPath == Path::kFp8)
+            if (valid < TT) zero_tail_rows<C::kNSub, TT>(vt, valid, lane);
         const uint32_t kb = smem_u32(kt), vb = smem_u32(vt);
         float x[NM][4];
 #pragma unroll
@@ -824,6 +947,10 @@ struct TablePrefetch {
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+// n = 16 copies the chunk, n = 0 writes 16 zero bytes and reads nothing
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, uint32_t n) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
@@ -846,9 +973,11 @@ struct IssueLane {
     uint32_t so[kP];
     int64_t goff;                          // r0 * row_stride + 16 * cr
     int64_t gstep;                         // kR * row_stride
+    int r0;                                // the lane's row within each instruction's kR rows
     __device__ void init(const DecodeParams& p) {
         const int lane = threadIdx.x & 31;
-        const int cr = lane % C::kChunksPerRow, r0 = lane / C::kChunksPerRow;
+        const int cr = lane % C::kChunksPerRow;
+        r0 = lane / C::kChunksPerRow;
 #pragma unroll
         for (int k = 0; k < kP; ++k) so[k] = sw_off<C::kTT>(k * kR + r0, cr);
         const int64_t row_stride = (int64_t)p.num_kv_heads * C::kRowBytes;  // bytes between tokens
@@ -894,13 +1023,31 @@ __device__ __forceinline__ void issue_tile(const DecodeParams& p, const Walk<C::
     const uint32_t kdst = smem_u32(stg), vdst = smem_u32(stg + C::kTensorTile);
     const uint8_t* kl = p.key_cache + il.goff;
     const uint8_t* vl = p.value_cache + il.goff;
+    // rows of the tile inside the sequence (16-bit caches zero-fill the rest:
+    // measured faster there; the FP8 and fp32 tiles mask or zero them after
+    // the load, which keeps their kernels' code and registers smaller)
+    const int nvalid = C::kPath == Path::kMma16 ? w.L - w.i * C::kTT : C::kTT;
+    if (nvalid >= C::kTT) {
 #pragma unroll
-    for (int it = 0; it < C::kTT / C::kRowsPerInst; ++it) {
-        // rows >= 16 exactly when it * kRowsPerInst >= 16
-        const int64_t off = (it * C::kRowsPerInst >= 16 ? base1 : base0) + it * il.gstep;
-        const uint32_t so = il.so[it % IssueLane<C>::kP] + (it / IssueLane<C>::kP) * 1024;
-        cp_async16(kdst + so, kl + off);
-        cp_async16(vdst + so, vl + off);
+        for (int it = 0; it < C::kTT / C::kRowsPerInst; ++it) {
+            // rows >= 16 exactly when it * kRowsPerInst >= 16
+            const int64_t off = (it * C::kRowsPerInst >= 16 ? base1 : base0) + it * il.gstep;
+            const uint32_t so = il.so[it % IssueLane<C>::kP] + (it / IssueLane<C>::kP) * 1024;
+            cp_async16(kdst + so, kl + off);
+            cp_async16(vdst + so, vl + off);
+        }
+    } else {
+        // the sequence's last, partly filled tile: rows past its end are
+        // zero-filled in shared memory and not read (their addresses stay
+        // inside the block, or the first block of the tile)
+#pragma unroll
+        for (int it = 0; it < C::kTT / C::kRowsPerInst; ++it) {
+            const int64_t off = (it * C::kRowsPerInst >= 16 ? base1 : base0) + it * il.gstep;
+            const uint32_t so = il.so[it % IssueLane<C>::kP] + (it / IssueLane<C>::kP) * 1024;
+            const uint32_t n = it * C::kRowsPerInst + il.r0 < nvalid ? 16u : 0u;
+            cp_async16_zfill(kdst + so, kl + off, n);
+            cp_async16_zfill(vdst + so, vl + off, n);
+        }
     }
     if (w.first()) {
         const int nh = min(kHeadsPerUnit, p.g - kHeadsPerUnit * c);
@@ -927,7 +1074,11 @@ struct WaitPrimaryAtExit {
     }
 };
 
-template <class C, bool kSuffix>
+// kWideScan: the CTA-wide length scans (batches that one round of a warp's
+// scan does not cover); false: each warp scans alone, with no CTA barrier.
+// Two instantiations rather than a branch: with the CTA-wide form compiled
+// in, a cold-started tiny batch measured 4 us slower.
+template <class C, bool kSuffix, bool kWideScan>
 __global__ void __launch_bounds__(C::kWarps * 32, 1)
 pkv_decode_kernel(const DecodeParams p, const SuffixArg<kSuffix> sx) {
     const WaitPrimaryAtExit<kSuffix> wait_at_exit;
@@ -946,15 +1097,28 @@ pkv_decode_kernel(const DecodeParams p, const SuffixArg<kSuffix> sx) {
                            p.max_blocks_per_seq * p.block_size};
     const int64_t workers = (int64_t)gridDim.x * C::kWarps;
     const int64_t wid = (int64_t)blockIdx.x * C::kWarps + warp;
+    // the total and every warp's first tile
     bool bad_len = false;
-    const int64_t W = total_tiles<C::kTT>(ln, &bad_len);
+    int64_t W, tb, te;
+    Walk<C::kTT, kSuffix> iw, cw;  // issue walk (runs kStages-1 tiles ahead) and compute walk
+    if constexpr (!kWideScan) {
+        W = total_tiles<C::kTT>(ln, &bad_len);
+        const int64_t chunk = (W + workers - 1) / workers;
+        tb = min(W, wid * chunk);
+        te = min(W, tb + chunk);
+        if (tb < te) iw.init(ln, tb, te);
+    } else {
+        __shared__ BlockScanSmem scan_sm;  // one pass over the lengths per CTA
+        W = block_total_tiles<C::kTT>(ln, scan_sm, &bad_len);
+        const int64_t chunk = (W + workers - 1) / workers;
+        tb = min(W, wid * chunk);
+        te = min(W, tb + chunk);
+        const SeqHit hit = block_find_seq<C::kTT>(ln, tb, scan_sm);  // every warp takes part
+        if (tb < te) iw.init(ln, tb, te, hit);
+    }
     if (bad_len && wid == 0 && lane == 0) raise_error(p.err, PKV_DEVERR_SEQ_LEN);
-    const int64_t chunk = (W + workers - 1) / workers;
-    const int64_t tb = min(W, wid * chunk), te = min(W, tb + chunk);
     if (tb >= te) return;
 
-    Walk<C::kTT, kSuffix> iw, cw;  // issue walk (runs kStages-1 tiles ahead) and compute walk
-    iw.init(ln, tb, te);
     cw = iw;
     TablePrefetch tp;
     IssueLane<C> il;
@@ -1117,6 +1281,146 @@ pkv_merge_kernel(const DecodeParams p, int64_t workers, const SuffixArg<kSuffix>
     QT* out = reinterpret_cast<QT*>(p.out) + (row0 + h) * D;
 #pragma unroll
     for (int e = 0; e < PER; ++e) out[lane + 32 * e] = from_f32<QT>(ls > 0.f ? o[e] / ls : 0.f);
+}
+
+
+// ----------------------------------------------------------------------------
+// The same merge for large batches, where every CTA of the one-boundary form
+// would repeat a long length scan: CTA c stands for the 8 worker boundaries
+// 8c .. 8c+7 (a warp each) and locates them with one CTA-wide pass over the
+// lengths, while the decode grid still runs for the CTAs resident beside it.
+// After the decode grid completes, the CTA's warps take the owned units'
+// head rows in turn.
+// ----------------------------------------------------------------------------
+constexpr int kMergeWarps = 8;  // boundaries (and warps) per CTA
+
+struct MergeTask {
+    int64_t u;       // unit index (workspace segment base)
+    int64_t row0;    // output row of the unit's first head
+    int64_t bf, bl;  // first and last worker holding a segment of the unit
+    int s;           // its sequence
+};
+
+template <typename QT, int D, int TT, bool kSuffix>
+__global__ void __launch_bounds__(kMergeWarps * 32)
+pkv_merge_wide_kernel(const DecodeParams p, int64_t workers, const SuffixArg<kSuffix> sx) {
+    // a following programmatic dependent (the cascade's combine pass) may be
+    // scheduled now; it waits for this grid before reading
+    if constexpr (kSuffix) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t gw = (int64_t)blockIdx.x * kMergeWarps + warp;
+    const Lens<kSuffix> ln{p.seq_lens, sx.seq_start, p.num_seqs, p.num_kv_heads * p.nch,
+                           p.max_blocks_per_seq * p.block_size};
+    // sequences with nothing to attend (independent of the decode grid): zero
+    // output, or an empty partial (m, l) = (-inf, 0) for a cascade suffix; a
+    // warp per 32 sequences
+    for (int64_t s0 = gw * 32; s0 < p.num_seqs; s0 += (int64_t)gridDim.x * kMergeWarps * 32) {
+        const int sl = (int)s0 + lane;
+        unsigned empty = __ballot_sync(kFull, sl < p.num_seqs && ln.eff(sl) == 0);
+        while (empty) {
+            const int s = (int)s0 + __ffs(empty) - 1;
+            empty &= empty - 1;
+            if constexpr (kSuffix) {
+                if (ln.first(s) > 0) {
+                    for (int i = lane; i < p.num_heads * D; i += 32)
+                        sx.part_o[(int64_t)s * p.num_heads * D + i] = 0.f;
+                    for (int h = lane; h < p.num_heads; h += 32)
+                        sx.part_ml[(int64_t)s * p.num_heads + h] = make_float2(-INFINITY, 0.f);
+                    continue;
+                }
+            }
+            QT* out = reinterpret_cast<QT*>(p.out) + (int64_t)s * p.num_heads * D;
+            for (int i = lane; i < p.num_heads * D; i += 32) out[i] = from_f32<QT>(0.f);
+        }
+    }
+
+    // the CTA's boundaries (every warp takes part in the scans)
+    __shared__ BlockScanSmem scan_sm;
+    __shared__ MergeTask tasks[kMergeWarps];
+    __shared__ int task_nh[kMergeWarps];
+    const int64_t W = block_total_tiles<TT>(ln, scan_sm);
+    const int64_t chunk = (W + workers - 1) / workers;
+    const int64_t b = gw;
+    const int64_t P = (b >= 1 && b < workers) ? min(W, b * chunk) : W;
+    const SeqHit hit = block_find_seq<TT>(ln, P, scan_sm);
+    int nh = 0;
+    if (P < W) {
+        const int nt = ntiles_of<TT>(ln.eff_of(hit.L, hit.st));
+        const int j = (int)((P - hit.base) / nt);
+        const int off = (int)((P - hit.base) % nt);
+        const int64_t T0 = hit.base + (int64_t)j * nt;
+        if (off != 0 && (b - 1) * chunk <= T0) {  // the unit's first interior boundary
+            const int kh = j / p.nch, c = j % p.nch;
+            nh = min(kHeadsPerUnit, p.g - kHeadsPerUnit * c);
+            if (lane == 0) {
+                tasks[warp] = MergeTask{((int64_t)hit.s * p.num_kv_heads + kh) * p.nch + c,
+                                        (int64_t)hit.s * p.num_heads + (int64_t)kh * p.g + kHeadsPerUnit * c,
+                                        T0 / chunk, (T0 + nt - 1) / chunk, hit.s};
+            }
+        }
+    }
+    if (lane == 0) task_nh[warp] = nh;
+    if (!__syncthreads_or(nh > 0)) return;
+    // launched as a programmatic dependent of the decode grid: its partials
+    // are complete and visible only after this point
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    int rows = 0;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) rows += task_nh[w];
+    constexpr int PER = D / 32;
+    constexpr int kBatch = 4;
+    for (int q = warp; q < rows; q += kMergeWarps) {
+        int tw = 0, h = q;
+        while (h >= task_nh[tw]) h -= task_nh[tw++];
+        const MergeTask t = tasks[tw];
+        float M = -INFINITY, ls = 0.f, o[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[e] = 0.f;
+        for (int64_t w0 = t.bf; w0 <= t.bl; w0 += kBatch) {
+            float2 ml[kBatch];
+            float v[kBatch][PER];
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k) {
+                const int64_t w = w0 + k;
+                ml[k] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+                for (int e = 0; e < PER; ++e) v[k][e] = 0.f;
+                if (w <= t.bl) {
+                    ml[k] = p.ws_ml[(w + t.u) * p.hpu + h];
+                    const float* src = p.ws_o + ((w + t.u) * p.hpu + h) * D;
+#pragma unroll
+                    for (int e = 0; e < PER; ++e) v[k][e] = src[lane + 32 * e];
+                }
+            }
+            float Mb = M;
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k) Mb = fmaxf(Mb, ml[k].x);
+            if (Mb == -INFINITY) continue;  // nothing attended yet
+            const float fo = M == -INFINITY ? 0.f : ex2(M - Mb);
+            ls *= fo;
+#pragma unroll
+            for (int e = 0; e < PER; ++e) o[e] *= fo;
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k) {
+                const float f = ml[k].x == -INFINITY ? 0.f : ex2(ml[k].x - Mb);
+                ls += ml[k].y * f;
+#pragma unroll
+                for (int e = 0; e < PER; ++e) o[e] += v[k][e] * f;
+            }
+            M = Mb;
+        }
+        if constexpr (kSuffix) {
+            if (ln.first(t.s) > 0) {  // cascade suffix: keep the partial
+#pragma unroll
+                for (int e = 0; e < PER; ++e) sx.part_o[(t.row0 + h) * D + lane + 32 * e] = o[e];
+                if (lane == 0) sx.part_ml[t.row0 + h] = make_float2(M, ls);
+                continue;
+            }
+        }
+        QT* out = reinterpret_cast<QT*>(p.out) + (t.row0 + h) * D;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) out[lane + 32 * e] = from_f32<QT>(ls > 0.f ? o[e] / ls : 0.f);
+    }
 }
 
 }  // namespace pkv

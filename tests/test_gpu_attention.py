@@ -276,3 +276,21 @@ def test_many_short_sequences():
     assert err3 == 0
     compare(out3, oracle_step(wl0), wl0)
     assert float(out3[3].abs().max()) == 0.0
+
+
+@pytest.mark.parametrize("heads,d,dtype,n", [((32, 32), 128, torch.float16, 700),
+                                             ((64, 8), 64, torch.bfloat16, 1000),
+                                             ((24, 2), 128, torch.bfloat16, 600)])
+def test_large_batches_merge_eight_boundaries_per_cta(heads, d, dtype, n):
+    """Batches above 512 sequences: the merge grid locates 8 worker boundaries
+    per CTA with one CTA-wide length scan (MHA, g = 8 with D = 64, and g = 12,
+    whose units are split into two head chunks), and the decode prologue scans
+    the lengths once per CTA."""
+    gen = torch.Generator().manual_seed(70 + n)
+    lens = torch.randint(0, 120, (n,), generator=gen).tolist()
+    wl = W.build_decode(f"large_batch_{n}", lens, heads[0], heads[1], d, 16, dtype, dtype, seed=71 + n)
+    ref = oracle_step(wl)
+    for num_ctas in (0, 5, 149):
+        out, err, _ = gpu_step(wl, num_ctas=num_ctas)
+        assert err == 0
+        compare(out, ref, wl)

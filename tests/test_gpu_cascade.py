@@ -50,6 +50,17 @@ def test_cascade_dtypes_and_head_groupings(dtype, heads, d):
     compare(out, oracle_step(wl), wl)
 
 
+def test_cascade_with_many_groups():
+    # 640 sequences: the suffix pass's merge takes its 8-boundaries-per-CTA form
+    wl = W.config5(num_prompts=80, samples=8, prefix=40, tail_lo=1, tail_hi=30)
+    for num_ctas in (0, 9):
+        out, plain, err = _cascade_step(wl, num_ctas=num_ctas)
+        assert err == 0
+        ref = oracle_step(wl)
+        compare(out, ref, wl)
+        compare(plain, ref, wl)
+
+
 def test_cascade_full_config5_sampled():
     wl = W.config5()
     out, plain, err = _cascade_step(wl)
