@@ -111,6 +111,9 @@ def recorded_traffic(workload: str):
 
 
 # ---------------------------------------------------------------- clocks
+HOST_GATE_CYCLES = 6_000_000  # about 3 ms of the SM clock
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons.  Started before
     the warm-up (nvidia-smi needs a few hundred ms to start); summary() keeps
@@ -382,6 +385,9 @@ def run_ours(args):
     wall0 = time.time()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    # the GPU first spins ~3 ms (before the start event) while the host
+    # enqueues all K steps, so no host-side pause can fall inside the interval
+    torch.cuda._sleep(HOST_GATE_CYCLES)
     t_start.record(stream)
     ev = timed_steps(K)
     t_end.record(stream)

@@ -210,13 +210,26 @@ def _step_args(wl, g, ws, num_ctas):
     return a
 
 
-@pytest.mark.parametrize("name", ["cfg5_mini", "fp8_g8_bs32_qbf16", "bf16_gqa4_d128"])
+STEP_CASES = {
+    # larger steps: 70 sequences with copy-on-write pairs, 96 GQA sequences
+    "prefix_cow_70": lambda: W.config5(num_prompts=10, samples=7, prefix=100, tail_lo=1, tail_hi=60),
+    "bf16_gqa4_96": lambda: W.build_decode("bf16_gqa4_96", [(i * 37) % 301 for i in range(96)],
+                                           32, 8, 128, 16, torch.bfloat16, torch.bfloat16, seed=36),
+}
+
+
+@pytest.mark.parametrize("name", ["cfg5_mini", "fp8_g8_bs32_qbf16", "bf16_gqa4_d128",
+                                  "prefix_cow_70", "bf16_gqa4_96"])
 def test_decode_step_host_packed_and_unpacked(name):
     """pkv_decode_step_host from host buffers, one copy per input and packed
     (one copy for all inputs), gives the device path's bits."""
-    wl = SMALL[name]()
-    ref, err, g = gpu_step(wl, num_ctas=37)
+    wl = STEP_CASES[name]() if name in STEP_CASES else SMALL[name]()
+    ref, err, _ = gpu_step(wl, num_ctas=37)
     assert err == 0
+    # each step starts from fresh caches: replaying a step's copy-on-write
+    # copies on caches it already advanced would copy source blocks that now
+    # hold other sequences' new tokens
+    g = gpu_inputs(wl)
     ws = pkv.alloc_workspace(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, 37)
     src = dict(q=wl.query, nk=wl.new_key.to(wl.q_dtype), nv=wl.new_value.to(wl.q_dtype),
                slots=wl.slot_mapping, tables=wl.block_tables, lens=wl.seq_lens, pairs=wl.cow_pairs)
@@ -247,7 +260,8 @@ def test_decode_step_host_packed_and_unpacked(name):
         hb[off:off + b.numel()] = b
     db = torch.empty(lay.total, dtype=torch.uint8, device="cuda")
     h_out2 = torch.full_like(wl.query, float("nan")).pin_memory()
-    p = _step_args(wl, g, ws, 37)
+    g2 = gpu_inputs(wl)  # kept alive: the args hold raw pointers
+    p = _step_args(wl, g2, ws, 37)
     p.h_packed, p.d_packed = hb.data_ptr(), db.data_ptr()
     d_out2 = torch.empty_like(ref)
     p.h_out, p.d_out = h_out2.data_ptr(), d_out2.data_ptr()
