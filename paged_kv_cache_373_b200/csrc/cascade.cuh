@@ -178,47 +178,65 @@ struct MmaRowsConsumer {
             }
         }
         uint32_t b0[NT], b1[NT], c0[NT], c1[NT];
-        float al[NT][2];
+        // Row maxima of the tile.  The reference maximum m of a row moves
+        // only when the tile's maximum passes it by more than 2^kLazyLog2
+        // (then every row of the warp is rescaled at once); otherwise P =
+        // 2^(x - m) <= 2^kLazyLog2, exact in the hi + lo parts, and o and l
+        // stay relative to the same m (the (m, l, o) partials and the merge
+        // accept any reference).
+        constexpr float kLazyLog2 = 8.f;
+        float x[NT][4], mx[NT][2];
+        bool grow = false;
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
-            float x0 = s[n][0] * sl, x1 = s[n][1] * sl, x2 = s[n][2] * sl, x3 = s[n][3] * sl;
-            if (gid >= valid) x0 = x1 = -INFINITY;
-            if (gid + 8 >= valid) x2 = x3 = -INFINITY;
-            float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+            x[n][0] = s[n][0] * sl; x[n][1] = s[n][1] * sl; x[n][2] = s[n][2] * sl; x[n][3] = s[n][3] * sl;
+            if (gid >= valid) x[n][0] = x[n][1] = -INFINITY;
+            if (gid + 8 >= valid) x[n][2] = x[n][3] = -INFINITY;
+            float mx0 = fmaxf(x[n][0], x[n][2]), mx1 = fmaxf(x[n][1], x[n][3]);
 #pragma unroll
             for (int o = 4; o < 32; o <<= 1) {
                 mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o));
                 mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, o));
             }
-            const float mn0 = fmaxf(m[n][0], mx0), mn1 = fmaxf(m[n][1], mx1);
-            al[n][0] = ex2(m[n][0] - mn0);
-            al[n][1] = ex2(m[n][1] - mn1);
-            m[n][0] = mn0;
-            m[n][1] = mn1;
-            const float e0 = ex2(x0 - mn0), e1 = ex2(x1 - mn1), e2 = ex2(x2 - mn0), e3 = ex2(x3 - mn1);
+            mx[n][0] = mx0;
+            mx[n][1] = mx1;
+            grow |= mx0 > m[n][0] + kLazyLog2 || mx1 > m[n][1] + kLazyLog2;
+        }
+        if (__any_sync(kFull, grow)) {
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const float mn0 = fmaxf(m[n][0], mx[n][0]), mn1 = fmaxf(m[n][1], mx[n][1]);
+                const float al0 = ex2(m[n][0] - mn0), al1 = ex2(m[n][1] - mn1);
+                m[n][0] = mn0;
+                m[n][1] = mn1;
+                l[n][0] *= al0;
+                l[n][1] *= al1;
+#pragma unroll
+                for (int mi = 0; mi < MT; ++mi) {
+                    acc[mi][n][0] *= al0; acc[mi][n][1] *= al1;
+                    acc[mi][n][2] *= al0; acc[mi][n][3] *= al1;
+                }
+            }
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const float e0 = ex2(x[n][0] - m[n][0]), e1 = ex2(x[n][1] - m[n][1]);
+            const float e2 = ex2(x[n][2] - m[n][0]), e3 = ex2(x[n][3] - m[n][1]);
             const uint32_t X0 = pack2<kOpBf16>(e0, e1), X1 = pack2<kOpBf16>(e2, e3);
             if constexpr (kOpBf16) {  // P as hi + lo bf16 parts (see MmaConsumer)
                 const float2 h0 = unpack2<true>(X0), h1 = unpack2<true>(X1);
                 c0[n] = movm_trans(pack2<true>(e0 - h0.x, e1 - h0.y));
                 c1[n] = movm_trans(pack2<true>(e2 - h1.x, e3 - h1.y));
-                l[n][0] = l[n][0] * al[n][0] + (e0 + e2);
-                l[n][1] = l[n][1] * al[n][1] + (e1 + e3);
+                l[n][0] += e0 + e2;
+                l[n][1] += e1 + e3;
             } else {
                 const float2 p0 = unpack2<false>(X0), p1 = unpack2<false>(X1);
-                l[n][0] = l[n][0] * al[n][0] + p0.x + p1.x;
-                l[n][1] = l[n][1] * al[n][1] + p0.y + p1.y;
+                l[n][0] += p0.x + p1.x;
+                l[n][1] += p0.y + p1.y;
                 c0[n] = c1[n] = 0u;
             }
             b0[n] = movm_trans(X0);
             b1[n] = movm_trans(X1);
-        }
-#pragma unroll
-        for (int mi = 0; mi < MT; ++mi) {
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                acc[mi][n][0] *= al[n][0]; acc[mi][n][1] *= al[n][1];
-                acc[mi][n][2] *= al[n][0]; acc[mi][n][3] *= al[n][1];
-            }
         }
 #pragma unroll
         for (int mi = 0; mi < MT; ++mi) {
