@@ -647,10 +647,24 @@ struct MmaConsumer {
             mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o));
             mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, o));
         }
-        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
-        m0 = mn0;
-        m1 = mn1;
+        // Lazy rescale: a head's reference maximum moves only when the tile's
+        // maximum passes it by more than 2^kLazyLog2 (then the whole warp
+        // rescales o and l at once); otherwise P = 2^(x - m) <= 2^kLazyLog2,
+        // still exact in its 16-bit parts, and o, l stay relative to the same
+        // m (the sinks and the (m, l) merge accept any reference).
+        constexpr float kLazyLog2 = 8.f;
+        if (__any_sync(kFull, mx0 > m0 + kLazyLog2 || mx1 > m1 + kLazyLog2)) {
+            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+            const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
+            m0 = mn0;
+            m1 = mn1;
+            l0 *= al0;
+            l1 *= al1;
+#pragma unroll
+            for (int mi = 0; mi < MT; ++mi) {
+                acc[mi][0] *= al0; acc[mi][1] *= al1; acc[mi][2] *= al0; acc[mi][3] *= al1;
+            }
+        }
         // P goes to the tensor core in the V operand's 16-bit type.  bf16 keeps
         // only 8 significant bits, so for bf16 caches P is carried as
         // hi + lo bf16 parts (two products, ~16 significant bits): the P.V sum
@@ -660,8 +674,8 @@ struct MmaConsumer {
         float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
-            const float e0 = ex2(x[m][0] - mn0), e1 = ex2(x[m][1] - mn1);
-            const float e2 = ex2(x[m][2] - mn0), e3 = ex2(x[m][3] - mn1);
+            const float e0 = ex2(x[m][0] - m0), e1 = ex2(x[m][1] - m1);
+            const float e2 = ex2(x[m][2] - m0), e3 = ex2(x[m][3] - m1);
             const uint32_t X0 = pack2<kOpBf16>(e0, e1);
             const uint32_t X1 = pack2<kOpBf16>(e2, e3);
             if constexpr (kOpBf16) {
@@ -679,12 +693,8 @@ struct MmaConsumer {
             b0[m] = movm_trans(X0);  // P^T as mma B
             b1[m] = movm_trans(X1);
         }
-        l0 = l0 * al0 + ls0;
-        l1 = l1 * al1 + ls1;
-#pragma unroll
-        for (int mi = 0; mi < MT; ++mi) {
-            acc[mi][0] *= al0; acc[mi][1] *= al1; acc[mi][2] *= al0; acc[mi][3] *= al1;
-        }
+        l0 += ls0;
+        l1 += ls1;
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
             if constexpr (!kFp8) {
