@@ -308,3 +308,29 @@ def test_large_batches_merge_eight_boundaries_per_cta(heads, d, dtype, n):
         out, err, _ = gpu_step(wl, num_ctas=num_ctas)
         assert err == 0
         compare(out, ref, wl)
+
+
+def _grow_keys(wl, rate):
+    """Scale each sequence's key at position t by (1 + t * rate): the scores'
+    running maximum keeps growing, past the 2^8 rescale threshold many times."""
+    bs = wl.block_size
+    for s in range(wl.num_seqs):
+        for t in range(int(wl.seq_lens[s]) - 1):      # the cached tokens
+            b = int(wl.block_tables[s, t // bs])
+            wl.key_cache[b, t % bs] = (wl.key_cache[b, t % bs].float() * (1.0 + t * rate)).to(wl.key_cache.dtype)
+    wl.query = (wl.query.float() * 3.0).to(wl.query.dtype)
+
+
+@pytest.mark.parametrize("dtype,heads", [(torch.bfloat16, (32, 8)), (torch.float16, (8, 8))])
+def test_growing_scores_exercise_the_lazy_rescale(dtype, heads):
+    """Scores that grow along each sequence move every head's reference
+    maximum on many tiles (a rescale whenever a tile's maximum passes it by
+    2^8) and leave P just below 2^8 between them; split units merge partials
+    taken against different references."""
+    wl = W.build_decode("grow", [37, 300, 1000, 1500], heads[0], heads[1], 128, 16, dtype, dtype, seed=81)
+    _grow_keys(wl, 1.0 / 64.0)
+    ref = oracle_step(wl)
+    for num_ctas in (0, 3):
+        out, err, _ = gpu_step(wl, num_ctas=num_ctas)
+        assert err == 0
+        compare(out, ref, wl)

@@ -112,3 +112,23 @@ def test_cascade_without_groups_is_plain_decode():
     out, plain, err = _cascade_step(wl, groups=groups)
     assert err == 0
     assert torch.equal(out.view(torch.int16), plain.view(torch.int16))
+
+
+def test_cascade_growing_scores_exercise_the_lazy_rescale():
+    # keys grow along the shared prefix and the tails: the prefix pass's rows
+    # and the suffix pass rescale on many tiles
+    wl = W.config5(num_prompts=2, samples=4, prefix=700, tail_lo=20, tail_hi=300)
+    bs = wl.block_size
+    for s in range(wl.num_seqs):
+        for t in range(int(wl.seq_lens[s]) - 1):
+            b = int(wl.block_tables[s, t // bs])
+            if t < 700 and s % 4 != 0:
+                continue  # shared prefix blocks: scaled once, through the group's first member
+            wl.key_cache[b, t % bs] = (wl.key_cache[b, t % bs].float() * (1.0 + t / 64.0)).to(torch.bfloat16)
+    wl.query = (wl.query.float() * 3.0).to(torch.bfloat16)
+    for num_ctas in (0, 5):
+        out, plain, err = _cascade_step(wl, num_ctas=num_ctas)
+        assert err == 0
+        ref = oracle_step(wl)
+        compare(out, ref, wl)
+        compare(plain, ref, wl)
