@@ -348,8 +348,10 @@ pkv_status pkv_paged_attention_decode_noalloc(void* out, const void* query, pkv_
  * pkv_decode_step_host -- one whole decode step driven from host buffers:
  * copies the step's inputs host -> device, runs copy_blocks (if
  * num_cow_pairs > 0), reshape_and_cache of one new token per sequence and
- * the decode attention, copies the output device -> host and synchronises
- * the stream.  Host buffers should be pinned for asynchronous copies.
+ * the decode attention, copies the output device -> host and waits for the
+ * stream (the calling thread polls cudaStreamQuery until the step is done,
+ * rather than sleeping in cudaStreamSynchronize).  Host buffers should be
+ * pinned for asynchronous copies.
  * The caches stay resident on the device.  Device staging buffers are
  * caller-owned and sized like their host counterparts.
  *
