@@ -3,6 +3,7 @@
 #include <atomic>
 
 #include "cascade.cuh"
+#include "cascade_tc.cuh"
 #include "pkv_internal.h"
 
 namespace pkv {
@@ -101,6 +102,26 @@ pkv_status launch_prefix_t(const DecodeParams& p, const CascadeParams& c, int nt
     return launch_prefix<Cfg<T, T, D, Path::kMma16, prefix_warps(4), kPrefixStages>, 4>(p, c, grid, st);
 }
 
+// The prefix pass on the tensor core (head_dim 128, 32-row units, 16-bit
+// caches, power-of-two blocks of 16 to 64 tokens).
+template <typename T>
+pkv_status launch_prefix_tc(const DecodeParams& p, const CascadeParams& c, int grid, cudaStream_t st) {
+    static_assert(kTcSmem <= kMaxSmem, "tensor-core prefix pass shared memory");
+    static std::atomic<unsigned long long> configured{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(PKV_ECUDA, "cudaGetDevice");
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured.load() & bit)) {
+        const cudaError_t e = cudaFuncSetAttribute(pkv_prefix_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   kTcSmem);
+        if (e != cudaSuccess) return fail(PKV_ECUDA, "prefix smem opt-in: %s", cudaGetErrorString(e));
+        configured.fetch_or(bit);
+    }
+    const cudaError_t e = launch_dependent(pkv_prefix_tc_kernel<T>, dim3(grid), dim3(kTcThreads), kTcSmem, st, p, c);
+    if (e != cudaSuccess) return fail(PKV_ECUDA, "prefix launch: %s", cudaGetErrorString(e));
+    return PKV_OK;
+}
+
 template <typename QT, int D>
 pkv_status launch_combine(const DecodeParams& p, const CascadeParams& c, int nt, cudaStream_t st) {
     const dim3 grid((unsigned)p.num_seqs, (unsigned)((p.num_heads + 7) / 8));  // a warp per (member, head)
@@ -174,7 +195,11 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
     c.row_chunks = L.row_chunks;
     c.pre_seg_o = reinterpret_cast<const float*>(base + L.pre_seg_o);
     c.pre_seg_ml = reinterpret_cast<const float2*>(base + L.pre_seg_ml);
-    c.prefix_workers = (int64_t)grid * prefix_warps(L.nt);
+    // the prefix pass on the tensor core where its shape allows, else on mma.sync
+    const bool tc_prefix = head_dim == kTcD && L.nt == 4 && block_size >= 16 && block_size <= kTcTok / 2 &&
+                           (block_size & (block_size - 1)) == 0;
+    c.prefix_workers = tc_prefix ? (int64_t)grid : (int64_t)grid * prefix_warps(L.nt);
+    c.prefix_tile = tc_prefix ? kTcTok : 16;
 
     cudaError_t e = cudaMemsetAsync(c.seq_start, 0, (size_t)num_seqs * sizeof(int32_t), cs);
     if (e != cudaSuccess) return fail(PKV_ECUDA, "seq_start memset: %s", cudaGetErrorString(e));
@@ -185,7 +210,10 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
     DecodeParams pp = p;  // prefix pass: its own split segments
     pp.ws_o = reinterpret_cast<float*>(base + L.pre_seg_o);
     pp.ws_ml = reinterpret_cast<float2*>(base + L.pre_seg_ml);
-    if (cache_dtype == PKV_F16)
+    if (tc_prefix)
+        st = cache_dtype == PKV_F16 ? launch_prefix_tc<__half>(pp, c, grid, cs)
+                                    : launch_prefix_tc<__nv_bfloat16>(pp, c, grid, cs);
+    else if (cache_dtype == PKV_F16)
         st = head_dim == 64 ? launch_prefix_t<__half, 64>(pp, c, L.nt, grid, cs)
                             : launch_prefix_t<__half, 128>(pp, c, L.nt, grid, cs);
     else

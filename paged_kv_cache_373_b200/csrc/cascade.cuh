@@ -45,7 +45,8 @@ struct CascadeParams {
     float2* suf_ml;              // [S * Hq]
     const float* pre_seg_o;      // prefix pass's split segments: [segments * R * D]
     const float2* pre_seg_ml;    // [segments * R]
-    int64_t prefix_workers;      // warps of the prefix pass (its tile split)
+    int64_t prefix_workers;      // workers of the prefix pass (its tile split): warps, or CTAs
+    int prefix_tile;             // tokens per tile of the prefix pass: 16, or 128 (tensor-core pass)
     int num_groups;
     int rows;                    // R = max_group_size * g (member query rows per kv head)
     int row_chunks;              // ceil(R / (8 * NT))
@@ -413,14 +414,15 @@ pkv_prefix_kernel(const DecodeParams p, const CascadeParams c) {
     cp_async_wait<0>();
 }
 
-// Sum over groups g' < g of the tiles of their units (warp-collective):
-// the index of group g's first tile in the prefix pass's tile sequence.
-__device__ inline int64_t group_tile_base(const Lens<false>& ln, int g) {
+// Sum over groups g' < g of the tiles (tt tokens each) of their units
+// (warp-collective): the index of group g's first tile in the prefix pass's
+// tile sequence (g = the number of groups: the total).
+__device__ inline int64_t group_tile_base(const Lens<false>& ln, int g, int tt) {
     const int lane = threadIdx.x & 31;
     int64_t base = 0;
     for (int g0 = 0; g0 < g; g0 += 32) {
         const int gi = g0 + lane;
-        int64_t t = gi < g ? (int64_t)ntiles_of<16>(ln.eff(gi)) * ln.units : 0;
+        int64_t t = gi < g ? (int64_t)((ln.eff(gi) + tt - 1) / tt) * ln.units : 0;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(kFull, t, o);
         base += t;
@@ -455,10 +457,11 @@ pkv_cascade_combine_kernel(const DecodeParams p, const CascadeParams c) {
     const int rc = row / R, rr = row % R;
     const Lens<false> ln{c.prefix_eff, nullptr, c.num_groups, p.num_kv_heads * c.row_chunks, 0x7fffffff};
     const int j = kh * c.row_chunks + rc;                   // unit of the group
-    const int nt = ntiles_of<16>(ln.eff(g));
-    const int64_t W = total_tiles<16>(ln);
+    const int tt = c.prefix_tile;
+    const int nt = (ln.eff(g) + tt - 1) / tt;
+    const int64_t W = group_tile_base(ln, c.num_groups, tt);
     const int64_t chunk = (W + c.prefix_workers - 1) / c.prefix_workers;
-    const int64_t T0 = group_tile_base(ln, g) + (int64_t)j * nt;
+    const int64_t T0 = group_tile_base(ln, g, tt) + (int64_t)j * nt;
     const int64_t bf = T0 / chunk, bl = (T0 + nt - 1) / chunk;
     const int64_t unit = (int64_t)g * ln.units + j;
 
