@@ -12,7 +12,9 @@
 //   - warps 5-8 gather each K and V tile through the group's block table
 //     (two warps per tile, 64 rows each) with 16-byte cp.async copies
 //     straight into the 128-byte-swizzled operand layout (2-stage rings;
-//     rows past the prefix zero-filled), and warp 5 copies a unit's q rows;
+//     rows past the prefix zero-filled; each lane's copies arrive on the
+//     tile's full barrier as they complete, and the issuing thread fences
+//     them to the tensor core's proxy), and warp 5 copies a unit's q rows;
 //   - warp 4 (one lane) issues S^T of tile n and then O^T += V^T P^T of tile
 //     n-1, so the softmax of one tile runs beside the products of the next;
 //   - warps 0-3 (thread = token for S^T, = head_dim index for O^T) mask and
@@ -155,8 +157,8 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
 
     if (tid == 0) {
         for (int i = 0; i < kTbCount; ++i) {
-            const bool two = (i >= kTbKFull && i < kTbKFull + kTcStages) || (i >= kTbVFull && i < kTbVFull + kTcStages);
-            mbar_init(bar(i), i == kTbP || i == kTbP + 1 ? 128 : (two ? 2 : 1));  // full: two copy warps
+            const bool full = (i >= kTbKFull && i < kTbKFull + kTcStages) || (i >= kTbVFull && i < kTbVFull + kTcStages);
+            mbar_init(bar(i), i == kTbP || i == kTbP + 1 ? 128 : (full ? 64 : 1));  // full: the 64 copy lanes
         }
         abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -189,10 +191,9 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
             // ================= copies: warps 5-6 the two 64-row halves of
             // each K tile (warp 5 also the q rows), warps 7-8 those of each V
             // tile.  16-byte cp.async per (row, chunk) into the 128-byte-
-            // swizzled operand layout, rows past the prefix zero-filled; a
-            // warp releases its half of a tile (proxy fence, then an arrival
-            // on the full barrier) once the half's copies completed, while
-            // the next tile's are in flight.
+            // swizzled operand layout, rows past the prefix zero-filled;
+            // every lane's copies of a tile arrive on its full barrier when
+            // they complete (64 arrivals), so no warp waits for its copies.
             const int lw = warp - kTcLoadWarp0;
             const bool is_k = lw < 2;
             const int half = lw & 1;
@@ -211,12 +212,6 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
             for (int k4 = 0; k4 < 4; ++k4) so[k4] = (uint32_t)((((ch & 7) ^ ((r0 + 2 * k4) & 7)) << 4) + (r0 + 2 * k4) * 128);
             const uint32_t col = (uint32_t)((ch >> 3) * (kTcTok * 128));
             bool ok = true;
-            int issued = 0;
-            auto release = [&](int m) {  // tile m's copies of this warp complete: publish them
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(full0 + (m & (kTcStages - 1))));
-            };
             for (int n = 0; ok && !w.done; ++n) {
                 u.locate(p, c, w.s, w.j);
                 const int st = n & (kTcStages - 1);
@@ -257,12 +252,8 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
                         }
                     }
                 }
-                cp_async_commit();
-                if (n > 0) {
-                    cp_async_wait<1>();
-                    release(n - 1);
-                }
-                issued = n + 1;
+                // each lane's copies arrive on the full barrier as they complete
+                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(full0 + st)) : "memory");
                 if (lw == 0 && w.first()) {
                     // the unit's q rows into q buffer (ord & 1), zero rows past the group
                     const int qb = w.ord & 1;
@@ -301,10 +292,8 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
                 }
                 w.advance(ln);
             }
-            // the last tile's copies (and, on the abort path, every copy in
-            // flight) complete before the warp moves on
+            // every copy in flight completes before the warp moves on
             cp_async_wait<0>();
-            if (ok && issued > 0) release(issued - 1);
             if (!ok) *abort = 1;
         } else if (warp == kTcMmaWarp) {
             // ================= tensor-core issue (one lane)
@@ -323,6 +312,7 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
                 ok = ok && __all_sync(kFull, mbar_wait(bar(kTbP + (m & 1)), (uint32_t)((m >> 1) & 1), abort, lim));
                 ok = ok && __all_sync(kFull, mbar_wait(bar(kTbVFull + st), (uint32_t)((m / kTcStages) & 1), abort, lim));
                 if (!ok) return;
+                fence_async_smem();  // the cp.async-written V tile to the tensor core
                 tc_after_sync();
                 if (lane == 0) {
                     const uint64_t vd = desc_add(dv0, (uint32_t)(st * (kTcTile >> 4)));
@@ -348,6 +338,7 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
                     ok = __all_sync(kFull, mbar_wait(bar(kTbQFull + qb), (uint32_t)((w.ord >> 1) & 1), abort, lim));
                 }
                 if (!ok) break;
+                fence_async_smem();  // the cp.async-written K tile (and q rows) to the tensor core
                 tc_after_sync();
                 if (lane == 0) {
                     const uint64_t kd = desc_add(dk0, (uint32_t)(st * (kTcTile >> 4)));
