@@ -158,7 +158,8 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
     if (tid == 0) {
         for (int i = 0; i < kTbCount; ++i) {
             const bool full = (i >= kTbKFull && i < kTbKFull + kTcStages) || (i >= kTbVFull && i < kTbVFull + kTcStages);
-            mbar_init(bar(i), i == kTbP || i == kTbP + 1 ? 128 : (full ? 64 : 1));  // full: the 64 copy lanes
+            const bool qfull = i == kTbQFull || i == kTbQFull + 1;
+            mbar_init(bar(i), i == kTbP || i == kTbP + 1 ? 128 : full ? 64 : qfull ? 32 : 1);  // copy lanes arrive
         }
         abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -218,6 +219,29 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
                 if (n >= kTcStages)
                     ok = __all_sync(kFull, mbar_wait(bar(empty0 + st), (uint32_t)(((n / kTcStages) & 1) ^ 1), abort, lim));
                 if (!ok) break;
+                if (lw == 0 && w.first()) {
+                    // the unit's q rows into q buffer (ord & 1) first: cp.async
+                    // of the rows' 16-byte chunks (rows past the group
+                    // zero-filled), arriving on the q barrier as they complete
+                    const int qb = w.ord & 1;
+                    if (w.ord >= 2)
+                        ok = __all_sync(kFull, mbar_wait(bar(kTbQEmpty + qb), (uint32_t)(((w.ord - 2) >> 1) & 1), abort, lim));
+                    if (!ok) break;
+                    const uint32_t q = smem_u32(qsm + qb * kTcQ);
+                    constexpr int CPR = kTcD * 2 / 16;  // 16-byte chunks per row
+                    const int row_l = kTcRows * u.rc + lane;  // lane l: the member of row l
+                    const int mem_l = lane < u.nrows ? __ldg(c.grp_members + u.o0 + row_l / p.g) : 0;
+#pragma unroll
+                    for (int k = 0; k < kTcRows * CPR / 32; ++k) {
+                        const int idx = lane + 32 * k, rr = idx / CPR, cc = idx % CPR;
+                        const int sq = __shfl_sync(kFull, mem_l, rr);
+                        const int row2 = kTcRows * u.rc + rr;  // member row within the group
+                        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.q) +
+                            (((int64_t)sq * p.num_heads + (int64_t)u.kh * p.g + row2 % p.g) * kTcD) * 2 + cc * 16;
+                        cp_async16_zfill(q + tc_off(rr, cc, kTcRows), src, rr < u.nrows ? 16u : 0u);
+                    }
+                    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(kTbQFull + qb)) : "memory");
+                }
                 const int tok0 = w.i * kTcTok;
                 const int nblk = (w.L + bs - 1) >> lg_bs;
                 int phys = 0;
@@ -254,42 +278,6 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
                 }
                 // each lane's copies arrive on the full barrier as they complete
                 asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(full0 + st)) : "memory");
-                if (lw == 0 && w.first()) {
-                    // the unit's q rows into q buffer (ord & 1), zero rows past the group
-                    const int qb = w.ord & 1;
-                    if (w.ord >= 2)
-                        ok = __all_sync(kFull, mbar_wait(bar(kTbQEmpty + qb), (uint32_t)(((w.ord - 2) >> 1) & 1), abort, lim));
-                    if (ok) {
-                        // every load in flight together: the rows' member
-                        // ids (one per lane, exchanged by shuffles), then the
-                        // 16 chunks of this lane
-                        uint8_t* q = qsm + qb * kTcQ;
-                        constexpr int CPR = kTcD * 2 / 16;  // 16-byte chunks per row
-                        const int row_l = kTcRows * u.rc + lane;  // lane l: the member of row l
-                        const int mem_l = lane < u.nrows ? __ldg(c.grp_members + u.o0 + row_l / p.g) : 0;
-                        uint4 v[kTcRows * CPR / 32];
-#pragma unroll
-                        for (int k = 0; k < kTcRows * CPR / 32; ++k) {
-                            const int idx = lane + 32 * k, rr = idx / CPR, cc = idx % CPR;
-                            const int sq = __shfl_sync(kFull, mem_l, rr);
-                            v[k] = make_uint4(0, 0, 0, 0);
-                            if (rr < u.nrows) {
-                                const int row2 = kTcRows * u.rc + rr;  // member row within the group
-                                const uint8_t* src = reinterpret_cast<const uint8_t*>(p.q) +
-                                    (((int64_t)sq * p.num_heads + (int64_t)u.kh * p.g + row2 % p.g) * kTcD) * 2 + cc * 16;
-                                v[k] = __ldg(reinterpret_cast<const uint4*>(src));
-                            }
-                        }
-#pragma unroll
-                        for (int k = 0; k < kTcRows * CPR / 32; ++k) {
-                            const int idx = lane + 32 * k, rr = idx / CPR, cc = idx % CPR;
-                            *reinterpret_cast<uint4*>(q + tc_off(rr, cc, kTcRows)) = v[k];
-                        }
-                        fence_async_smem();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(bar(kTbQFull + qb));
-                    }
-                }
                 w.advance(ln);
             }
             // every copy in flight completes before the warp moves on
