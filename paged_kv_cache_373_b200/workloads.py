@@ -237,7 +237,8 @@ def config4(num_seqs: int = 32, lo: int = 16384, hi: int = 32768) -> DecodeWorkl
 
 def config5(num_prompts: int = 16, samples: int = 8, prefix: int = 3000,
             tail_lo: int = 32, tail_hi: int = 512, dtype: torch.dtype = torch.bfloat16,
-            num_heads: int = 32, num_kv_heads: int = 8, head_dim: int = 128) -> DecodeWorkload:
+            num_heads: int = 32, num_kv_heads: int = 8, head_dim: int = 128,
+            block_size: int = 16) -> DecodeWorkload:
     """Shared prompt prefix + copy-on-write of its partially filled last block.
 
     Each prompt's prefix is prefilled once and forked ``samples`` times
@@ -251,7 +252,7 @@ def config5(num_prompts: int = 16, samples: int = 8, prefix: int = 3000,
     that share the copied block take the values the copy brings.  The step
     replays: copy_blocks(cow_pairs) -> reshape_and_cache(new tokens) -> decode.
     """
-    bs, Hq, Hkv, D = 16, num_heads, num_kv_heads, head_dim
+    bs, Hq, Hkv, D = block_size, num_heads, num_kv_heads, head_dim
     gen = torch.Generator().manual_seed(_seed(5))
     tails = torch.randint(tail_lo, tail_hi + 1, (num_prompts, samples), generator=gen)
     pblocks = (prefix + bs - 1) // bs

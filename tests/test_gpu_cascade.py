@@ -61,6 +61,19 @@ def test_cascade_with_many_groups():
         compare(plain, ref, wl)
 
 
+@pytest.mark.parametrize("bs", [32, 64])
+def test_cascade_block_sizes(bs):
+    # 32- and 64-token blocks: a 128-token K/V tile of the prefix pass spans 4
+    # or 2 blocks (2 or 1 per copy warp), and the prefix ends inside a tile
+    wl = W.config5(num_prompts=3, samples=4, prefix=700, tail_lo=5, tail_hi=200, block_size=bs)
+    for num_ctas in (0, 4):
+        out, plain, err = _cascade_step(wl, num_ctas=num_ctas)
+        assert err == 0
+        ref = oracle_step(wl)
+        compare(out, ref, wl)
+        compare(plain, ref, wl)
+
+
 def test_cascade_full_config5_sampled():
     wl = W.config5()
     out, plain, err = _cascade_step(wl)
