@@ -36,7 +36,9 @@ namespace pkv {
 constexpr int kTcTok = 128;            // prefix tokens per K/V tile (M of S^T, K of O^T)
 constexpr int kTcRows = 32;            // member rows per unit (N); missing rows are zero
 constexpr int kTcD = 128;              // head_dim (M of O^T)
-constexpr int kTcStages = 2;           // K and V ring depth
+constexpr int kTcKStages = 2;          // K ring depth (a slot frees when S^T of its tile finishes)
+constexpr int kTcVStages = 2;          // V ring depth (a slot frees only after the tile's O^T product;
+                                       // 3 stages measured no faster)
 constexpr int kTcMmaWarp = 4;
 constexpr int kTcLoadWarp0 = 5;        // warps 5-6: K tile halves (and q rows); 7-8: V tile halves
 constexpr int kTcThreads = 9 * 32;
@@ -48,15 +50,16 @@ constexpr int kTcTmemCols = 128;
 constexpr int kTcTile = kTcTok * kTcD * 2;       // one K or V tile: 32 KB
 constexpr int kTcQ = kTcRows * kTcD * 2;         // one unit's q rows: 8 KB
 constexpr int kTcP = kTcRows * kTcTok * 2;       // one P^T part: 8 KB
-constexpr int kTcSmem = 2 * kTcStages * kTcTile + 2 * kTcQ + 2 * 2 * kTcP + 1024;
+constexpr int kTcSmem = (kTcKStages + kTcVStages) * kTcTile + 2 * kTcQ + 2 * 2 * kTcP + 1024;
+static_assert(kTcSmem <= 227 * 1024, "shared memory budget");
 constexpr uint64_t kTcWaitNs = 200000000ull;     // limit of every wait (0.2 s)
 
 enum : int {
-    kTbKFull = 0,                          // [stage] K tile landed (TMA transaction bytes)
-    kTbVFull = kTbKFull + kTcStages,       // [stage] V tile landed
-    kTbKEmpty = kTbVFull + kTcStages,      // [stage] S^T of the tile finished
-    kTbVEmpty = kTbKEmpty + kTcStages,     // [stage] O^T product of the tile finished
-    kTbQFull = kTbVEmpty + kTcStages,      // [q buffer] a unit's q rows written
+    kTbKFull = 0,                          // [stage] K tile landed (64 copy-lane arrivals)
+    kTbVFull = kTbKFull + kTcKStages,      // [stage] V tile landed
+    kTbKEmpty = kTbVFull + kTcVStages,     // [stage] S^T of the tile finished
+    kTbVEmpty = kTbKEmpty + kTcKStages,    // [stage] O^T product of the tile finished
+    kTbQFull = kTbVEmpty + kTcVStages,     // [q buffer] a unit's q rows written
     kTbQEmpty = kTbQFull + 2,              // [q buffer] the unit's last S^T finished
     kTbS = kTbQEmpty + 2,                  // [S buffer] S^T ready
     kTbP = kTbS + 2,                       // [P buffer] P^T written (128 arrivals)
@@ -143,8 +146,8 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
     extern __shared__ uint8_t tc_raw[];
     uint8_t* sm = tc_raw + ((1024 - (smem_u32(tc_raw) & 1023)) & 1023);  // 1024-byte aligned operands
     uint8_t* ksm = sm;                               // [stage]
-    uint8_t* vsm = ksm + kTcStages * kTcTile;        // [stage]
-    uint8_t* qsm = vsm + kTcStages * kTcTile;        // [q buffer]
+    uint8_t* vsm = ksm + kTcKStages * kTcTile;       // [stage]
+    uint8_t* qsm = vsm + kTcVStages * kTcTile;       // [q buffer]
     uint8_t* psm = qsm + 2 * kTcQ;                   // [P buffer][part]
     __shared__ __align__(8) uint64_t bars[kTbCount];
     __shared__ uint32_t tmem_base;
@@ -157,7 +160,7 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
 
     if (tid == 0) {
         for (int i = 0; i < kTbCount; ++i) {
-            const bool full = (i >= kTbKFull && i < kTbKFull + kTcStages) || (i >= kTbVFull && i < kTbVFull + kTcStages);
+            const bool full = (i >= kTbKFull && i < kTbKFull + kTcKStages) || (i >= kTbVFull && i < kTbVFull + kTcVStages);
             const bool qfull = i == kTbQFull || i == kTbQFull + 1;
             mbar_init(bar(i), i == kTbP || i == kTbP + 1 ? 128 : full ? 64 : qfull ? 32 : 1);  // copy lanes arrive
         }
@@ -201,6 +204,7 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
             const uint8_t* cache = is_k ? p.key_cache : p.value_cache;
             uint8_t* ring = is_k ? ksm : vsm;
             const int full0 = is_k ? kTbKFull : kTbVFull, empty0 = is_k ? kTbKEmpty : kTbVEmpty;
+            const int stages = is_k ? kTcKStages : kTcVStages;
             const int lg_bs = 31 - __clz(p.block_size);
             const int bs = 1 << lg_bs;
             const int bpt = kTcTok >> lg_bs;   // blocks per tile
@@ -215,9 +219,9 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
             bool ok = true;
             for (int n = 0; ok && !w.done; ++n) {
                 u.locate(p, c, w.s, w.j);
-                const int st = n & (kTcStages - 1);
-                if (n >= kTcStages)
-                    ok = __all_sync(kFull, mbar_wait(bar(empty0 + st), (uint32_t)(((n / kTcStages) & 1) ^ 1), abort, lim));
+                const int st = n % stages;
+                if (n >= stages)
+                    ok = __all_sync(kFull, mbar_wait(bar(empty0 + st), (uint32_t)(((n / stages) & 1) ^ 1), abort, lim));
                 if (!ok) break;
                 if (lw == 0 && w.first()) {
                     // the unit's q rows into q buffer (ord & 1) first: cp.async
@@ -296,9 +300,9 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
             int qb = 0;
             // O^T += V^T P^T of tile m (its first tile in this range overwrites)
             auto issue_pv = [&](int m, bool first) {
-                const int st = m & (kTcStages - 1);
+                const int st = m % kTcVStages;
                 ok = ok && __all_sync(kFull, mbar_wait(bar(kTbP + (m & 1)), (uint32_t)((m >> 1) & 1), abort, lim));
-                ok = ok && __all_sync(kFull, mbar_wait(bar(kTbVFull + st), (uint32_t)((m / kTcStages) & 1), abort, lim));
+                ok = ok && __all_sync(kFull, mbar_wait(bar(kTbVFull + st), (uint32_t)((m / kTcVStages) & 1), abort, lim));
                 if (!ok) return;
                 fence_async_smem();  // the cp.async-written V tile to the tensor core
                 tc_after_sync();
@@ -318,8 +322,8 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
             bool prev_first = false;
             int n = 0;
             for (; ok && !w.done; ++n) {
-                const int st = n & (kTcStages - 1);
-                ok = __all_sync(kFull, mbar_wait(bar(kTbKFull + st), (uint32_t)((n / kTcStages) & 1), abort, lim));
+                const int st = n % kTcKStages;
+                ok = __all_sync(kFull, mbar_wait(bar(kTbKFull + st), (uint32_t)((n / kTcKStages) & 1), abort, lim));
                 const bool first = w.first();
                 if (ok && first) {
                     qb = w.ord & 1;

@@ -310,6 +310,32 @@ def test_large_batches_merge_eight_boundaries_per_cta(heads, d, dtype, n):
         compare(out, ref, wl)
 
 
+@pytest.mark.parametrize("name,num_ctas", [("bf16_gqa4_d128", 17), ("fp8_g8_bs32_qbf16", 3),
+                                           ("f32_d128", 5), ("bf16_g16_two_chunks", 1000),
+                                           ("f16_mha_d128", 1)])
+def test_split_units_over_a_garbage_workspace_are_repeatable(name, num_ctas):
+    """The workspace needs no initialisation: filled with 0xFF bytes before
+    every call it changes nothing, and repeated calls give the same bits (the
+    split units' partials are merged in worker order).  Grids of 1000 CTAs
+    split most units many ways; one CTA splits the units its 8 warps share."""
+    wl = SMALL[name]()
+    _, err, g = gpu_step(wl)
+    assert err == 0
+    S, Hq, D = g["q"].shape
+    ws = pkv.alloc_workspace(S, Hq, g["kc"].shape[2], D, num_ctas)
+    outs = []
+    for _ in range(3):
+        ws.fill_(0xFF)
+        out = torch.empty_like(g["q"])
+        pkv.paged_attention_decode(out, g["q"], g["kc"], g["vc"], g["tables"], g["lens"], wl.scale,
+                                   g["ks"], g["vs"], workspace=ws, num_ctas=num_ctas)
+        outs.append(out)
+    assert pkv.get_device_error() == 0
+    compare(outs[0], oracle_step(wl), wl)
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+
+
 def _grow_keys(wl, rate):
     """Scale each sequence's key at position t by (1 + t * rate): the scores'
     running maximum keeps growing, past the 2^8 rescale threshold many times."""

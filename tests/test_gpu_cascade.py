@@ -61,11 +61,12 @@ def test_cascade_with_many_groups():
         compare(plain, ref, wl)
 
 
-@pytest.mark.parametrize("bs", [32, 64])
-def test_cascade_block_sizes(bs):
-    # 32- and 64-token blocks: a 128-token K/V tile of the prefix pass spans 4
-    # or 2 blocks (2 or 1 per copy warp), and the prefix ends inside a tile
-    wl = W.config5(num_prompts=3, samples=4, prefix=700, tail_lo=5, tail_hi=200, block_size=bs)
+@pytest.mark.parametrize("prefix", [700, 1000])
+def test_cascade_block_sizes(prefix):
+    # 32-token blocks: a 128-token K/V tile of the prefix pass spans 4 blocks
+    # (2 per copy warp); the shared run (672 or 992 tokens) ends 32 or 96
+    # tokens into its last tile
+    wl = W.config5(num_prompts=3, samples=4, prefix=prefix, tail_lo=5, tail_hi=200, block_size=32)
     for num_ctas in (0, 4):
         out, plain, err = _cascade_step(wl, num_ctas=num_ctas)
         assert err == 0
