@@ -61,6 +61,7 @@ pkv_status launch_decode_k(const DecodeLaunchArgs& a, cudaStream_t st) {
     const pkv_status ds = p.num_seqs > 32 * kScanPerLane ? launch_decode_grid<C, kSuffix, true>(a, sx, st)
                                                           : launch_decode_grid<C, kSuffix, false>(a, sx, st);
     if (ds != PKV_OK) return ds;
+    if (kSuffix && a.skip_merge) return PKV_OK;  // the cascade's finish pass merges the split units
     cudaError_t e = cudaSuccess;
     // the merge kernel is a programmatic dependent launch: its CTAs start
     // while the decode grid drains, locate their unit from the lengths (which

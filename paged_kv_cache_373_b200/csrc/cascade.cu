@@ -35,7 +35,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 struct CascadeLayout {
     int g, rows, nt, row_chunks;
     size_t dec, pre_seg_o, pre_seg_ml, seq_start, member_info, prefix_eff, suf_o, suf_ml, pre_o, pre_ml,
-        total;
+        seq_grp, total;
 };
 
 bool cascade_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int num_groups,
@@ -66,6 +66,7 @@ bool cascade_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
     const size_t prows = (size_t)num_groups * num_kv_heads * L->rows;
     L->pre_o = off;      off = align256(off + prows * head_dim * sizeof(float));
     L->pre_ml = off;     off = align256(off + prows * sizeof(float2));
+    L->seq_grp = off;    off = align256(off + (size_t)num_seqs * sizeof(int2));
     L->total = off;
     return true;
 }
@@ -128,6 +129,15 @@ pkv_status launch_combine(const DecodeParams& p, const CascadeParams& c, int nt,
     const cudaError_t e = nt == 2 ? launch_dependent(pkv_cascade_combine_kernel<QT, D, 2>, grid, dim3(256), 0, st, p, c)
                                   : launch_dependent(pkv_cascade_combine_kernel<QT, D, 4>, grid, dim3(256), 0, st, p, c);
     if (e != cudaSuccess) return fail(PKV_ECUDA, "combine launch: %s", cudaGetErrorString(e));
+    return PKV_OK;
+}
+
+template <typename QT, int D>
+pkv_status launch_finish(const DecodeParams& p, const CascadeParams& c, int nt, cudaStream_t st) {
+    const dim3 grid((unsigned)p.num_seqs, (unsigned)((p.num_heads + 7) / 8));  // a warp per (sequence, head)
+    const cudaError_t e = nt == 2 ? launch_dependent(pkv_cascade_finish_kernel<QT, D, 2>, grid, dim3(256), 0, st, p, c)
+                                  : launch_dependent(pkv_cascade_finish_kernel<QT, D, 4>, grid, dim3(256), 0, st, p, c);
+    if (e != cudaSuccess) return fail(PKV_ECUDA, "finish launch: %s", cudaGetErrorString(e));
     return PKV_OK;
 }
 
@@ -195,6 +205,8 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
     c.row_chunks = L.row_chunks;
     c.pre_seg_o = reinterpret_cast<const float*>(base + L.pre_seg_o);
     c.pre_seg_ml = reinterpret_cast<const float2*>(base + L.pre_seg_ml);
+    c.seq_grp = reinterpret_cast<int2*>(base + L.seq_grp);
+    c.suffix_workers = (int64_t)grid * kWarps16;
     // the prefix pass on the tensor core where its shape allows, else on mma.sync
     const bool tc_prefix = head_dim == kTcD && L.nt == 4 && block_size >= 16 && block_size <= kTcTok / 2 &&
                            (block_size & (block_size - 1)) == 0;
@@ -221,10 +233,22 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
                             : launch_prefix_t<__nv_bfloat16, 128>(pp, c, L.nt, grid, cs);
     if (st != PKV_OK) return st;
 
-    // suffix pass: members from their shared-prefix end, partial outputs
-    DecodeLaunchArgs sa{&p, grid, true, c.seq_start, c.suf_o, c.suf_ml};
+    // suffix pass: members from their shared-prefix end, partial outputs.
+    // Batches whose length scan takes one round of a warp end with the
+    // finish pass, which merges the suffix pass's split units itself (no
+    // merge kernel between them); larger ones with the merge and combine
+    // passes.
+    const bool direct = num_seqs <= 32 * kScanPerLane;
+    DecodeLaunchArgs sa{&p, grid, true, c.seq_start, c.suf_o, c.suf_ml, direct};
     if ((st = launch(sa, cs)) != PKV_OK) return st;
 
+    if (direct) {
+        if (cache_dtype == PKV_F16)
+            return head_dim == 64 ? launch_finish<__half, 64>(p, c, L.nt, cs)
+                                  : launch_finish<__half, 128>(p, c, L.nt, cs);
+        return head_dim == 64 ? launch_finish<__nv_bfloat16, 64>(p, c, L.nt, cs)
+                              : launch_finish<__nv_bfloat16, 128>(p, c, L.nt, cs);
+    }
     if (cache_dtype == PKV_F16)
         return head_dim == 64 ? launch_combine<__half, 64>(p, c, L.nt, cs)
                               : launch_combine<__half, 128>(p, c, L.nt, cs);

@@ -45,6 +45,8 @@ struct CascadeParams {
     float2* suf_ml;              // [S * Hq]
     const float* pre_seg_o;      // prefix pass's split segments: [segments * R * D]
     const float2* pre_seg_ml;    // [segments * R]
+    int2* seq_grp;               // [S] (group, index in the group) of a sequence with a shared prefix
+    int64_t suffix_workers;      // workers (warps) of the suffix pass's tile split
     int64_t prefix_workers;      // workers of the prefix pass (its tile split): warps, or CTAs
     int prefix_tile;             // tokens per tile of the prefix pass: 16, or 128 (tensor-core pass)
     int num_groups;
@@ -103,7 +105,10 @@ pkv_cascade_setup_kernel(const DecodeParams p, const CascadeParams c) {
     if (tid == 0) c.prefix_eff[g] = eff;
     for (int i = o0 + tid; i < o1; i += blockDim.x) {
         const int s = __ldg(c.grp_members + i);
-        if (eff > 0) c.seq_start[s] = eff;  // eff > 0: every member id is valid
+        if (eff > 0) {  // eff > 0: every member id is valid
+            c.seq_start[s] = eff;
+            c.seq_grp[s] = make_int2(g, i - o0);
+        }
         if (i < p.num_seqs) c.member_info[i] = make_int4(s, g, i - o0, eff > 0);
     }
 }
@@ -441,8 +446,9 @@ __global__ void __launch_bounds__(256)
 pkv_cascade_combine_kernel(const DecodeParams p, const CascadeParams c) {
     // a programmatic dependent of the suffix pass's merge: every partial (the
     // prefix pass's included, which the suffix pass waited for) is complete
-    // and visible after the wait
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // and visible after the wait; before it, only what the setup pass wrote
+    // is read (complete before this grid starts: every pass between waited
+    // for it before releasing its dependent)
     constexpr int R = 8 * NT;
     constexpr int PER = D / 32;
     const int k = blockIdx.x;  // member slot
@@ -489,6 +495,7 @@ pkv_cascade_combine_kernel(const DecodeParams p, const CascadeParams c) {
     // the prefix partial: one whole-unit row, or segments bf..bl; then the
     // suffix partial (index n of the sequence of partials)
     const int n = bf == bl ? 1 : (int)(bl - bf + 1);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int i0 = 0; i0 <= n; i0 += 4) {
         float2 ml[4];
         float v[4][PER];
@@ -520,6 +527,130 @@ pkv_cascade_combine_kernel(const DecodeParams p, const CascadeParams c) {
             }
         }
         fold(ml, v);
+    }
+    QT* out = reinterpret_cast<QT*>(p.out) + ((int64_t)s * p.num_heads + h) * D;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) out[lane + 32 * e] = from_f32<QT>(ls > 0.f ? o[e] / ls : 0.f);
+}
+
+
+// Pass 4 for batches whose length scan takes one round of a warp (the
+// suffix pass then skips its merge kernel): one warp per (sequence s, q head
+// h) folds, in order, the prefix partial of s's row (if s shares a prefix:
+// the prefix kernel's whole-unit row or its split segments) and the suffix
+// pass's partials of s's unit (its whole-unit partial, or the segments of
+// the workers it was split between), with the (m, l) rule of zwxr.cn
+// section 3.3, and writes out.  A sequence without a shared prefix whose
+// unit was whole was written by the suffix pass itself; an empty one gets
+// zeros.  Everything before the dependency wait reads only what the setup
+// pass wrote, which is complete before this grid starts (every pass between
+// waited for it before releasing its dependent).
+template <typename QT, int D, int NT>
+__global__ void __launch_bounds__(256)
+pkv_cascade_finish_kernel(const DecodeParams p, const CascadeParams c) {
+    constexpr int R = 8 * NT;
+    constexpr int PER = D / 32;
+    const int s = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int h = (int)blockIdx.y * 8 + warp;
+    if (h >= p.num_heads) return;
+    const int kh = h / p.g, hg = h % p.g;
+    // the suffix pass's unit of (s, h): its tile range and the workers holding it
+    const Lens<true> lsuf{p.seq_lens, c.seq_start, p.num_seqs, p.num_kv_heads * p.nch,
+                          p.max_blocks_per_seq * p.block_size};
+    int64_t Ws, base;
+    seq_tile_base<kTileTokens>(lsuf, s, &Ws, &base);
+    const int st = lsuf.first(s), eff = lsuf.eff(s);
+    const int cch = hg / kHeadsPerUnit, hh = hg % kHeadsPerUnit;
+    const int nts = ntiles_of<kTileTokens>(eff);
+    const int64_t chunk_s = (Ws + c.suffix_workers - 1) / c.suffix_workers;
+    const int64_t T0s = base + (int64_t)(kh * p.nch + cch) * nts;
+    const int64_t us = ((int64_t)s * p.num_kv_heads + kh) * p.nch + cch;
+    const int64_t sbf = eff > 0 ? T0s / chunk_s : 0, sbl = eff > 0 ? (T0s + nts - 1) / chunk_s : -1;
+    const bool suf_whole = eff > 0 && sbf == sbl;
+    if (st == 0 && suf_whole) return;  // written by the suffix pass
+    const int nsuf = eff == 0 ? 0 : (suf_whole ? 1 : (int)(sbl - sbf + 1));
+    // the prefix partial of the row (sequences with a shared prefix)
+    int npre = 0;
+    int64_t pr = 0, pbf = 0, punit = 0;
+    int rr = 0;
+    if (st > 0) {
+        const int2 gm = c.seq_grp[s];
+        const int g = gm.x, row = gm.y * p.g + hg;
+        const int rc = row / R;
+        rr = row % R;
+        const Lens<false> ln{c.prefix_eff, nullptr, c.num_groups, p.num_kv_heads * c.row_chunks, 0x7fffffff};
+        const int j = kh * c.row_chunks + rc;
+        const int tt = c.prefix_tile;
+        const int nt = (ln.eff(g) + tt - 1) / tt;
+        const int64_t W = group_tile_base(ln, c.num_groups, tt);
+        const int64_t chunk = (W + c.prefix_workers - 1) / c.prefix_workers;
+        const int64_t T0 = group_tile_base(ln, g, tt) + (int64_t)j * nt;
+        pbf = T0 / chunk;
+        const int64_t pbl = (T0 + nt - 1) / chunk;
+        punit = (int64_t)g * ln.units + j;
+        pr = ((int64_t)g * p.num_kv_heads + kh) * c.rows + row;
+        npre = pbf == pbl ? 1 : (int)(pbl - pbf + 1);
+        if (pbf == pbl) pbf = -1;  // the whole-unit row
+    }
+    // the partials are complete and visible after the wait
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    float M = -INFINITY, ls = 0.f, o[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) o[e] = 0.f;
+    const int n = npre + nsuf;
+    for (int i0 = 0; i0 < n; i0 += 4) {
+        float2 ml[4];
+        float v[4][PER];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int i = i0 + q;
+            ml[q] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+            for (int e = 0; e < PER; ++e) v[q][e] = 0.f;
+            const float* src = nullptr;
+            if (i < npre) {
+                if (pbf < 0) {
+                    ml[q] = c.pre_ml[pr];
+                    src = c.pre_o + pr * D;
+                } else {
+                    const int64_t sg = (pbf + i + punit) * R + rr;
+                    ml[q] = c.pre_seg_ml[sg];
+                    src = c.pre_seg_o + sg * D;
+                }
+            } else if (i < n) {
+                if (suf_whole) {
+                    const int64_t sr = (int64_t)s * p.num_heads + h;
+                    ml[q] = c.suf_ml[sr];
+                    src = c.suf_o + sr * D;
+                } else {
+                    const int64_t sg = (sbf + (i - npre) + us) * p.hpu + hh;
+                    ml[q] = p.ws_ml[sg];
+                    src = p.ws_o + sg * D;
+                }
+            }
+            if (src) {
+#pragma unroll
+                for (int e = 0; e < PER; ++e) v[q][e] = src[lane + 32 * e];
+            }
+        }
+        float Mb = M;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) Mb = fmaxf(Mb, ml[q].x);
+        if (Mb == -INFINITY) continue;
+        const float fo = M == -INFINITY ? 0.f : ex2(M - Mb);
+        ls *= fo;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[e] *= fo;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float f = ml[q].x == -INFINITY ? 0.f : ex2(ml[q].x - Mb);
+            ls += ml[q].y * f;
+#pragma unroll
+            for (int e = 0; e < PER; ++e) o[e] += v[q][e] * f;
+        }
+        M = Mb;
     }
     QT* out = reinterpret_cast<QT*>(p.out) + ((int64_t)s * p.num_heads + h) * D;
 #pragma unroll

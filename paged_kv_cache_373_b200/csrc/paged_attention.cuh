@@ -41,6 +41,7 @@ namespace pkv {
 constexpr int kTileTokens = 16;    // tokens per pipeline tile (32 for FP8 caches with 32-token blocks)
 constexpr int kHeadsPerUnit = 8;   // q heads served by one KV read (one mma N tile)
 constexpr int kMaxWarpsPerCta = 12; // workspace is sized for this many workers per CTA
+constexpr int kWarps16 = 8;         // warps (workers) per CTA of the 16-bit-cache decode kernels
 constexpr int kMaxCtas = 1 << 20;   // bound on num_ctas: every worker count (CTAs x warps) fits a grid dimension
 
 struct DecodeParams {
@@ -160,6 +161,35 @@ __device__ inline int64_t total_tiles(const LN& ln, bool* bad_len = nullptr) {
     }
     if (bad_len) *bad_len = __any_sync(kFull, bad);
     return tot * ln.units;
+}
+
+// Warp-collective: the total tiles W (as total_tiles) and the index of
+// sequence s's first tile, in one pass over the lengths.
+template <int TT, int E = kScanPerLane, class LN>
+__device__ inline void seq_tile_base(const LN& ln, int s, int64_t* W, int64_t* base) {
+    const int lane = threadIdx.x & 31;
+    int64_t tot = 0, before = 0;
+    for (int r0 = 0; r0 < ln.S; r0 += 32 * E) {
+        const int s0 = r0 + lane * E;
+        int v[E], st[E];
+        load_lens<E>(ln, s0, v, st);
+        int64_t part = 0, pb = 0;
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+            const int64_t t = (s0 + k < ln.S) ? ntiles_of<TT>(ln.eff_of(v[k], st[k])) : 0;
+            part += t;
+            pb += s0 + k < s ? t : 0;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            part += __shfl_xor_sync(kFull, part, o);
+            pb += __shfl_xor_sync(kFull, pb, o);
+        }
+        tot += part;
+        before += pb;
+    }
+    *W = tot * ln.units;
+    *base = before * ln.units;
 }
 
 struct SeqHit {

@@ -41,6 +41,7 @@ struct DecodeLaunchArgs {
     const int32_t* seq_start = nullptr;  // first attended token per sequence
     float* part_o = nullptr;             // partial outputs of sequences with a start > 0
     float2* part_ml = nullptr;
+    bool skip_merge = false;             // suffix pass: split units left to the cascade's finish pass
 };
 
 using DecodeLauncher = pkv_status (*)(const DecodeLaunchArgs&, cudaStream_t);

@@ -128,6 +128,24 @@ def test_cascade_without_groups_is_plain_decode():
     assert torch.equal(out.view(torch.int16), plain.view(torch.int16))
 
 
+@pytest.mark.parametrize("num_ctas", [0, 3, 11])
+def test_cascade_finish_pass_merges_unshared_and_zeroes_empty_sequences(num_ctas):
+    # groups whose members share no blocks (and request no prefix): every
+    # sequence takes the suffix pass from token 0, and the finish pass must
+    # merge its split units and zero the empty ones -- the same partials, in
+    # the same order, as plain decode's merge, so the bits match it
+    wl = W.build_decode("unshared", [0, 300, 17, 0, 900, 64, 5, 1200], 32, 8, 128, 16, torch.bfloat16,
+                        torch.bfloat16, seed=92)
+    wl.meta.update(prompts=0, samples=1, prefix=0)
+    groups = (torch.tensor([0, 3, 8], dtype=torch.int32), torch.arange(8, dtype=torch.int32),
+              torch.zeros(2, dtype=torch.int32), 5)
+    out, plain, err = _cascade_step(wl, groups=groups, num_ctas=num_ctas)
+    assert err == 0
+    compare(out, oracle_step(wl), wl)
+    assert torch.equal(out, plain)
+    assert float(out[0].abs().max()) == 0.0 and float(out[3].abs().max()) == 0.0
+
+
 def test_cascade_growing_scores_exercise_the_lazy_rescale():
     # keys grow along the shared prefix and the tails: the prefix pass's rows
     # and the suffix pass rescale on many tiles
