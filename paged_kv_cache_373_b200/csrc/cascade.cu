@@ -1,5 +1,6 @@
 // cascade.cu -- host side of pkv_paged_attention_decode_cascade: workspace
 // layout, validation, and the launch sequence of the passes in cascade.cuh.
+#include <algorithm>
 #include <atomic>
 
 #include "cascade.cuh"
@@ -213,10 +214,10 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
     c.prefix_workers = tc_prefix ? (int64_t)grid : (int64_t)grid * prefix_warps(L.nt);
     c.prefix_tile = tc_prefix ? kTcTok : 16;
 
-    cudaError_t e = cudaMemsetAsync(c.seq_start, 0, (size_t)num_seqs * sizeof(int32_t), cs);
-    if (e != cudaSuccess) return fail(PKV_ECUDA, "seq_start memset: %s", cudaGetErrorString(e));
-    pkv_cascade_setup_kernel<<<num_groups, 256, 0, cs>>>(p, c);
-    e = cudaGetLastError();
+    pkv_cascade_zero_kernel<<<(unsigned)std::min(148, (num_seqs + 255) / 256), 256, 0, cs>>>(c.seq_start, num_seqs);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PKV_ECUDA, "zero launch: %s", cudaGetErrorString(e));
+    e = launch_dependent(pkv_cascade_setup_kernel, dim3(num_groups), dim3(256), 0, cs, p, c);
     if (e != cudaSuccess) return fail(PKV_ECUDA, "setup launch: %s", cudaGetErrorString(e));
 
     DecodeParams pp = p;  // prefix pass: its own split segments

@@ -54,7 +54,15 @@ struct CascadeParams {
     int row_chunks;              // ceil(R / (8 * NT))
 };
 
-// Pass 1 (one CTA per group; seq_start zeroed beforehand): the group's
+// Zeroes seq_start ahead of the setup pass, which is its programmatic
+// dependent and waits for it only before its own writes.
+__global__ void __launch_bounds__(256) pkv_cascade_zero_kernel(int32_t* a, int n) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    for (int i = blockIdx.x * 256 + threadIdx.x; i < n; i += gridDim.x * 256) a[i] = 0;
+}
+
+// Pass 1 (one CTA per group; a programmatic dependent of the kernel that
+// zeroes seq_start, waited for only before the writes): the group's
 // effective prefix, scattered to its members as their suffix start.
 __global__ void __launch_bounds__(256)
 pkv_cascade_setup_kernel(const DecodeParams p, const CascadeParams c) {
@@ -102,6 +110,7 @@ pkv_cascade_setup_kernel(const DecodeParams p, const CascadeParams c) {
     __syncthreads();
     int eff = min(nblk, s_diff) * p.block_size;
     if (eff < kPrefixMinTiles * 16) eff = 0;  // too short to be worth a shared pass
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // seq_start zeroed
     if (tid == 0) c.prefix_eff[g] = eff;
     for (int i = o0 + tid; i < o1; i += blockDim.x) {
         const int s = __ldg(c.grp_members + i);
