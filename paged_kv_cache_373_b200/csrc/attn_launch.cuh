@@ -55,7 +55,9 @@ pkv_status launch_decode_k(const DecodeLaunchArgs& a, cudaStream_t st) {
     static_assert(C::kSmemBytes + sizeof(BlockScanSmem) <= 227 * 1024, "shared memory budget");
     const DecodeParams& p = *a.params;
     SuffixArg<kSuffix> sx{};
-    if constexpr (kSuffix) sx = SuffixArg<true>{a.seq_start, a.part_o, a.part_ml};
+    if constexpr (kSuffix)
+        sx = SuffixArg<true>{a.seq_start, a.part_o, a.part_ml, a.prefix_eff, a.cta_ticket, a.num_groups,
+                             a.prefix_units, a.prefix_tile};
     // the length scans: each warp alone while one round of a warp's scan
     // covers the batch, else once per CTA
     const pkv_status ds = p.num_seqs > 32 * kScanPerLane ? launch_decode_grid<C, kSuffix, true>(a, sx, st)

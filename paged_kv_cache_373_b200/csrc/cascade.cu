@@ -59,7 +59,7 @@ bool cascade_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
     L->dec = dec;
     L->pre_seg_o = off;  off = align256(off + segs * rpu * head_dim * sizeof(float));
     L->pre_seg_ml = off; off = align256(off + segs * rpu * sizeof(float2));
-    L->seq_start = off;  off = align256(off + (size_t)num_seqs * sizeof(int32_t));
+    L->seq_start = off;  off = align256(off + (size_t)(num_seqs + 1) * sizeof(int32_t));  // + the suffix CTA ticket
     L->member_info = off; off = align256(off + (size_t)num_seqs * sizeof(int4));
     L->prefix_eff = off; off = align256(off + (size_t)num_groups * sizeof(int32_t));
     L->suf_o = off;      off = align256(off + (size_t)num_seqs * num_heads * head_dim * sizeof(float));
@@ -213,8 +213,14 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
                            (block_size & (block_size - 1)) == 0;
     c.prefix_workers = tc_prefix ? (int64_t)grid : (int64_t)grid * prefix_warps(L.nt);
     c.prefix_tile = tc_prefix ? kTcTok : 16;
+    // The tensor-core prefix pass (one CTA per SM) and the suffix pass of a
+    // finish-pass batch run side by side on disjoint SMs, in proportion to
+    // their tokens; otherwise the suffix pass takes the SMs as the prefix
+    // pass frees them.
+    c.split_grid = tc_prefix && num_seqs <= 32 * kScanPerLane && grid >= 8 ? grid : 0;
 
-    pkv_cascade_zero_kernel<<<(unsigned)std::min(148, (num_seqs + 255) / 256), 256, 0, cs>>>(c.seq_start, num_seqs);
+    // seq_start and, after it, the suffix pass's CTA ticket
+    pkv_cascade_zero_kernel<<<(unsigned)std::min(148, (num_seqs + 256) / 256), 256, 0, cs>>>(c.seq_start, num_seqs + 1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ECUDA, "zero launch: %s", cudaGetErrorString(e));
     e = launch_dependent(pkv_cascade_setup_kernel, dim3(num_groups), dim3(256), 0, cs, p, c);
@@ -241,6 +247,13 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
     // passes.
     const bool direct = num_seqs <= 32 * kScanPerLane;
     DecodeLaunchArgs sa{&p, grid, true, c.seq_start, c.suf_o, c.suf_ml, direct};
+    if (c.split_grid > 0) {
+        sa.prefix_eff = c.prefix_eff;
+        sa.cta_ticket = c.seq_start + num_seqs;
+        sa.num_groups = num_groups;
+        sa.prefix_units = num_kv_heads * L.row_chunks;
+        sa.prefix_tile = kTcTok;
+    }
     if ((st = launch(sa, cs)) != PKV_OK) return st;
 
     if (direct) {

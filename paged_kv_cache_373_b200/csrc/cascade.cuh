@@ -47,6 +47,8 @@ struct CascadeParams {
     const float2* pre_seg_ml;    // [segments * R]
     int2* seq_grp;               // [S] (group, index in the group) of a sequence with a shared prefix
     int64_t suffix_workers;      // workers (warps) of the suffix pass's tile split
+    int split_grid;              // > 0: the prefix and suffix passes side by side on this many SMs
+                                 // (cascade_prefix_ctas; prefix_workers / suffix_workers unused)
     int64_t prefix_workers;      // workers of the prefix pass (its tile split): warps, or CTAs
     int prefix_tile;             // tokens per tile of the prefix pass: 16, or 128 (tensor-core pass)
     int num_groups;
@@ -54,8 +56,9 @@ struct CascadeParams {
     int row_chunks;              // ceil(R / (8 * NT))
 };
 
-// Zeroes seq_start ahead of the setup pass, which is its programmatic
-// dependent and waits for it only before its own writes.
+// Zeroes seq_start (and the suffix pass's CTA ticket after it) ahead of the
+// setup pass, which is its programmatic dependent and waits for it only
+// before its own writes.
 __global__ void __launch_bounds__(256) pkv_cascade_zero_kernel(int32_t* a, int n) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int i = blockIdx.x * 256 + threadIdx.x; i < n; i += gridDim.x * 256) a[i] = 0;
@@ -572,7 +575,17 @@ pkv_cascade_finish_kernel(const DecodeParams p, const CascadeParams c) {
     const int st = lsuf.first(s), eff = lsuf.eff(s);
     const int cch = hg / kHeadsPerUnit, hh = hg % kHeadsPerUnit;
     const int nts = ntiles_of<kTileTokens>(eff);
-    const int64_t chunk_s = (Ws + c.suffix_workers - 1) / c.suffix_workers;
+    const Lens<false> ln{c.prefix_eff, nullptr, c.num_groups, p.num_kv_heads * c.row_chunks, 0x7fffffff};
+    const int tt = c.prefix_tile;
+    const int64_t Wpre = group_tile_base(ln, c.num_groups, tt);
+    // the two passes' worker counts (their tile splits)
+    int64_t suffix_workers = c.suffix_workers, prefix_workers = c.prefix_workers;
+    if (c.split_grid > 0) {
+        const int P = cascade_prefix_ctas(Wpre, tt, Ws, kTileTokens, c.split_grid);
+        prefix_workers = max(1, P);
+        suffix_workers = (int64_t)(c.split_grid - P) * kWarps16;
+    }
+    const int64_t chunk_s = (Ws + suffix_workers - 1) / suffix_workers;
     const int64_t T0s = base + (int64_t)(kh * p.nch + cch) * nts;
     const int64_t us = ((int64_t)s * p.num_kv_heads + kh) * p.nch + cch;
     const int64_t sbf = eff > 0 ? T0s / chunk_s : 0, sbl = eff > 0 ? (T0s + nts - 1) / chunk_s : -1;
@@ -588,12 +601,9 @@ pkv_cascade_finish_kernel(const DecodeParams p, const CascadeParams c) {
         const int g = gm.x, row = gm.y * p.g + hg;
         const int rc = row / R;
         rr = row % R;
-        const Lens<false> ln{c.prefix_eff, nullptr, c.num_groups, p.num_kv_heads * c.row_chunks, 0x7fffffff};
         const int j = kh * c.row_chunks + rc;
-        const int tt = c.prefix_tile;
         const int nt = (ln.eff(g) + tt - 1) / tt;
-        const int64_t W = group_tile_base(ln, c.num_groups, tt);
-        const int64_t chunk = (W + c.prefix_workers - 1) / c.prefix_workers;
+        const int64_t chunk = (Wpre + prefix_workers - 1) / prefix_workers;
         const int64_t T0 = group_tile_base(ln, g, tt) + (int64_t)j * nt;
         pbf = T0 / chunk;
         const int64_t pbl = (T0 + nt - 1) / chunk;

@@ -180,8 +180,15 @@ pkv_prefix_tc_kernel(const DecodeParams p, const CascadeParams c) {
     // every role walks the same tile range: units (group, kv head, row chunk)
     // of ceil(prefix / 128) tiles, laid end to end and cut in equal ranges
     const Lens<false> ln{c.prefix_eff, nullptr, c.num_groups, p.num_kv_heads * c.row_chunks, 0x7fffffff};
-    const int64_t workers = gridDim.x;
+    int64_t workers = gridDim.x;
     const int64_t W = total_tiles<kTcTok>(ln);
+    if (c.split_grid > 0) {
+        // beside the suffix pass: this pass's share of the grid (the CTAs past
+        // it find no tiles; they free their SMs for the suffix pass)
+        const Lens<true> lsuf{p.seq_lens, c.seq_start, p.num_seqs, p.num_kv_heads * p.nch,
+                              p.max_blocks_per_seq * p.block_size};
+        workers = max(1, cascade_prefix_ctas(W, kTcTok, total_tiles<kTileTokens>(lsuf), kTileTokens, gridDim.x));
+    }
     const int64_t chunk = (W + workers - 1) / workers;
     const int64_t tb = min(W, (int64_t)blockIdx.x * chunk), te = min(W, tb + chunk);
     const uint64_t lim = kTcWaitNs;

@@ -76,7 +76,43 @@ template <> struct SuffixArg<true> {
     const int32_t* seq_start;  // [num_seqs]
     float* part_o;             // [num_seqs * num_heads * D]
     float2* part_ml;           // [num_seqs * num_heads]
+    // The passes side by side (prefix_tile > 0): the grid's SMs are split
+    // between the cascade's prefix pass and this one by cascade_prefix_ctas;
+    // the CTAs past this pass's share leave at once.
+    const int32_t* prefix_eff; // [num_groups] shared prefix per group
+    int* cta_ticket;           // zeroed before the pass: its CTAs take worker slots in order of arrival
+    int num_groups;
+    int prefix_units;          // prefix units per group (kv heads x row chunks)
+    int prefix_tile;           // tokens per prefix tile, 0: the passes run one after the other
 };
+
+// The cascade's prefix and suffix passes side by side on disjoint SMs: of a
+// grid of `grid` SMs the prefix pass takes P (its CTAs [0, P)) and the
+// suffix pass the other grid - P (its CTAs [0, grid - P)), in proportion to
+// the time each needs: Wp tiles of tp tokens against Ws tiles of ts (the
+// same K/V bytes per token), a prefix token weighted kPrefixCost /
+// kSuffixCost (an SM of the prefix pass streamed ~31 GB/s beside the suffix
+// pass, one of the suffix pass ~45 GB/s).  Integer arithmetic: every pass
+// computes the same split from the same setup results.  With nothing shared
+// the suffix pass takes the whole grid; otherwise each pass keeps at least
+// one CTA.
+constexpr int kPrefixCost = 3, kSuffixCost = 2;
+__device__ __forceinline__ int cascade_prefix_ctas(int64_t Wp, int tp, int64_t Ws, int ts, int grid) {
+    const int64_t bp = Wp * tp * kPrefixCost, bs = Ws * ts * kSuffixCost;
+    if (bp == 0 || grid < 2) return 0;
+    const int64_t P = (grid * bp + (bp + bs) / 2) / (bp + bs);
+    return (int)min((int64_t)grid - 1, max((int64_t)1, P));
+}
+
+// Warp-collective: tiles of the prefix pass, units * sum_g ceil(eff_g / tp).
+__device__ inline int64_t cascade_prefix_tiles(const int32_t* prefix_eff, int num_groups, int units, int tp) {
+    const int lane = threadIdx.x & 31;
+    int64_t t = 0;
+    for (int g = lane; g < num_groups; g += 32) t += (__ldg(prefix_eff + g) + tp - 1) / tp;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(kFull, t, o);
+    return t * units;
+}
 
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
 
@@ -1135,14 +1171,38 @@ pkv_decode_kernel(const DecodeParams p, const SuffixArg<kSuffix> sx) {
 
     const Lens<kSuffix> ln{p.seq_lens, sx.seq_start, p.num_seqs, p.num_kv_heads * p.nch,
                            p.max_blocks_per_seq * p.block_size};
-    const int64_t workers = (int64_t)gridDim.x * C::kWarps;
-    const int64_t wid = (int64_t)blockIdx.x * C::kWarps + warp;
+    int64_t workers = (int64_t)gridDim.x * C::kWarps;
+    int64_t cta = blockIdx.x;
+    if constexpr (kSuffix) {
+        if (sx.prefix_tile > 0) {
+            // beside the prefix pass the CTAs do not start in index order
+            // (some wait for a prefix CTA's SM): the first to arrive take the
+            // worker slots, so the pass's share runs on the SMs free first
+            __shared__ int slot;
+            if (threadIdx.x == 0) slot = atomicAdd(sx.cta_ticket, 1);
+            __syncthreads();
+            cta = slot;
+        }
+    }
+    const int64_t wid = cta * C::kWarps + warp;
+    // the cascade suffix pass beside the prefix pass: this pass's share of
+    // the grid (the warps past it find no tiles and leave)
+    auto side_by_side = [&](int64_t Wsuf) {
+        if constexpr (kSuffix) {
+            if (sx.prefix_tile > 0) {
+                const int64_t Wp = cascade_prefix_tiles(sx.prefix_eff, sx.num_groups, sx.prefix_units, sx.prefix_tile);
+                workers = (int64_t)(gridDim.x - cascade_prefix_ctas(Wp, sx.prefix_tile, Wsuf, C::kTT, gridDim.x)) *
+                          C::kWarps;
+            }
+        }
+    };
     // the total and every warp's first tile
     bool bad_len = false;
     int64_t W, tb, te;
     Walk<C::kTT, kSuffix> iw, cw;  // issue walk (runs kStages-1 tiles ahead) and compute walk
     if constexpr (!kWideScan) {
         W = total_tiles<C::kTT>(ln, &bad_len);
+        side_by_side(W);
         const int64_t chunk = (W + workers - 1) / workers;
         tb = min(W, wid * chunk);
         te = min(W, tb + chunk);
@@ -1150,6 +1210,7 @@ pkv_decode_kernel(const DecodeParams p, const SuffixArg<kSuffix> sx) {
     } else {
         __shared__ BlockScanSmem scan_sm;  // one pass over the lengths per CTA
         W = block_total_tiles<C::kTT>(ln, scan_sm, &bad_len);
+        side_by_side(W);
         const int64_t chunk = (W + workers - 1) / workers;
         tb = min(W, wid * chunk);
         te = min(W, tb + chunk);

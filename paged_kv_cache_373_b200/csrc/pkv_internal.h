@@ -42,6 +42,10 @@ struct DecodeLaunchArgs {
     float* part_o = nullptr;             // partial outputs of sequences with a start > 0
     float2* part_ml = nullptr;
     bool skip_merge = false;             // suffix pass: split units left to the cascade's finish pass
+    // suffix pass beside the prefix pass (prefix_tile > 0; see SuffixArg)
+    const int32_t* prefix_eff = nullptr;
+    int* cta_ticket = nullptr;
+    int num_groups = 0, prefix_units = 0, prefix_tile = 0;
 };
 
 using DecodeLauncher = pkv_status (*)(const DecodeLaunchArgs&, cudaStream_t);
