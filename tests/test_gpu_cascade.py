@@ -146,6 +146,23 @@ def test_cascade_finish_pass_merges_unshared_and_zeroes_empty_sequences(num_ctas
     assert float(out[0].abs().max()) == 0.0 and float(out[3].abs().max()) == 0.0
 
 
+@pytest.mark.parametrize("num_ctas", [8, 20, 300])
+def test_cascade_side_by_side_split_edges(num_ctas):
+    # the prefix and suffix passes split the grid between them (8 CTAs: the
+    # smallest grid that splits; 300: more CTAs than SMs, so the suffix
+    # pass's arrival tickets outnumber the free SMs); two groups share a
+    # prefix, a third shares nothing
+    wl = W.config5(num_prompts=3, samples=6, prefix=900, tail_lo=10, tail_hi=260)
+    off, mem, pre, mgs = W.cascade_groups(wl)
+    pre = pre.clone()
+    pre[1] = 0  # the second prompt's members: unshared
+    out, plain, err = _cascade_step(wl, groups=(off, mem, pre, mgs), num_ctas=num_ctas)
+    assert err == 0
+    ref = oracle_step(wl)
+    compare(out, ref, wl)
+    compare(plain, ref, wl)
+
+
 def test_cascade_growing_scores_exercise_the_lazy_rescale():
     # keys grow along the shared prefix and the tails: the prefix pass's rows
     # and the suffix pass rescale on many tiles
