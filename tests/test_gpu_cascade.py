@@ -40,9 +40,12 @@ def test_cascade_matches_oracle(shape):
 
 
 @pytest.mark.parametrize("dtype,heads,d", [(torch.float16, (16, 4), 64), (torch.bfloat16, (24, 2), 128),
-                                           (torch.float16, (8, 8), 128), (torch.float32, (8, 2), 64)])
+                                           (torch.float16, (8, 8), 128), (torch.float32, (8, 2), 64),
+                                           (torch.float16, (32, 8), 128)])
 def test_cascade_dtypes_and_head_groupings(dtype, heads, d):
-    # f16 / bf16 with g = 4, 12 (two head chunks) and 1; fp32 takes the plain path
+    # f16 / bf16 with g = 4, 12 (two head chunks) and 1; fp32 takes the plain
+    # path; f16 with head_dim 128 and 20 rows per kv head takes the
+    # tensor-core prefix pass (f16 operands)
     wl = W.config5(num_prompts=3, samples=5, prefix=333, tail_lo=1, tail_hi=70, dtype=dtype,
                    num_heads=heads[0], num_kv_heads=heads[1], head_dim=d)
     out, _, err = _cascade_step(wl)
