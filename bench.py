@@ -447,7 +447,8 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_line(wl, args.ref_budget)
 
-    # copy_blocks, reshape_and_cache, then decode + merge (cascade: setup, prefix, suffix decode + merge, combine)
+    # copy_blocks, reshape_and_cache, then decode + merge (cascade, batches of up to 256 sequences:
+    # zeroing, setup, prefix, suffix decode, finish)
     launches_per_step = (1 if has_pairs else 0) + 1 + (5 if args.cascade else 2)
     if rank == 0:
         line = {
@@ -471,8 +472,9 @@ def run_ours(args):
                          "traffic": traffic,
                          "traffic_source": None if traffic is None else
                          "profiles/traffic.json: ncu dram__bytes_read.sum + dram__bytes_write.sum of one "
-                         "attention call (every kernel of the call: decode + merge, or the cascade's setup, "
-                         "prefix, suffix decode, merge and combine) on this workload, not measured in this run"},
+                         "attention call (every kernel of the call: decode + merge, or the cascade's zeroing, "
+                         "setup, prefix, suffix decode and finish passes) on this workload, not measured in "
+                         "this run"},
             "clocks": clk.summary(),
             "protocol": proto,
             "gpu_launches": launches_per_step * K,
