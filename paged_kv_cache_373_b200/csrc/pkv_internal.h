@@ -37,7 +37,7 @@ struct DecodeParams;  // paged_attention.cuh
 struct DecodeLaunchArgs {
     const DecodeParams* params;
     int grid;            // CTAs of the persistent grid
-    bool suffix = false; // cascade suffix pass: the three fields below are used
+    bool suffix = false; // cascade suffix pass: the fields below are used
     const int32_t* seq_start = nullptr;  // first attended token per sequence
     float* part_o = nullptr;             // partial outputs of sequences with a start > 0
     float2* part_ml = nullptr;
