@@ -166,6 +166,40 @@ def test_cascade_side_by_side_split_edges(num_ctas):
     compare(plain, ref, wl)
 
 
+def test_cascade_replays_in_a_cuda_graph():
+    # the whole call (zeroing, setup, the side-by-side prefix and suffix
+    # passes with their arrival tickets, finish) captured once and replayed:
+    # every replay gives the eager call's bits
+    wl = W.config5(num_prompts=4, samples=8, prefix=1200, tail_lo=10, tail_hi=300)
+    g = gpu_inputs(wl)
+    if g["pairs"].numel():
+        pkv.copy_blocks([g["kc"]], [g["vc"]], g["pairs"])
+    pkv.reshape_and_cache(g["nk"], g["nv"], g["kc"], g["vc"], g["slots"], g["ks"], g["vs"])
+    off, mem, pre, mgs = W.cascade_groups(wl)
+    off, mem, pre = off.cuda(), mem.cuda(), pre.cuda()
+    n = pkv.paged_attention_cascade_workspace_bytes(wl.num_seqs, wl.num_heads, wl.num_kv_heads,
+                                                    wl.head_dim, pre.shape[0], mgs, 0)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    eager = torch.empty_like(g["q"])
+    pkv.paged_attention_decode_cascade(eager, g["q"], g["kc"], g["vc"], g["tables"], g["lens"], off, mem, pre,
+                                       mgs, wl.scale, workspace=ws)
+    torch.cuda.synchronize()
+    out = torch.zeros_like(g["q"])
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        pkv.paged_attention_decode_cascade(out, g["q"], g["kc"], g["vc"], g["tables"], g["lens"], off, mem, pre,
+                                           mgs, wl.scale, workspace=ws)
+    for _ in range(2):
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+    assert pkv.get_device_error() == 0
+    compare(eager, oracle_step(wl), wl)
+
+
 def test_cascade_growing_scores_exercise_the_lazy_rescale():
     # keys grow along the shared prefix and the tails: the prefix pass's rows
     # and the suffix pass rescale on many tiles
