@@ -438,10 +438,12 @@ def run_ours(args):
     traffic = recorded_traffic(wl.name + ("_cascade" if args.cascade else ""))
 
     # ---- end-to-end through the C ABI with host buffers
-    e2e = e2e_leg(pkv, wl, g, ws, args, dev, out_ref=None if args.cascade else out) if not args.no_e2e else None
+    casc = (W.cascade_groups(wl), cws) if args.cascade else None
+    e2e = e2e_leg(pkv, wl, g, ws, args, dev, out_ref=out, cascade=casc) if not args.no_e2e else None
     e2e_pipe = reduce_max(e2e["pipelined_ms"], world, dev) if e2e else None
-    e2e_serial = reduce_max(e2e["serial_ms"], world, dev) if e2e else None
-    e2e_value = min(e2e_pipe, e2e_serial) if e2e else None  # the faster of the two host-driven modes
+    # (the cascade call has no host-step entry point: pipelined mode only)
+    e2e_serial = reduce_max(e2e["serial_ms"], world, dev) if e2e and e2e["serial_ms"] is not None else None
+    e2e_value = None if e2e is None else (e2e_pipe if e2e_serial is None else min(e2e_pipe, e2e_serial))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -480,19 +482,24 @@ def run_ours(args):
             "gpu_launches": launches_per_step * K,
             "e2e": None if e2e is None else {
                 "value": world * wl.num_seqs / (e2e_value / 1000.0), "unit": "seq-steps/s",
-                "mode": "pipelined" if e2e_pipe <= e2e_serial else "serial",
+                "mode": "pipelined" if e2e_serial is None or e2e_pipe <= e2e_serial else "serial",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                 "copies_per_step": e2e["copies"], "output_matches_device_path": e2e["matches_device_path"],
-                "api": "the faster of two host-driven modes, both below; in each, every step copies its "
-                       "packed inputs host -> device and its output device -> host",
+                "api": "the faster of the host-driven modes below (the cascade call: pipelined only, it "
+                       "has no host-step entry point); in each, every step copies its inputs host -> device "
+                       "and its output device -> host",
                 "pipelined": {"value": world * wl.num_seqs / (e2e_pipe / 1000.0),
                               "api": "two steps in flight: one H2D copy of the packed inputs (pinned host "
-                                     "buffer) on the step's copy stream, copy_blocks / reshape_and_cache / "
-                                     "paged_attention_decode on one compute stream, one D2H copy of the "
-                                     "output; step n+1's input copy overlaps step n's kernels"},
-                "serial": {"value": world * wl.num_seqs / (e2e_serial / 1000.0),
-                           "api": "pkv_decode_step_host, packed inputs (one H2D, one D2H, one stream sync "
-                                  "per step, one step at a time)"}},
+                                     "buffer" + (", and one of the group arrays" if args.cascade else "") +
+                                     ") on the step's copy stream, copy_blocks / reshape_and_cache / " +
+                                     ("paged_attention_decode_cascade" if args.cascade else
+                                      "paged_attention_decode") +
+                                     " on one compute stream, one D2H copy of the output; step n+1's input "
+                                     "copy overlaps step n's kernels"},
+                "serial": None if e2e_serial is None else {
+                    "value": world * wl.num_seqs / (e2e_serial / 1000.0),
+                    "api": "pkv_decode_step_host, packed inputs (one H2D, one D2H, one stream sync "
+                           "per step, one step at a time)"}},
             "cpu_baseline": cpu,
         }
         print(json.dumps(line))
@@ -787,7 +794,7 @@ class _OracleAdapter:
         self.ob.free_sequence(sid)
 
 
-def e2e_leg(pkv, wl, g, ws, args, dev, out_ref=None):
+def e2e_leg(pkv, wl, g, ws, args, dev, out_ref=None, cascade=None):
     """decode_step_host with packed inputs: the step's inputs sit in one pinned
     host buffer (laid out by pkv_decode_step_layout) -> one H2D copy ->
     copy_blocks / reshape_and_cache / decode -> one D2H copy of the output ->
@@ -810,6 +817,12 @@ def e2e_leg(pkv, wl, g, ws, args, dev, out_ref=None):
     put(lay.seq_lens, wl.seq_lens)
     if npairs:
         put(lay.cow_pairs, wl.cow_pairs)
+    if cascade is not None:
+        # the cascade call: pipelined mode only, its group arrays copied in every step too
+        pipe = e2e_pipelined(pkv, wl, g, ws, args, dev, lay, hbuf, out_ref, cascade)
+        return {"pipelined_ms": pipe["ms"], "serial_ms": None, "h2d": int(lay.total) + pipe["extra_h2d"],
+                "d2h": wl.query.numel() * wl.query.element_size(), "copies": 3,
+                "matches_device_path": pipe["same"]}
     dbuf = torch.empty(max(lay.total, 16), dtype=torch.uint8, device=dev)
     h_out = torch.empty_like(wl.query).pin_memory()
     d_out = torch.empty_like(g["q"])
@@ -847,7 +860,7 @@ def e2e_leg(pkv, wl, g, ws, args, dev, out_ref=None):
             "matches_device_path": same if pipe["same"] is None else (bool(same) and pipe["same"])}
 
 
-def e2e_pipelined(pkv, wl, g, ws, args, dev, lay, hbuf, out_ref=None):
+def e2e_pipelined(pkv, wl, g, ws, args, dev, lay, hbuf, out_ref=None, cascade=None):
     """The same steps with two in flight: every step still copies its packed
     inputs host -> device (one copy) and its output device -> host (one
     copy), but step n+1's input copy runs on its own copy stream while step
@@ -884,18 +897,36 @@ def e2e_pipelined(pkv, wl, g, ws, args, dev, lay, hbuf, out_ref=None):
             "pairs": view(b, lay.cow_pairs, 2 * npairs, torch.int64, (npairs, 2)) if npairs else None,
         })
 
+    # the cascade call's group arrays (offsets, members, prefix lengths), one
+    # more pinned buffer copied in every step
+    h_grp, d_grps, grp_views, gmax, cws = None, None, None, 0, None
+    if cascade is not None:
+        (goff, gmem, gpre, gmax), cws = cascade
+        h_grp = torch.cat([goff, gmem, gpre]).to(torch.int32).pin_memory()
+        d_grps = [torch.empty_like(h_grp, device=dev) for _ in range(2)]
+        n0, n1 = goff.numel(), gmem.numel()
+        grp_views = [(d[:n0], d[n0:n0 + n1], d[n0 + n1:]) for d in d_grps]
+
     def step(i):
         k = i & 1
         v = views[k]
         with torch.cuda.stream(cps[k]):
             dbufs[k][:lay.total].copy_(hbuf, non_blocking=True)
+            if h_grp is not None:
+                d_grps[k].copy_(h_grp, non_blocking=True)
             ev_in[k].record(cps[k])
         comp.wait_event(ev_in[k])
         if npairs:
             pkv.copy_blocks([g["kc"]], [g["vc"]], v["pairs"], stream=comp)
         pkv.reshape_and_cache(v["nk"], v["nv"], g["kc"], g["vc"], v["slots"], g["ks"], g["vs"], stream=comp)
-        pkv.paged_attention_decode(d_outs[k], v["q"], g["kc"], g["vc"], v["tables"], v["lens"], wl.scale,
-                                   g["ks"], g["vs"], workspace=ws, num_ctas=args.num_ctas, stream=comp)
+        if cascade is not None:
+            go, gm, gp = grp_views[k]
+            pkv.paged_attention_decode_cascade(d_outs[k], v["q"], g["kc"], g["vc"], v["tables"], v["lens"],
+                                               go, gm, gp, gmax, wl.scale, g["ks"], g["vs"], workspace=cws,
+                                               num_ctas=args.num_ctas, stream=comp)
+        else:
+            pkv.paged_attention_decode(d_outs[k], v["q"], g["kc"], g["vc"], v["tables"], v["lens"], wl.scale,
+                                       g["ks"], g["vs"], workspace=ws, num_ctas=args.num_ctas, stream=comp)
         ev_k[k].record(comp)
         cps[k].wait_event(ev_k[k])
         with torch.cuda.stream(cps[k]):
@@ -921,7 +952,8 @@ def e2e_pipelined(pkv, wl, g, ws, args, dev, lay, hbuf, out_ref=None):
     if out_ref is not None:
         ref = out_ref.cpu().view(-1).view(torch.uint8)
         same = all(bool(torch.equal(h.view(-1).view(torch.uint8), ref)) for h in h_outs)
-    return {"ms": e0.elapsed_time(e1) / K, "same": same}
+    return {"ms": e0.elapsed_time(e1) / K, "same": same,
+            "extra_h2d": 0 if h_grp is None else h_grp.numel() * h_grp.element_size()}
 
 
 def main():
